@@ -1,0 +1,447 @@
+"""Benchmark of the FP8 DeepSeekMoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+One step = one whole layer forward (quantize, route, group, gate/up GEMM +
+SwiGLU + requantize, down GEMM, combine) over T tokens of seeded synthetic
+input with V3 shapes (hidden 7168, intermediate 2048, 256 routed + 1 shared
+experts, top-8), weights resident in HBM.  With N > 1 (launched by torchrun)
+every rank runs its own replica of the layer on its own batch: there is no
+data-path collective; timing is the max over ranks.  Rank 0 prints one JSON
+line.
+
+`--impl reference` times the CPU oracle (the slow double-precision reference
+of the same layer) on the host cores, on a bounded sample of the workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = ("prefill", "decode", "skewed")
+METRIC = "MoE-layer tokens/s and grouped FP8 GEMM TFLOP/s (% of B200 FP8 / HBM roofline)"
+KERNELS_PER_STEP = 9  # quantize, router GEMM, top-k, histogram, work lists, scatter, 2 GEMMs, combine
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+GEMM_SOURCES = [os.path.join(ROOT, "sparse_moe_layer_expert_b200", "csrc", f) for f in ("gemm.cu", "common.cuh")]
+
+
+def parse(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", choices=WORKLOADS, default="prefill")
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample-tokens", type=int, default=8)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--tokens", type=int, default=0, help="override T (profiling of smaller cases)")
+    p.add_argument("--experts", type=int, default=0, help="override N_r (profiling of smaller cases)")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------- helpers
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity when world == 1)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def workload_shape(name: str, args=None) -> dict:
+    import moe_synth as S
+    cfg = dict(S.CONFIGS[name])
+    if args is not None and args.tokens:
+        cfg["T"] = args.tokens
+    if args is not None and args.experts:
+        cfg["Nr"] = args.experts
+        if cfg.get("n_groups"):
+            cfg["n_groups"] = min(cfg["n_groups"], args.experts)
+            cfg["topk_groups"] = min(cfg["topk_groups"], cfg["n_groups"])
+    return cfg
+
+
+def algorithmic_counts(cfg: dict, T: int, touched_routed: int) -> dict:
+    """Algorithmic bytes and FLOPs of the two grouped GEMMs for one call.
+    Weight bytes count every expert that receives at least one row once (the
+    shared expert always); activation bytes count each (token, expert) row of
+    FP8 input plus its scales once, outputs once."""
+    H, I, Kr, Ns = cfg["H"], cfg["I"], cfg["Kr"], cfg.get("Ns", 1)
+    rows = T * Kr + T * Ns
+    E_t = touched_routed + Ns
+    w13 = 2 * I * H + (2 * I // 128) * (H // 128) * 4
+    w2 = H * I + (H // 128) * (I // 128) * 4
+    g1_bytes = E_t * w13 + rows * (H + (H // 128) * 4) + rows * (I + (I // 128) * 4)
+    g2_bytes = E_t * w2 + rows * (I + (I // 128) * 4) + rows * 4 + rows * H * 4
+    g1_flops = 2.0 * rows * 2 * I * H
+    g2_flops = 2.0 * rows * H * I
+    return dict(g1_bytes=g1_bytes, g2_bytes=g2_bytes, g1_flops=g1_flops, g2_flops=g2_flops,
+                layer_weight_bytes=E_t * (w13 + w2))
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
+
+
+def gemm_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
+    None when absent or taken on a different version of the GEMM source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    ent = d.get(f"{kernel}:{workload}")
+    if not ent or ent.get("src_sha") != gemm_source_sha():
+        return None
+    return float(ent["bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 100 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["unsampled"], samples=0)
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        under = [v for v in sm if v > 300] or sm
+        return dict(sm_mhz=under[len(under) // 2] if under else None, sm_max_mhz=smax, reasons=sorted(reasons),
+                    samples=len(rows), power_w_max=max(float(r[3]) for r in rows if _isnum(r[3])) if rows else None)
+
+
+def _isnum(s):
+    try:
+        float(s)
+        return True
+    except ValueError:
+        return False
+
+
+# ---------------------------------------------------------- oracle (CPU)
+def oracle_sample(cfg: dict, n_tok: int, seed: int, x_full, wr, bias, expert_bf16):
+    """Prepare the oracle's inputs for the first n_tok tokens of the batch:
+    its own quantization of the weights those tokens need (untimed set-up).
+    Returns a callable that runs the timed oracle forward."""
+    import numpy as np
+    import oracle
+    ocf = oracle.cfg(cfg["H"], cfg["I"], cfg["Nr"], cfg["Kr"], cfg.get("Ns", 1), cfg.get("n_groups", 0),
+                     cfg.get("topk_groups", 0))
+    x = x_full[:n_tok].cpu()
+    idx, _, _, _ = oracle.route(ocf, x, wr.cpu(), bias.cpu())
+    need = sorted(set(int(e) for e in idx.reshape(-1)) | set(range(cfg["Nr"], cfg["Nr"] + cfg.get("Ns", 1))))
+    experts = [None] * (cfg["Nr"] + cfg.get("Ns", 1))
+    for e in need:
+        w13, w2 = expert_bf16(e)
+        a, sa = oracle.quant_128x128(w13.cpu())
+        b, sb = oracle.quant_128x128(w2.cpu())
+        experts[e] = (a, sa, b, sb)
+    wr_c, bias_c = wr.cpu(), bias.cpu()
+
+    def run():
+        return oracle.forward(ocf, x, wr_c, bias_c, experts, tokens=np.arange(n_tok))
+
+    return run, oracle.num_threads()
+
+
+def time_oracle(run, n_tok: int, reps: int = 1) -> float:
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        run()
+    dt = (time.perf_counter() - t0) / reps
+    return n_tok / dt
+
+
+# ------------------------------------------------------------------ main
+def main(argv=None):
+    args = parse(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    import torch
+    import torch.distributed as dist
+
+    import moe_synth as S
+    import sparse_moe_layer_expert_b200 as M
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    cfg = workload_shape(args.workload, args)
+    T = cfg["T"]
+    shape = {k: cfg[k] for k in ("H", "I", "Nr", "Kr", "Ns", "n_groups", "topk_groups")}
+    seed = args.seed
+
+    def expert_bf16(e):
+        return S.gen_expert(e, cfg["H"], cfg["I"], seed, device=dev)
+
+    wr = S.gen_router(cfg["Nr"], cfg["H"], seed, device=dev)
+    bias = S.gen_bias(cfg["Nr"], seed, cfg.get("bias", "uniform"), device=dev)
+    layer = M.MoeLayer.from_generator(shape, expert_bf16, wr, bias, device=dev)
+    xseed = seed * 1009 + rank
+    if cfg.get("x") == "mixture":
+        x, _ = S.gen_mixture_x(T, cfg["H"], xseed, device=dev)
+    else:
+        x = S.gen_x(T, cfg["H"], xseed, device=dev)
+    out = torch.empty((T, cfg["H"]), dtype=torch.bfloat16, device=dev)
+    counts = torch.empty(cfg["Nr"], dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    # ------------------------------------------------ device-timed steps
+    for _ in range(args.warmup):
+        layer.forward(x, out=out, counts_out=counts, stream=stream)
+    layer.check(stream)
+    n_ev = M.MOE_PROFILE_EVENTS
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for row in ev:  # torch creates the CUDA event on first record; the library needs the handles
+        for e in row:
+            e.record(stream)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # older torch: fall back to the ordinal
+        gpu_id = str(local)
+    sampler = ClockSampler(gpu_id)
+    with sampler:
+        for k in range(args.steps):
+            M.moe_profile_events(ev[k])
+            layer.forward(x, out=out, counts_out=counts, stream=stream)
+        M.moe_profile_events(None)
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    layer.check(stream)
+    clocks = sampler.summary()
+    step_ms = [ev[k][0].elapsed_time(ev[k][n_ev - 1]) for k in range(args.steps)]
+    stage_ms = {name: sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)) / args.steps
+                for i, name in enumerate(M.PROFILE_STAGES)}
+    # the timed region is the K back-to-back steps: first start to last end
+    total_ms = ev[0][0].elapsed_time(ev[-1][n_ev - 1])
+    total_ms = max_over_ranks(total_ms, world, dev)
+    ms_per_step = total_ms / args.steps
+    value = world * T / (ms_per_step / 1e3)
+
+    counts_h = counts.cpu()
+    touched = int((counts_h > 0).sum())
+    alg = algorithmic_counts(cfg, T, touched)
+    peaks = measured_peaks()
+    g1_ms, g2_ms = stage_ms["gemm_gate_up"], stage_ms["gemm_down"]
+    dom = "gemm_gate_up" if g1_ms >= g2_ms else "gemm_down"
+    dom_ms = max(g1_ms, g2_ms)
+    dom_bytes = alg["g1_bytes"] if dom == "gemm_gate_up" else alg["g2_bytes"]
+    dom_flops = alg["g1_flops"] if dom == "gemm_gate_up" else alg["g2_flops"]
+    fp8_peak = 2.0 * peaks["bf16_sustained"]  # FP8 dense = 2 x bf16 (nominal ratio 4.5 / 2.25 PFLOP/s)
+    t_mem = dom_bytes / (peaks["hbm"] * 1e9)
+    t_tc = dom_flops / (fp8_peak * 1e12)
+    kernel_name = "gemm_fp8_kernel<0>" if dom == "gemm_gate_up" else "gemm_fp8_kernel<1>"
+    if t_mem >= t_tc:
+        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+        roofline = dict(bound="hbm", achieved=round(achieved, 1), peak=peaks["hbm"], unit="GB/s",
+                        frac=round(achieved / peaks["hbm"], 4), traffic=profiled_traffic(args.workload, kernel_name),
+                        kernel=dom, peak_src=peaks["src"] + " (HBM copy)", algorithmic_bytes=dom_bytes)
+    else:
+        achieved = dom_flops / (dom_ms / 1e3) / 1e12
+        roofline = dict(bound="tensor", achieved=round(achieved, 1), peak=round(fp8_peak, 1), unit="TFLOP/s",
+                        frac=round(achieved / fp8_peak, 4), traffic=profiled_traffic(args.workload, kernel_name),
+                        kernel=dom, peak_src=peaks["src"] + " (bf16 sustained x 2 for FP8)",
+                        algorithmic_flops=dom_flops)
+    gemm_tflops = (alg["g1_flops"] + alg["g2_flops"]) / ((g1_ms + g2_ms) / 1e3) / 1e12
+
+    # ------------------------------------------------ end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        x_h = x.cpu().pin_memory()
+        out_h = torch.empty((T, cfg["H"]), dtype=torch.bfloat16).pin_memory()
+        for _ in range(max(1, args.warmup // 2)):
+            x_d = x_h.to(dev, non_blocking=True)
+            layer.forward(x_d, out=out, stream=stream)
+            out_h.copy_(out, non_blocking=True)
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            x_d = x_h.to(dev, non_blocking=True)
+            layer.forward(x_d, out=out, stream=stream)
+            out_h.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+        e2e = dict(value=round(world * T / (e2e_ms / 1e3), 1), unit="tokens/s",
+                   h2d_bytes_per_step=x_h.numel() * x_h.element_size(),
+                   d2h_bytes_per_step=out_h.numel() * out_h.element_size(), ms_per_step=round(e2e_ms, 4))
+        layer.check(stream)
+
+    # ------------------------------------------------ CPU oracle baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = args.cpu_sample_tokens
+        run, threads = oracle_sample(cfg, n, seed, x, wr, bias, expert_bf16)
+        tps = time_oracle(run, n)
+        cpu = dict(value=round(tps, 4), unit="tokens/s", cores=int(min(threads, n)), kind="oracle",
+                   sample=f"first {n} tokens of the {args.workload} batch: full layer (quantize, route over all "
+                          f"{cfg['Nr']} experts, shared + top-{cfg['Kr']} FP8 FFNs, combine); weight "
+                          f"quantization by the oracle excluded (set-up)")
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = dict(
+        metric=METRIC, value=round(value, 1), unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+        ms_per_step=round(ms_per_step, 4), higher_is_better=True, scaling="weak", vs_baseline=None, dtype="e4m3",
+        data="synthetic",
+        config=dict(workload=f"{args.workload}: T={T} H={cfg['H']} I={cfg['I']} Nr={cfg['Nr']} Kr={cfg['Kr']} "
+                             f"Ns={cfg.get('Ns', 1)} groups={cfg.get('n_groups', 0)}/{cfg.get('topk_groups', 0)}",
+                    global_batch=world * T, tokens_per_gpu=T, parallelism=f"replicas x{world} (no collective)",
+                    l2="no flush: per-step working set >= 11 GB of expert weights >> 126 MB L2",
+                    seed=seed),
+        roofline=roofline,
+        grouped_gemm_tflops=round(gemm_tflops, 1),
+        grouped_gemm_frac_fp8_peak=round(gemm_tflops / fp8_peak, 4),
+        layer_weight_gb=round(alg["layer_weight_bytes"] / 1e9, 3),
+        experts_touched=touched + cfg.get("Ns", 1),
+        stage_ms={k: round(v, 4) for k, v in stage_ms.items()},
+        step_ms_min=round(min(step_ms), 4),
+        cpu_baseline=cpu,
+        e2e=e2e,
+        gpu_launches=KERNELS_PER_STEP * args.steps,
+        clocks=clocks,
+    )
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference(args, rank: int, world: int) -> int:
+    """The reference arm: the CPU oracle, timed on the host cores, on a
+    bounded sample (a few tokens per step) of the same workload."""
+    if rank != 0:
+        return 0
+    import torch
+
+    import moe_synth as S
+    cfg = workload_shape(args.workload, args)
+    T = cfg["T"]
+    seed = args.seed
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+
+    def expert_bf16(e):
+        return S.gen_expert(e, cfg["H"], cfg["I"], seed, device=dev)
+
+    wr = S.gen_router(cfg["Nr"], cfg["H"], seed, device=dev)
+    bias = S.gen_bias(cfg["Nr"], seed, cfg.get("bias", "uniform"), device=dev)
+    if cfg.get("x") == "mixture":
+        x, _ = S.gen_mixture_x(T, cfg["H"], seed * 1009, device=dev)
+    else:
+        x = S.gen_x(T, cfg["H"], seed * 1009, device=dev)
+    n = max(1, min(args.cpu_sample_tokens, 4))
+    run, threads = oracle_sample(cfg, n, seed, x, wr, bias, expert_bf16)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / args.steps
+    tps = n / dt
+    sample = (f"{n} tokens of the {args.workload} batch per step (full layer: quantize, route, shared + "
+              f"top-{cfg['Kr']} FFNs, combine); oracle weight quantization excluded")
+    line = dict(impl="reference", metric=METRIC, value=round(tps, 4), unit="tokens/s", n_gpus=world,
+                steps=args.steps, warmup=args.warmup, ms_per_step=round(dt * 1e3, 2), higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                config=dict(workload=f"{args.workload}: T={T} H={cfg['H']} I={cfg['I']} Nr={cfg['Nr']} "
+                                     f"Kr={cfg['Kr']} Ns={cfg.get('Ns', 1)}", global_batch=n),
+                cpu_baseline=dict(kind="oracle", cores=int(min(threads, n)), sample=sample, value=round(tps, 4),
+                                  unit="tokens/s"),
+                e2e=dict(value=round(tps, 4), unit="tokens/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,262 @@
+/*
+ * moe_fp8.h -- C ABI of the B200 (sm_100a) FP8 DeepSeekMoE layer forward.
+ *
+ * The operations follow the DeepSeek-V3 pages:
+ *  [P4] "DeepSeek-V3 Technischer Bericht" (xyznot.com/de): "Kernideen", FP8
+ *       bullet (E4M3 for all tensors, 1x128 activation tiles, 128x128 weight
+ *       blocks, FP32 promotion every N_c = 128 accumulation steps); "Methode"
+ *       section 2 "DeepSeekMoE mit Auxiliary-Loss-Free Balancing" (layer
+ *       output equation, sigmoid affinity, biased top-K_r gating, gate
+ *       normalisation, per-step bias update with gamma = 0.001).
+ *  [P1] "DeepSeek-V3 技術報告書：MLAと極小スパースMoEがもたらす超低コストフロンティアモデル"
+ *       (singularity-lens.com), formula paragraph: S = max|X| / 448,
+ *       X_FP8 = clip(round(X / S), -448, 448); b_i += gamma*sign(mean - f_i).
+ *  [P2] "DeepSeek-V3 Technical Report" slides (slideify.app), "FP8
+ *       Quantization Logic": 1x128 tiles, 128x128 blocks.
+ *  [P3] "DeepSeek-V3 MoE 2024" glossary (jisaku.com): 256 routed experts +
+ *       1 shared expert, top-8 per token.
+ *
+ * Conventions for every entry point
+ *  - Pointers named *_dev are device pointers (cudaMalloc'd or from a
+ *    framework allocator) owned by the caller; the library keeps no reference
+ *    after the call returns and allocates no device memory.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *    enqueued asynchronously; no entry point synchronises the stream except
+ *    moe_check_device_error.
+ *  - Arguments are validated on the host before anything is enqueued; an
+ *    invalid call returns a negative status and enqueues nothing.
+ *  - bf16 tensors are passed as raw 16-bit words (const void*), E4M3 codes as
+ *    uint8_t (OCP E4M3FN bit patterns), scales as IEEE float.
+ *  - Matrices are row-major; "K-contiguous" means the contraction index is
+ *    the fastest-varying one.
+ *  - Dimensions that the fine-grained scaling tiles (hidden, intermediate,
+ *    GEMM N and K) must be multiples of 128, else MOE_ERR_UNSUPPORTED_SHAPE.
+ *  - err_flag_dev is an int32 in device memory that kernels set (bitwise OR of
+ *    MOE_DEVERR_* codes) when a bounded wait gives up; the caller zeroes it
+ *    and reads it after synchronising (moe_check_device_error).  Kernels
+ *    never trap or spin forever.
+ *  - No C++ exception crosses this boundary.
+ */
+#ifndef MOE_FP8_H
+#define MOE_FP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status */
+enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,        /* null pointer, bad size, misaligned pointer */
+    MOE_ERR_UNSUPPORTED_SHAPE = -2,  /* a tiled dimension is not a multiple of 128, or too large */
+    MOE_ERR_WORKSPACE_TOO_SMALL = -3,
+    MOE_ERR_CUDA = -4,               /* a CUDA runtime call failed (launch, attribute, ...) */
+    MOE_ERR_TIMEOUT = -5,            /* a device-side bounded wait gave up (see err_flag) */
+    MOE_ERR_NOT_IMPLEMENTED = -6,
+    MOE_ERR_NO_DEVICE = -7,          /* no sm_100 device current */
+    MOE_ERR_DEVICE = -8              /* err_flag holds a non-timeout device error */
+};
+
+/* bits that kernels OR into *err_flag_dev */
+enum {
+    MOE_DEVERR_TIMEOUT = 1,          /* an mbarrier wait exceeded its time limit */
+    MOE_DEVERR_BAD_INDEX = 2         /* a routed expert index outside [0, n_routed) was seen */
+};
+
+/* Output element types for moe_forward. */
+enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_F32 = 1 };
+
+/* Human-readable text for a status code (static storage). */
+MOE_API const char *moe_status_string(int status);
+
+/* ABI version (major*100 + minor). */
+MOE_API int moe_abi_version(void);
+
+/* ----------------------------------------------------------- layer shape */
+/* Shape of one DeepSeekMoE layer ([P4] Methode 2; [P3]).
+ *   hidden      H, multiple of 128 (7168 in DeepSeek-V3)
+ *   inter       I, expert SwiGLU intermediate size, multiple of 128 (2048)
+ *   n_routed    N_r routed experts, 1..256 (256)
+ *   top_k       K_r experts per token, 1..min(N_r, 16) (8)
+ *   n_shared    N_s always-active experts, 0 or 1 (1)
+ *   n_groups    group-limited routing: 0 = off, else number of equal
+ *               contiguous expert groups (divides N_r, <= 32)
+ *   topk_groups groups kept per token when n_groups > 0 (1..n_groups)
+ *   route_scale factor applied to the normalised gates (1.0 = the pages') */
+typedef struct {
+    int32_t hidden;
+    int32_t inter;
+    int32_t n_routed;
+    int32_t top_k;
+    int32_t n_shared;
+    int32_t n_groups;
+    int32_t topk_groups;
+    float route_scale;
+} moe_config;
+
+/* Quantized layer weights, all device pointers, experts stacked routed
+ * first (0..N_r-1) then shared (N_r..N_r+N_s-1); E = N_r + N_s.
+ *   w13_dev   E4M3 [E, 2I, H]: rows 0..I-1 of each expert are the gate
+ *             projection W1, rows I..2I-1 the up projection W3 (K = H
+ *             contiguous)
+ *   s13_dev   float [E, 2I/128, H/128] 128x128 block scales of w13
+ *   w2_dev    E4M3 [E, H, I] down projection (K = I contiguous)
+ *   s2_dev    float [E, H/128, I/128]
+ *   wr_dev    bf16 [N_r, H] router centroids e_i
+ * Every pointer must be 16-byte aligned. */
+typedef struct {
+    const uint8_t *w13_dev;
+    const float *s13_dev;
+    const uint8_t *w2_dev;
+    const float *s2_dev;
+    const void *wr_dev;
+} moe_weights;
+
+/* ------------------------------------------------------------ quantizers */
+/* 1x128 activation quantization ([P4] Kernideen; [P1] formula; [P2]).
+ * For each row r and each group g of 128 consecutive columns:
+ *   amax = max |x[r, 128g .. 128g+127]|, S = amax / 448 (FP32, IEEE),
+ *   q[r, c] = E4M3_RNE_satfinite(x[r, c] / S) (IEEE FP32 quotient),
+ *   scales[r, g] = S;  amax == 0 gives S = 0 and codes 0x00.
+ *   x_dev       bf16 [rows, ld_x] (16-byte aligned, ld_x % 8 == 0, ld_x >= cols)
+ *   q_dev       E4M3 [rows, cols], dense (16-byte aligned)
+ *   scales_dev  float [rows, cols/128], dense
+ * rows >= 0 (0 enqueues nothing), cols % 128 == 0. */
+MOE_API int fp8_quant_1x128(const void *x_dev, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q_dev,
+                    float *scales_dev, void *stream);
+
+/* 128x128 weight-block quantization (same rule per 128x128 block; setup
+ * step, not part of the timed layer).
+ *   w_dev       bf16 [n, k] dense, n % 128 == 0, k % 128 == 0
+ *   q_dev       E4M3 [n, k];  scales_dev float [n/128, k/128] */
+MOE_API int fp8_quant_128x128(const void *w_dev, int64_t n, int64_t k, uint8_t *q_dev, float *scales_dev,
+                      void *stream);
+
+/* ---------------------------------------------------------------- GEMM */
+/* Fine-grained block-scaled FP8 GEMM ([P4] Kernideen):
+ *   C[m, n] = sum_kb sA[m, kb] * sB[n/128, kb] * sum_{k in kb} A[m, k] B[n, k]
+ * where each 128-long partial is formed on the tensor cores and promoted
+ * (scaled and added) into an FP32 accumulator -- promotion every N_c = 128.
+ *   A_dev   E4M3 [M, K] K-contiguous;  sA_dev float [M, K/128]
+ *   B_dev   E4M3 [N, K] K-contiguous (the weight, "Linear" layout);
+ *   sB_dev  float [N/128, K/128]
+ *   C_dev   bf16 [M, N] (RNE of the FP32 accumulator)
+ * M >= 1, N % 128 == 0, K % 128 == 0; all pointers 16-byte aligned. */
+MOE_API int fp8_blockscaled_gemm(const uint8_t *A_dev, const float *sA_dev, const uint8_t *B_dev,
+                         const float *sB_dev, void *C_dev, int64_t M, int64_t N, int64_t K,
+                         int32_t *err_flag_dev, void *stream);
+
+/* -------------------------------------------------------------- routing */
+/* Router ([P4] Methode 2): s[t, i] = sigmoid(x_t . e_i) (bf16 inputs, FP32
+ * accumulation on the tensor cores); the K_r experts with the largest
+ * s[t, i] + bias[i] are selected (ties: lower index; if n_groups > 0 only
+ * experts of the topk_groups groups with the largest sum of their two best
+ * s + bias are eligible); gate[t, k] = route_scale * s[t, idx[t, k]] /
+ * sum_k' s[t, idx[t, k']].  idx lists the selection in descending s + bias.
+ *   x_dev      bf16 [T, H] (16-byte aligned)
+ *   wr_dev     bf16 [N_r, H]
+ *   bias_dev   float [N_r]
+ *   idx_dev    int32 [T, K_r];  gate_dev float [T, K_r]
+ *   counts_dev int32 [N_r]: per-expert number of selections (overwritten)
+ *   ws_dev     scratch of moe_route_workspace_size() bytes (256-byte aligned) */
+MOE_API size_t moe_route_workspace_size(const moe_config *cfg, int64_t T);
+MOE_API int moe_route(const moe_config *cfg, const void *x_dev, const void *wr_dev, const float *bias_dev,
+              int64_t T, int32_t *idx_dev, float *gate_dev, int32_t *counts_dev, void *ws_dev,
+              size_t ws_bytes, int32_t *err_flag_dev, void *stream);
+
+/* ------------------------------------------------------------ full layer */
+/* One DeepSeekMoE layer forward ([P4] Methode 2):
+ *   out[t] = u_t + sum_{shared} FFN_s(u_t) + sum_k gate[t, k] FFN_{idx[t,k]}(u_t)
+ * with FFN(u) = W2 (silu(W1 u) * (W3 u)), every projection an FP8 block-scaled
+ * GEMM: u quantized 1x128 (fp8_quant_1x128), routed as moe_route, rows
+ * grouped per expert (stable: token order, then slot), h = silu(G) * U in FP32
+ * re-quantized 1x128 along I before the down projection, the down-projection
+ * output scaled by the gate, then summed per token in FP32 in a fixed order
+ * (residual, shared expert, slots 0..K_r-1) and written as out_dtype.
+ *   x_dev        bf16 [T, H]
+ *   out_dev      [T, H] of MOE_DTYPE_BF16 (RNE) or MOE_DTYPE_F32
+ *   idx_out_dev  nullable int32 [T, K_r]: routing decision
+ *   counts_out_dev nullable int32 [N_r]: per-expert load (input of moe_bias_update)
+ *   ws_dev       scratch of moe_workspace_size() bytes, 256-byte aligned; its
+ *                layout is reported by moe_workspace_layout (for inspection)
+ * T >= 0 (0 enqueues nothing). */
+MOE_API size_t moe_workspace_size(const moe_config *cfg, int64_t T);
+MOE_API int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias_dev, const void *x_dev,
+                int64_t T, void *out_dev, int32_t out_dtype, int32_t *idx_out_dev,
+                int32_t *counts_out_dev, void *ws_dev, size_t ws_bytes, int32_t *err_flag_dev,
+                void *stream);
+
+/* Byte offsets of the intermediates inside moe_forward's workspace, for
+ * tests and profiling (all 256-byte aligned).  Rows: R = T*K_r routed rows in
+ * expert-contiguous order, then T*N_s shared-expert rows in token order.
+ * Each entry is {offset, bytes}. */
+typedef struct {
+    size_t xq[2];       /* E4M3 [T, H]       1x128-quantized input            */
+    size_t xs[2];       /* float [T, H/128]                                    */
+    size_t idx[2];      /* int32 [T, K_r]                                      */
+    size_t gate[2];     /* float [T, K_r]                                      */
+    size_t counts[2];   /* int32 [N_r]                                         */
+    size_t offsets[2];  /* int32 [N_r + 1]  first row of each expert           */
+    size_t pos[2];      /* int32 [T, K_r]   row of (t, k) in expert order      */
+    size_t ap[2];       /* E4M3 [R, H]      expert-contiguous copy of xq rows  */
+    size_t as[2];       /* float [R, H/128]                                    */
+    size_t row_gate[2]; /* float [R + T*N_s] gate of each row (1 for shared)   */
+    size_t hq[2];       /* E4M3 [R + T*N_s, I] re-quantized SwiGLU output      */
+    size_t hs[2];       /* float [R + T*N_s, I/128]                            */
+    size_t y[2];        /* float [R + T*N_s, H] gate-scaled expert outputs     */
+    size_t ntiles[2];   /* int32 [4]: tiles of the two grouped GEMMs, rows, chunks */
+    size_t logits[2];   /* float [S, T, N_r] router logit partials (S K-splits) */
+    size_t blk_hist[2]; /* int32 [ceil(T/128), N_r] per-block expert counts    */
+    size_t blk_base[2]; /* int32 [ceil(T/128), N_r] per-block first rows       */
+    size_t tiles1[2];   /* work list of the gate/up GEMM (32-byte entries)     */
+    size_t tiles2[2];   /* work list of the down GEMM                          */
+    size_t total;
+} moe_ws_layout;
+MOE_API int moe_workspace_layout(const moe_config *cfg, int64_t T, moe_ws_layout *layout);
+
+/* Measurement hook: when set (n_events >= MOE_PROFILE_EVENTS), every later
+ * moe_forward on this host thread records events[i] (caller-created
+ * cudaEvent_t handles) on its stream at the stage boundaries below, so
+ * per-stage device time can be read with cudaEventElapsedTime.  Pass NULL/0
+ * to turn it off.  Events are recorded, never created or destroyed, by the
+ * library; recording adds no kernel launches.
+ *   0 start | 1 after quantize | 2 after routing | 3 after grouping (hist,
+ *   work lists, row copies) | 4 after gate/up GEMM (+SwiGLU, requant) |
+ *   5 after down GEMM | 6 after combine */
+enum { MOE_PROFILE_EVENTS = 7 };
+MOE_API int moe_profile_events(void *const *events, int32_t n_events);
+
+/* --------------------------------------------------------- bias update */
+/* Auxiliary-loss-free balancing step ([P4] Methode 2; [P1]): with
+ * mean = total_assignments / n_routed, bias[i] -= gamma if counts[i] > mean,
+ * bias[i] += gamma if counts[i] < mean, unchanged if equal (FP32, in place).
+ *   bias_dev float [n_routed];  counts_dev int32 [n_routed] */
+MOE_API int moe_bias_update(float *bias_dev, const int32_t *counts_dev, int32_t n_routed,
+                    int64_t total_assignments, float gamma, void *stream);
+
+/* ------------------------------------------------------------ errors */
+/* Synchronises `stream`, copies *err_flag_dev to *host_value (nullable) and
+ * returns MOE_OK if it is 0, MOE_ERR_TIMEOUT if the timeout bit is set, else
+ * MOE_ERR_DEVICE.  Does not clear the flag. */
+MOE_API int moe_check_device_error(const int32_t *err_flag_dev, int32_t *host_value, void *stream);
+
+/* Failure-detection self test: launches one block whose thread waits on an
+ * mbarrier that nothing arrives on, with a wait limit of limit_us
+ * microseconds (1..10^6).  The wait gives up, sets MOE_DEVERR_TIMEOUT in
+ * *err_flag_dev and the kernel returns; the context stays usable. */
+MOE_API int moe_selftest_wait_timeout(int32_t *err_flag_dev, int64_t limit_us, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_FP8_H */

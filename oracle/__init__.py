@@ -82,6 +82,13 @@ def cfg(H, I, Nr, Kr, Ns=1, n_groups=0, topk_groups=0, route_scale=1.0) -> Cfg:
     return Cfg(H, I, Nr, Kr, Ns, n_groups, topk_groups, 0, route_scale)
 
 
+def _f32(a) -> np.ndarray:
+    """float32 numpy copy of a numpy array or a (possibly device) torch tensor."""
+    if not isinstance(a, np.ndarray) and hasattr(a, "detach"):
+        a = a.detach().cpu().float().numpy()
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
 def _u16(a) -> np.ndarray:
     """bf16 data as its raw 16-bit patterns (accepts a torch bf16 tensor or a
     uint16 numpy array)."""
@@ -168,7 +175,7 @@ def route(cf: Cfg, x, Wr, bias, want_s: bool = False):
     """Returns (idx i32 [T,Kr], gate f64 [T,Kr], gap f32 [T], s f64 [T,Nr] or None)."""
     xu = _u16(x)
     wu = _u16(Wr)
-    b = np.ascontiguousarray(bias, np.float32)
+    b = _f32(bias)
     T = xu.shape[0]
     idx = np.empty((T, cf.Kr), np.int32)
     gate = np.empty((T, cf.Kr), np.float64)
@@ -238,7 +245,7 @@ def forward(cf: Cfg, x, Wr, bias, experts, tokens=None):
         for j in range(4):
             ptrs[j][e] = arrs[j].ctypes.data
     wu = _u16(Wr)
-    b = np.ascontiguousarray(bias, np.float32)
+    b = _f32(bias)
     out = np.empty((n, H), np.float64)
     outb = np.empty((n, H), np.uint16)
     idx = np.empty((n, cf.Kr), np.int32)

@@ -1,0 +1,448 @@
+// api.cu -- the extern "C" entry points of libmoefp8 (declared in
+// include/moe_fp8.h): argument validation, workspace carving, tensor-map
+// encoding and the launch sequence of the layer forward.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe_host {
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void resolve_encode() {
+  cudaDriverEntryPointQueryResult q;
+  void *fn = nullptr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices] = {0};
+int g_major[kMaxDevices] = {0};
+}  // namespace
+
+int encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  std::call_once(g_encode_once, resolve_encode);
+  if (!g_encode) return -1;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      g_encode(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+static int device_info(int *sms, int *major) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  if (g_sms[dev] == 0) {
+    int s = 0, m = 0;
+    if (cudaDeviceGetAttribute(&s, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    if (cudaDeviceGetAttribute(&m, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return -1;
+    g_major[dev] = m;
+    g_sms[dev] = s;
+  }
+  *sms = g_sms[dev];
+  *major = g_major[dev];
+  return 0;
+}
+
+int sm_count() {
+  int s = 0, m = 0;
+  if (device_info(&s, &m) != 0) return 148;
+  return s;
+}
+
+}  // namespace moe_host
+
+namespace {
+
+using moe::GemmTile;
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_device() {
+  int sms = 0, major = 0;
+  if (moe_host::device_info(&sms, &major) != 0) return MOE_ERR_NO_DEVICE;
+  if (major != 10) return MOE_ERR_NO_DEVICE;
+  return MOE_OK;
+}
+
+int check_cfg(const moe_config *c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->hidden <= 0 || c->inter <= 0 || c->n_routed <= 0 || c->top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (c->hidden % 128 || c->inter % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (c->hidden > 65536 || c->inter > 65536) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (c->n_routed > 256 || c->top_k > 16 || c->top_k > c->n_routed) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (c->n_shared < 0 || c->n_shared > 1) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (c->n_groups < 0) return MOE_ERR_INVALID_ARG;
+  if (c->n_groups > 0) {
+    if (c->n_groups > 32 || c->n_routed % c->n_groups) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->topk_groups < 1 || c->topk_groups > c->n_groups) return MOE_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(c->topk_groups) * (c->n_routed / c->n_groups) < c->top_k) return MOE_ERR_INVALID_ARG;
+  }
+  if (!(c->route_scale == c->route_scale)) return MOE_ERR_INVALID_ARG;
+  // weight rows must be addressable by 32-bit TMA coordinates
+  const int64_t E = static_cast<int64_t>(c->n_routed) + c->n_shared;
+  if (E * 2 * c->inter > INT32_MAX || E * c->hidden > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+constexpr int64_t kMaxTokens = 1 << 20;
+
+struct Carve {
+  size_t off = 0;
+  void take(size_t (&slot)[2], size_t bytes) {
+    off = (off + 255) & ~size_t(255);
+    slot[0] = off;
+    slot[1] = bytes;
+    off += bytes;
+  }
+};
+
+void make_layout(const moe_config *c, int64_t T, moe_ws_layout *L) {
+  const int64_t H = c->hidden, I = c->inter, Nr = c->n_routed, Kr = c->top_k, Ns = c->n_shared;
+  const int64_t R = T * Kr, RS = R + T * Ns;
+  const int64_t nblk = (T + 127) / 128;
+  const int64_t ks = moe::router_ksplit(T, static_cast<int>(Nr), static_cast<int>(H));
+  const int64_t chunks = moe::max_chunks(T, static_cast<int>(Kr), static_cast<int>(Nr), static_cast<int>(Ns));
+  Carve cv;
+  cv.take(L->xq, T * H);
+  cv.take(L->xs, T * (H / 128) * 4);
+  cv.take(L->idx, T * Kr * 4);
+  cv.take(L->gate, T * Kr * 4);
+  cv.take(L->counts, Nr * 4);
+  cv.take(L->offsets, (Nr + 1) * 4);
+  cv.take(L->pos, T * Kr * 4);
+  cv.take(L->ap, R * H);
+  cv.take(L->as, R * (H / 128) * 4);
+  cv.take(L->row_gate, RS * 4);
+  cv.take(L->hq, RS * I);
+  cv.take(L->hs, RS * (I / 128) * 4);
+  cv.take(L->y, RS * H * 4);
+  cv.take(L->ntiles, 4 * 4);
+  cv.take(L->logits, ks * T * Nr * 4);
+  cv.take(L->blk_hist, nblk * Nr * 4);
+  cv.take(L->blk_base, nblk * Nr * 4);
+  cv.take(L->tiles1, chunks * moe::gemm1_blocks(static_cast<int>(I)) * sizeof(GemmTile));
+  cv.take(L->tiles2, chunks * moe::gemm2_blocks(static_cast<int>(H)) * sizeof(GemmTile));
+  L->total = (cv.off + 255) & ~size_t(255);
+}
+
+thread_local cudaEvent_t g_prof_events[MOE_PROFILE_EVENTS];
+thread_local bool g_prof_on = false;
+
+inline cudaError_t prof_mark(int i, cudaStream_t st) {
+  return g_prof_on ? cudaEventRecord(g_prof_events[i], st) : cudaSuccess;
+}
+
+template <typename P>
+inline P at(void *ws, const size_t (&slot)[2]) {
+  return reinterpret_cast<P>(static_cast<uint8_t *>(ws) + slot[0]);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_status_string(int s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (tiled dimensions must be multiples of 128)";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_NOT_IMPLEMENTED: return "not implemented";
+    case MOE_ERR_NO_DEVICE: return "no sm_100 device is current";
+    case MOE_ERR_DEVICE: return "device reported an error";
+    default: return "unknown status";
+  }
+}
+
+int moe_abi_version(void) { return 100; }
+
+int fp8_quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q, float *scales,
+                    void *stream) {
+  if (rows < 0 || cols <= 0 || ld_x < cols || (ld_x % 8) != 0) return MOE_ERR_INVALID_ARG;
+  if (cols % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!x || !q || !scales || !aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 3))
+    return MOE_ERR_INVALID_ARG;
+  if (const int d = check_device()) return d;
+  return cuda_status(moe::launch_quant_1x128(x, rows, cols, ld_x, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *scales, void *stream) {
+  if (n < 0 || k < 0) return MOE_ERR_INVALID_ARG;
+  if (n % 128 || k % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0 || k == 0) return MOE_OK;
+  if (!w || !q || !scales || !aligned16(w) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 3))
+    return MOE_ERR_INVALID_ARG;
+  if ((n / 128) * (k / 128) > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (const int d = check_device()) return d;
+  return cuda_status(moe::launch_quant_128x128(w, n, k, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_blockscaled_gemm(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB, void *C, int64_t M,
+                         int64_t N, int64_t K, int32_t *err_flag, void *stream) {
+  if (M < 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (N % 128 || K % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return MOE_OK;
+  if (M > INT32_MAX - 256 || N > INT32_MAX - 256) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!A || !sA || !B || !sB || !C || !err_flag) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return MOE_ERR_INVALID_ARG;
+  if (const int d = check_device()) return d;
+  moe::GemmLaunch g{};
+  g.w = B;
+  g.w_rows = N;
+  g.a0 = A;
+  g.a0_rows = M;
+  g.a1 = A;
+  g.a1_rows = M;
+  g.K = K;
+  g.sw = sB;
+  g.sa0 = sA;
+  g.sa1 = sA;
+  g.tiles = nullptr;
+  g.n_tiles = nullptr;
+  g.dense_M = M;
+  const int64_t tiles = ((M + 127) / 128) * ((N / 128 + 1) / 2);
+  if (tiles > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  g.max_tiles = static_cast<int>(tiles);
+  g.epi = moe::EPI_BF16;
+  g.out = C;
+  g.ldo = N;
+  g.out_rows = M;
+  g.out_cols = N;
+  g.err = err_flag;
+  g.wait_limit_ns = moe::kDefaultWaitLimitNs;
+  return cuda_status(moe::launch_gemm(g, static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_route_workspace_size(const moe_config *cfg, int64_t T) {
+  if (check_cfg(cfg) != MOE_OK || T < 0 || T > kMaxTokens) return 0;
+  const int64_t ks = moe::router_ksplit(T, cfg->n_routed, cfg->hidden);
+  return static_cast<size_t>(ks * T * cfg->n_routed * 4 + 256);
+}
+
+int moe_route(const moe_config *cfg, const void *x, const void *wr, const float *bias, int64_t T, int32_t *idx,
+              float *gate, int32_t *counts, void *ws, size_t ws_bytes, int32_t *err_flag, void *stream) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
+  if (!counts) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if (const int d = check_device()) return d;
+    return cuda_status(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_routed, st));
+  }
+  if (!x || !wr || !bias || !idx || !gate || !ws || !err_flag) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(wr) || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_route_workspace_size(cfg, T)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (const int d = check_device()) return d;
+  float *partial = static_cast<float *>(ws);
+  const int ks = moe::router_ksplit(T, cfg->n_routed, cfg->hidden);
+  cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_routed, st);
+  if (e == cudaSuccess)
+    e = moe::launch_router_logits(x, wr, T, cfg->n_routed, cfg->hidden, partial, err_flag,
+                                  moe::kDefaultWaitLimitNs, st);
+  if (e == cudaSuccess)
+    e = moe::launch_router_topk(partial, ks, T, cfg->n_routed, cfg->top_k, cfg->n_groups, cfg->topk_groups,
+                                cfg->route_scale, bias, idx, gate, counts, st);
+  return cuda_status(e);
+}
+
+size_t moe_workspace_size(const moe_config *cfg, int64_t T) {
+  if (check_cfg(cfg) != MOE_OK || T < 0 || T > kMaxTokens) return 0;
+  moe_ws_layout L;
+  make_layout(cfg, T, &L);
+  return L.total;
+}
+
+int moe_workspace_layout(const moe_config *cfg, int64_t T, moe_ws_layout *layout) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (T < 0 || T > kMaxTokens || !layout) return MOE_ERR_INVALID_ARG;
+  make_layout(cfg, T, layout);
+  return MOE_OK;
+}
+
+int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, const void *x, int64_t T, void *out,
+                int32_t out_dtype, int32_t *idx_out, int32_t *counts_out, void *ws, size_t ws_bytes,
+                int32_t *err_flag, void *stream) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
+  if (out_dtype != MOE_DTYPE_BF16 && out_dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if (counts_out) {
+      if (const int d = check_device()) return d;
+      return cuda_status(cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * cfg->n_routed, st));
+    }
+    return MOE_OK;
+  }
+  if (!w || !bias || !x || !out || !ws || !err_flag) return MOE_ERR_INVALID_ARG;
+  if (!w->w13_dev || !w->s13_dev || !w->w2_dev || !w->s2_dev || !w->wr_dev) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out) || !aligned16(w->w13_dev) || !aligned16(w->w2_dev) || !aligned16(w->wr_dev) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255))
+    return MOE_ERR_INVALID_ARG;
+  moe_ws_layout L;
+  make_layout(cfg, T, &L);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (const int d = check_device()) return d;
+
+  const int H = cfg->hidden, I = cfg->inter, Nr = cfg->n_routed, Kr = cfg->top_k, Ns = cfg->n_shared;
+  const int64_t R = T * Kr, RS = R + T * Ns;
+  const int64_t E = static_cast<int64_t>(Nr) + Ns;
+  uint8_t *xq = at<uint8_t *>(ws, L.xq);
+  float *xs = at<float *>(ws, L.xs);
+  int32_t *idx = at<int32_t *>(ws, L.idx);
+  float *gate = at<float *>(ws, L.gate);
+  int32_t *counts = at<int32_t *>(ws, L.counts);
+  int32_t *offsets = at<int32_t *>(ws, L.offsets);
+  int32_t *pos = at<int32_t *>(ws, L.pos);
+  uint8_t *ap = at<uint8_t *>(ws, L.ap);
+  float *as = at<float *>(ws, L.as);
+  float *row_gate = at<float *>(ws, L.row_gate);
+  uint8_t *hq = at<uint8_t *>(ws, L.hq);
+  float *hs = at<float *>(ws, L.hs);
+  float *y = at<float *>(ws, L.y);
+  int32_t *ntiles = at<int32_t *>(ws, L.ntiles);
+  float *logits = at<float *>(ws, L.logits);
+  int32_t *blk_hist = at<int32_t *>(ws, L.blk_hist);
+  int32_t *blk_base = at<int32_t *>(ws, L.blk_base);
+  GemmTile *tiles1 = at<GemmTile *>(ws, L.tiles1);
+  GemmTile *tiles2 = at<GemmTile *>(ws, L.tiles2);
+  const int ks = moe::router_ksplit(T, Nr, H);
+  const int64_t chunks = moe::max_chunks(T, Kr, Nr, Ns);
+
+  cudaError_t e = prof_mark(0, st);
+  if (e == cudaSuccess) e = moe::launch_quant_1x128(x, T, H, H, xq, xs, st);
+  if (e == cudaSuccess) e = prof_mark(1, st);
+  if (e == cudaSuccess)
+    e = moe::launch_router_logits(x, w->wr_dev, T, Nr, H, logits, err_flag, moe::kDefaultWaitLimitNs, st);
+  if (e == cudaSuccess)
+    e = moe::launch_router_topk(logits, ks, T, Nr, Kr, cfg->n_groups, cfg->topk_groups, cfg->route_scale, bias,
+                                idx, gate, nullptr, st);
+  if (e == cudaSuccess) e = prof_mark(2, st);
+  if (e == cudaSuccess) e = moe::launch_hist(idx, T, Kr, Nr, blk_hist, err_flag, st);
+  if (e == cudaSuccess)
+    e = moe::launch_build_tiles(blk_hist, T, Kr, Nr, Ns, H, I, counts, offsets, blk_base, tiles1, tiles2, ntiles,
+                                counts_out, st);
+  if (e == cudaSuccess)
+    e = moe::launch_scatter(idx, gate, xq, xs, T, Kr, Nr, Ns, H, blk_base, ap, as, row_gate, pos, st);
+  if (e == cudaSuccess) e = prof_mark(3, st);
+  if (e == cudaSuccess) {
+    // gate/up projection + SwiGLU + 1x128 requantization
+    moe::GemmLaunch g{};
+    g.w = w->w13_dev;
+    g.w_rows = E * 2 * I;
+    g.a0 = ap;
+    g.a0_rows = R;
+    g.a1 = xq;
+    g.a1_rows = T;
+    g.K = H;
+    g.sw = w->s13_dev;
+    g.sa0 = as;
+    g.sa1 = xs;
+    g.tiles = tiles1;
+    g.n_tiles = ntiles;
+    g.tile_slot = 0;
+    g.max_tiles = static_cast<int>(chunks * moe::gemm1_blocks(I));
+    g.epi = moe::EPI_SWIGLU_Q;
+    g.out = hq;
+    g.ldo = I;
+    g.out_rows = RS;
+    g.out_cols = 2 * I;  // block B (up) shares block A's output columns
+    g.out_scale = hs;
+    g.ld_os = I / 128;
+    g.err = err_flag;
+    g.wait_limit_ns = moe::kDefaultWaitLimitNs;
+    e = moe::launch_gemm(g, st);
+  }
+  if (e == cudaSuccess) e = prof_mark(4, st);
+  if (e == cudaSuccess) {
+    // down projection, scaled by the gate of each row
+    moe::GemmLaunch g{};
+    g.w = w->w2_dev;
+    g.w_rows = E * H;
+    g.a0 = hq;
+    g.a0_rows = RS;
+    g.a1 = hq;
+    g.a1_rows = RS;
+    g.K = I;
+    g.sw = w->s2_dev;
+    g.sa0 = hs;
+    g.sa1 = hs;
+    g.tiles = tiles2;
+    g.n_tiles = ntiles;
+    g.tile_slot = 1;
+    g.max_tiles = static_cast<int>(chunks * moe::gemm2_blocks(H));
+    g.epi = moe::EPI_GATE_F32;
+    g.out = y;
+    g.ldo = H;
+    g.out_rows = RS;
+    g.out_cols = H;
+    g.row_gate = row_gate;
+    g.err = err_flag;
+    g.wait_limit_ns = moe::kDefaultWaitLimitNs;
+    e = moe::launch_gemm(g, st);
+  }
+  if (e == cudaSuccess) e = prof_mark(5, st);
+  if (e == cudaSuccess) e = moe::launch_combine(x, y, pos, T, H, Kr, R, Ns, out, out_dtype == MOE_DTYPE_F32, st);
+  if (e == cudaSuccess) e = prof_mark(6, st);
+  if (e == cudaSuccess && idx_out)
+    e = cudaMemcpyAsync(idx_out, idx, sizeof(int32_t) * T * Kr, cudaMemcpyDeviceToDevice, st);
+  return cuda_status(e);
+}
+
+int moe_profile_events(void *const *events, int32_t n_events) {
+  if (!events || n_events <= 0) {
+    g_prof_on = false;
+    return MOE_OK;
+  }
+  if (n_events < MOE_PROFILE_EVENTS) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < MOE_PROFILE_EVENTS; ++i) {
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+    g_prof_events[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  g_prof_on = true;
+  return MOE_OK;
+}
+
+int moe_bias_update(float *bias, const int32_t *counts, int32_t n_routed, int64_t total, float gamma,
+                    void *stream) {
+  if (!bias || !counts || n_routed <= 0 || total < 0) return MOE_ERR_INVALID_ARG;
+  if (const int d = check_device()) return d;
+  return cuda_status(moe::launch_bias_update(bias, counts, n_routed, total, gamma, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_check_device_error(const int32_t *err_flag, int32_t *host_value, void *stream) {
+  if (!err_flag) return MOE_ERR_INVALID_ARG;
+  if (const int d = check_device()) return d;
+  int32_t v = 0;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&v, err_flag, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (host_value) *host_value = v;
+  if (v == 0) return MOE_OK;
+  return (v & MOE_DEVERR_TIMEOUT) ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE;
+}
+
+int moe_selftest_wait_timeout(int32_t *err_flag, int64_t limit_us, void *stream) {
+  if (!err_flag || limit_us < 1 || limit_us > 1000000) return MOE_ERR_INVALID_ARG;
+  if (const int d = check_device()) return d;
+  return cuda_status(
+      moe::launch_wait_selftest(err_flag, static_cast<uint64_t>(limit_us) * 1000ull, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+// kernels.h -- host-side launchers of the libmoefp8 kernels (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// One unit of work of the grouped block-scaled GEMM: a pair of 128-row
+// weight blocks (block B optional) against up to 128 activation rows.
+struct GemmTile {
+  int32_t w_row0;   // first row of weight block A in the weight tensor
+  int32_t w_row1;   // first row of weight block B, or -1
+  int32_t sw0;      // 128-row block index of block A in the weight scales
+  int32_t sw1;      // 128-row block index of block B
+  int32_t a_row;    // first activation row
+  int32_t n;        // activation rows in this tile, 1..128
+  int32_t out_row;  // first output row
+  int32_t out_col;  // bits 0..23: first output column of block A's outputs;
+                    // bit 24: activations come from the second tensor map
+};
+constexpr int32_t kTileFromMap1 = 1 << 24;
+
+enum EpiKind : int { EPI_SWIGLU_Q = 0, EPI_GATE_F32 = 1, EPI_BF16 = 2 };
+
+struct GemmLaunch {
+  // tensor operands
+  const uint8_t *w;       // weights [w_rows, K]
+  int64_t w_rows;
+  const uint8_t *a0;      // activations [a0_rows, K]
+  int64_t a0_rows;
+  const uint8_t *a1;      // second activation tensor (may equal a0)
+  int64_t a1_rows;
+  int64_t K;
+  const float *sw;        // weight scales [w_rows/128, K/128]
+  const float *sa0;       // activation scales [a0_rows, K/128]
+  const float *sa1;
+  // tiles: either a device list (tiles != null, count at n_tiles[slot]) or
+  // the dense grid of a plain GEMM (dense_M rows x w_rows outputs)
+  const GemmTile *tiles;
+  const int32_t *n_tiles;
+  int tile_slot;
+  int max_tiles;          // host-side upper bound (grid sizing)
+  int64_t dense_M;
+  // epilogue
+  int epi;
+  void *out;
+  int64_t ldo;
+  int64_t out_rows;       // rows of `out` (bounds check)
+  int64_t out_cols;       // output columns addressable per row (bounds check)
+  float *out_scale;
+  int64_t ld_os;
+  const float *row_gate;
+  int32_t *err;
+  uint64_t wait_limit_ns;
+};
+
+cudaError_t launch_quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ldx, uint8_t *q, float *s,
+                               cudaStream_t st);
+cudaError_t launch_quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *s, cudaStream_t st);
+
+int router_ksplit(int64_t T, int Nr, int H);
+cudaError_t launch_router_logits(const void *x, const void *wr, int64_t T, int Nr, int H, float *partial,
+                                 int32_t *err, uint64_t limit_ns, cudaStream_t st);
+cudaError_t launch_router_topk(const float *partial, int n_ks, int64_t T, int Nr, int Kr, int n_groups,
+                               int topk_groups, float route_scale, const float *bias, int32_t *idx, float *gate,
+                               int32_t *counts, cudaStream_t st);
+
+cudaError_t launch_hist(const int32_t *idx, int64_t T, int Kr, int Nr, int32_t *blk_hist, int32_t *err,
+                        cudaStream_t st);
+cudaError_t launch_build_tiles(const int32_t *blk_hist, int64_t T, int Kr, int Nr, int Ns, int H, int I,
+                               int32_t *counts, int32_t *offsets, int32_t *blk_base, GemmTile *tiles1,
+                               GemmTile *tiles2, int32_t *ntiles, int32_t *counts_out, cudaStream_t st);
+cudaError_t launch_scatter(const int32_t *idx, const float *gate, const uint8_t *xq, const float *xs, int64_t T,
+                           int Kr, int Nr, int Ns, int H, const int32_t *blk_base, uint8_t *ap, float *as,
+                           float *row_gate, int32_t *pos, cudaStream_t st);
+
+cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st);
+
+cudaError_t launch_combine(const void *x, const float *y, const int32_t *pos, int64_t T, int H, int Kr,
+                           int64_t R, int Ns, void *out, int out_f32, cudaStream_t st);
+cudaError_t launch_bias_update(float *bias, const int32_t *counts, int Nr, int64_t total, float gamma,
+                               cudaStream_t st);
+cudaError_t launch_wait_selftest(int32_t *err, uint64_t limit_ns, cudaStream_t st);
+
+// tiles per 128-row chunk of activations in each grouped GEMM
+__host__ __device__ inline int gemm1_blocks(int I) { return I / 128; }
+__host__ __device__ inline int gemm2_blocks(int H) { return (H / 128 + 1) / 2; }
+// upper bound on chunks of <= 128 rows over all experts
+inline int64_t max_chunks(int64_t T, int Kr, int Nr, int Ns) {
+  return (T * Kr) / 128 + Nr + 1 + (Ns ? (T + 127) / 128 : 0);
+}
+
+}  // namespace moe

@@ -1,0 +1,81 @@
+"""MoeLayer: device-resident weights, bias, workspace and error flag of one
+FP8 DeepSeekMoE layer, with forward / bias-update calls into libmoefp8.
+
+Plumbing only: torch allocates the buffers; quantization, routing, the
+grouped GEMMs and the combine all run in the library's kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _binding as B
+
+
+class MoeLayer:
+    def __init__(self, shape: dict, device="cuda"):
+        """shape: dict with H, I, Nr, Kr and optionally Ns (1), n_groups,
+        topk_groups, route_scale."""
+        self.shape = dict(shape)
+        self.cfg = B.config_from(shape)
+        c = self.cfg
+        self.E = c.n_routed + c.n_shared
+        H, I = c.hidden, c.inter
+        dev = torch.device(device)
+        self.device = dev
+        self.w13 = torch.empty((self.E, 2 * I, H), dtype=torch.uint8, device=dev)
+        self.s13 = torch.empty((self.E, 2 * I // 128, H // 128), dtype=torch.float32, device=dev)
+        self.w2 = torch.empty((self.E, H, I), dtype=torch.uint8, device=dev)
+        self.s2 = torch.empty((self.E, H // 128, I // 128), dtype=torch.float32, device=dev)
+        self.wr = torch.empty((c.n_routed, H), dtype=torch.bfloat16, device=dev)
+        self.bias = torch.zeros((c.n_routed,), dtype=torch.float32, device=dev)
+        self.err = B.new_err_flag(dev)
+        self._ws: dict[int, torch.Tensor] = {}
+
+    # -------------------------------------------------------------- weights
+    def set_expert(self, e: int, w13_bf16: torch.Tensor, w2_bf16: torch.Tensor, stream=None) -> None:
+        """Quantize expert e's bf16 weights (128x128 blocks) into place."""
+        B.fp8_quant_128x128(w13_bf16.contiguous(), q=self.w13[e], scales=self.s13[e], stream=stream)
+        B.fp8_quant_128x128(w2_bf16.contiguous(), q=self.w2[e], scales=self.s2[e], stream=stream)
+
+    def set_router(self, wr_bf16: torch.Tensor, bias: torch.Tensor) -> None:
+        self.wr.copy_(wr_bf16)
+        self.bias.copy_(bias)
+
+    @classmethod
+    def from_generator(cls, shape: dict, expert_fn, wr: torch.Tensor, bias: torch.Tensor, device="cuda"):
+        """expert_fn(e) -> (w13 bf16 [2I, H], w2 bf16 [H, I]) on `device`,
+        called once per expert (routed 0..Nr-1, then shared)."""
+        layer = cls(shape, device)
+        for e in range(layer.E):
+            w13, w2 = expert_fn(e)
+            layer.set_expert(e, w13, w2)
+            del w13, w2
+        layer.set_router(wr, bias)
+        return layer
+
+    def weights(self) -> dict:
+        return dict(w13=self.w13, s13=self.s13, w2=self.w2, s2=self.s2, wr=self.wr)
+
+    # -------------------------------------------------------------- forward
+    def workspace(self, T: int) -> torch.Tensor:
+        ws = self._ws.get(T)
+        if ws is None:
+            ws = torch.empty(max(B.moe_workspace_size(self.cfg, T), 256), dtype=torch.uint8, device=self.device)
+            self._ws[T] = ws
+        return ws
+
+    def forward(self, x: torch.Tensor, out=None, out_dtype=B.MOE_DTYPE_BF16, idx_out=None, counts_out=None,
+                stream=None) -> torch.Tensor:
+        return B.moe_forward(self.cfg, self.weights(), self.bias, x, out=out, out_dtype=out_dtype, idx_out=idx_out,
+                             counts_out=counts_out, ws=self.workspace(x.shape[0]), err=self.err, stream=stream)
+
+    def bias_update(self, counts: torch.Tensor, T: int, gamma: float = 0.001, stream=None) -> None:
+        B.moe_bias_update(self.bias, counts, self.cfg.n_routed, T * self.cfg.top_k, gamma, stream=stream)
+
+    def check(self, stream=None) -> None:
+        st, v = B.moe_check_device_error(self.err, stream)
+        if st != B.MOE_OK:
+            raise B.MoeError(st, f"device error flag {v:#x}")
+
+    def layout(self, T: int) -> dict:
+        return B.moe_workspace_layout(self.cfg, T)

@@ -1,0 +1,111 @@
+"""Shared helpers of the test suite: the comparison rule and problem builders.
+
+Comparison rule (the layer's stated tolerance): floating outputs within a
+relative Frobenius error of 2e-3 and a max |diff| of 1e-2 * rms(ref); for an
+output stored as bf16, the format's own rounding (half a bf16 ulp of the
+reference value) is added to the elementwise bound.  Integer and code
+outputs compare bit-exactly.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import moe_synth as S
+
+REL_FRO = 2e-3
+MAX_REL_RMS = 1e-2
+# Routing near-tie rule.  A token is exempt from the bit-exact comparison of
+# its expert set when the oracle's gap between the last selected and the first
+# rejected biased score is below NEAR_TIE.  The layer's stated rule uses 1e-5;
+# on the V3-shaped workloads about 0.3% of tokens have such gaps (the top-8
+# sigmoid scores crowd near 0.96, mean 8th/9th spacing ~3.6e-3), more than the
+# 0.1% the rule tolerates, so the comparison uses the stricter 1e-6: every
+# token with a gap of 1e-6 or more must match exactly and the exempt share
+# stays well under 0.1%.  Tokens below the stated 1e-5 are still counted and
+# reported.
+NEAR_TIE = 1e-6
+STATED_NEAR_TIE = 1e-5
+
+
+def half_ulp_bf16(ref: np.ndarray) -> np.ndarray:
+    a = np.abs(ref)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(e - 8), 2.0 ** -134)
+
+
+def assert_close(got, ref, bf16_out: bool = False, what: str = "", rel_fro=REL_FRO, max_rel_rms=MAX_REL_RMS):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    d = got - ref
+    nref = np.linalg.norm(ref)
+    rms = math.sqrt(float(np.mean(ref * ref))) if ref.size else 0.0
+    fro = np.linalg.norm(d) / nref if nref > 0 else np.linalg.norm(d)
+    allow = max_rel_rms * rms + (half_ulp_bf16(ref) if bf16_out else 0.0)
+    bad = np.abs(d) > allow
+    assert fro <= rel_fro, f"{what}: rel-Frobenius {fro:.3e} > {rel_fro}"
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond the bound; worst |d|="
+                           f"{np.abs(d).max():.3e}, rms(ref)={rms:.3e}")
+    return fro, float(np.abs(d).max()), rms
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().float().numpy().astype(np.float64)
+
+
+def shape_of(cfg: dict) -> dict:
+    return {k: cfg[k] for k in ("H", "I", "Nr", "Kr", "Ns", "n_groups", "topk_groups") if k in cfg}
+
+
+def oracle_cfg(oracle, cfg: dict):
+    return oracle.cfg(cfg["H"], cfg["I"], cfg["Nr"], cfg["Kr"], cfg.get("Ns", 1), cfg.get("n_groups", 0),
+                      cfg.get("topk_groups", 0), cfg.get("route_scale", 1.0))
+
+
+def route_sets_match(idx_gpu: np.ndarray, idx_ref: np.ndarray, gap: np.ndarray):
+    """Bit-exact routing up to near-ties: returns (mismatching tokens that are
+    not exempt, number of exempt tokens)."""
+    exempt = gap < NEAR_TIE
+    bad = []
+    for t in range(idx_ref.shape[0]):
+        if exempt[t]:
+            continue
+        if set(idx_gpu[t].tolist()) != set(idx_ref[t].tolist()):
+            bad.append(t)
+    return bad, int(exempt.sum())
+
+
+class Problem:
+    """Seeded synthetic layer problem: bf16 inputs shared by the CUDA path
+    and the oracle (which quantizes the weights itself)."""
+
+    def __init__(self, cfg: dict, T: int, seed: int = 0, device="cpu", x_kind=None):
+        self.cfg = dict(cfg)
+        self.T = T
+        self.seed = seed
+        self.device = device
+        H, Nr = cfg["H"], cfg["Nr"]
+        kind = x_kind or cfg.get("x", "normal")
+        if kind == "mixture":
+            self.x, _ = S.gen_mixture_x(T, H, seed, device=device)
+        else:
+            self.x = S.gen_x(T, H, seed, device=device)
+        self.wr = S.gen_router(Nr, H, seed, device=device)
+        self.bias = S.gen_bias(Nr, seed, cfg.get("bias", "uniform"), device=device)
+        self.E = Nr + cfg.get("Ns", 1)
+
+    def expert_bf16(self, e: int):
+        return S.gen_expert(e, self.cfg["H"], self.cfg["I"], self.seed, device=self.device)
+
+    def oracle_expert(self, oracle, e: int):
+        w13, w2 = self.expert_bf16(e)
+        W13q, s13 = oracle.quant_128x128(w13)
+        W2q, s2 = oracle.quant_128x128(w2)
+        return W13q, s13, W2q, s2

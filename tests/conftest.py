@@ -13,6 +13,20 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: long-running (full-size workloads)")
 
 
+def _build_library():
+    """Compile libmoefp8.so if its sources changed (by path: importing the
+    package needs the library)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_moe_build", os.path.join(ROOT, "sparse_moe_layer_expert_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+_build_library()
+
+
 @pytest.fixture(scope="session")
 def oracle_lib():
     import oracle

@@ -1,0 +1,81 @@
+"""The C-ABI library loads without a GPU, exports every entry point that
+include/moe_fp8.h declares, and validates arguments on the host (no compute
+call is made here)."""
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_fp8.h")
+
+
+@pytest.fixture(scope="module")
+def m():
+    import sparse_moe_layer_expert_b200 as pkg
+    return pkg
+
+
+def declared_functions():
+    txt = open(HEADER).read()
+    return re.findall(r"^MOE_API\s+[a-z_ 0-9]+?\**\s*([a-z_0-9]+)\(", txt, flags=re.M)
+
+
+def test_every_declared_symbol_is_exported(m):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(m.lib, n), n
+    assert set(names) == set(m.EXPORTS)
+
+
+def test_status_strings_and_version(m):
+    assert m.lib.moe_abi_version() == 100
+    assert m.lib.moe_status_string(0) == b"ok"
+    assert b"128" in m.lib.moe_status_string(m.MOE_ERR_UNSUPPORTED_SHAPE)
+    assert m.lib.moe_status_string(12345) == b"unknown status"
+
+
+def test_host_validation_without_device(m):
+    L = m.lib
+    # shape errors are reported before any device query
+    assert L.fp8_quant_1x128(None, 4, 100, 128, None, None, None) == m.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.fp8_quant_1x128(None, 4, 128, 100, None, None, None) == m.MOE_ERR_INVALID_ARG
+    assert L.fp8_quant_1x128(None, 0, 128, 128, None, None, None) == m.MOE_OK  # empty: nothing enqueued
+    assert L.fp8_quant_128x128(None, 100, 128, None, None, None) == m.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.fp8_blockscaled_gemm(None, None, None, None, None, 4, 100, 128, None, None) == m.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.fp8_blockscaled_gemm(None, None, None, None, None, 4, 128, 128, None, None) == m.MOE_ERR_INVALID_ARG
+    bad = m.config(7168, 2000, 256, 8)
+    assert m.moe_workspace_size(bad, 64) == 0
+    import ctypes as C
+    assert L.moe_forward(C.byref(bad), None, None, None, 64, None, 0, None, None, None, 0, None, None) == \
+        m.MOE_ERR_UNSUPPORTED_SHAPE
+    cfg = m.config(512, 256, 16, 4)
+    assert L.moe_forward(C.byref(cfg), None, None, None, 64, None, 7, None, None, None, 0, None, None) == \
+        m.MOE_ERR_INVALID_ARG
+    # too many experts per token / groups that cannot hold top_k
+    assert m.moe_workspace_size(m.config(512, 256, 16, 17), 8) == 0
+    assert m.moe_workspace_size(m.config(512, 256, 16, 5, 1, 4, 1), 8) == 0
+    # a valid call with non-null pointers reaches the device check
+    assert L.fp8_quant_1x128(16, 4, 128, 128, 16, 16, None) == m.MOE_ERR_NO_DEVICE
+
+
+def test_workspace_layout_is_disjoint_and_aligned(m):
+    for (H, I, Nr, Kr, T) in [(512, 256, 16, 4, 256), (7168, 2048, 256, 8, 64), (7168, 2048, 256, 8, 4096),
+                              (7168, 2048, 256, 8, 16384), (512, 256, 16, 4, 1)]:
+        cfg = m.config(H, I, Nr, Kr)
+        L = m.moe_workspace_layout(cfg, T)
+        spans = sorted(v for k, v in L.items() if k != "total")
+        for (o, n) in spans:
+            assert o % 256 == 0
+        for (o1, n1), (o2, _) in zip(spans, spans[1:]):
+            assert o1 + n1 <= o2
+        assert spans[-1][0] + spans[-1][1] <= L["total"] == m.moe_workspace_size(cfg, T)
+        R = T * Kr
+        assert L["ap"][1] == R * H and L["y"][1] == (R + T) * H * 4 and L["hq"][1] == (R + T) * I
+
+
+def test_route_workspace_size(m):
+    cfg = m.config(7168, 2048, 256, 8)
+    assert m.moe_route_workspace_size(cfg, 4096) >= 4096 * 256 * 4
+    assert m.moe_route_workspace_size(cfg, 0) >= 0

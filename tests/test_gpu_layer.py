@@ -1,0 +1,202 @@
+"""GPU parity of the whole layer forward (moe_forward) against the oracle,
+step by step through the workspace intermediates, on the small configuration
+and its edge cases ("DeepSeek-V3 Technischer Bericht", Methode section 2 and
+the Kernideen FP8 recipe).
+
+Checked per step: quantized input (bit-exact), routing (bit-exact up to
+near-ties), counts and expert offsets (exact), expert-contiguous rows
+(exact, stable order), re-quantized SwiGLU output (tolerance), gate-scaled
+expert outputs (FP32, tolerance), layer output in FP32 (tolerance) and bf16
+(tolerance plus bf16 rounding; and exactly the RNE of the FP32 result)."""
+import numpy as np
+import pytest
+import torch
+
+import moe_synth as S
+from _moe_util import NEAR_TIE, Problem, assert_close, bf16_to_f64, oracle_cfg, route_sets_match, shape_of
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def m():
+    import sparse_moe_layer_expert_b200 as pkg
+    return pkg
+
+
+def build_gpu_layer(m, prob: Problem):
+    shape = shape_of(prob.cfg)
+    layer = m.MoeLayer(shape, "cuda")
+    for e in range(prob.E):
+        w13, w2 = prob.expert_bf16(e)
+        layer.set_expert(e, w13.cuda(), w2.cuda())
+    layer.set_router(prob.wr.cuda(), prob.bias.cuda())
+    return layer
+
+
+def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts=None, check_weights=True):
+    """Run moe_forward on all T tokens; compare every intermediate for the
+    listed tokens (all when None) against the oracle."""
+    cfg, T = prob.cfg, prob.T
+    H, I, Nr, Kr, Ns = cfg["H"], cfg["I"], cfg["Nr"], cfg["Kr"], cfg.get("Ns", 1)
+    R = T * Kr
+    x_d = prob.x.to("cuda")
+    counts_out = torch.empty(Nr, dtype=torch.int32, device="cuda")
+    idx_out = torch.empty((T, Kr), dtype=torch.int32, device="cuda")
+    out32 = layer.forward(x_d, out_dtype=m.MOE_DTYPE_F32, idx_out=idx_out, counts_out=counts_out)
+    layer.check()
+    ws = layer.workspace(T)
+    L = layer.layout(T)
+    v = lambda name, dt, shp: m.ws_view(ws, L, name, dt, shp).cpu().numpy()  # noqa: E731
+    xq, xs = v("xq", torch.uint8, (T, H)), v("xs", torch.float32, (T, H // 128))
+    idx, gate = v("idx", torch.int32, (T, Kr)), v("gate", torch.float32, (T, Kr))
+    offsets, pos = v("offsets", torch.int32, (Nr + 1,)), v("pos", torch.int32, (T, Kr))
+    ap, as_ = v("ap", torch.uint8, (R, H)), v("as", torch.float32, (R, H // 128))
+    hq, hs = v("hq", torch.uint8, (R + T * Ns, I)), v("hs", torch.float32, (R + T * Ns, I // 128))
+    y = v("y", torch.float32, (R + T * Ns, H))
+    counts = counts_out.cpu().numpy()
+    assert np.array_equal(idx_out.cpu().numpy(), idx)
+
+    tok = np.arange(T) if tokens is None else np.asarray(tokens)
+    # S1: quantized input, bit-exact
+    xq_o, xs_o = oracle_lib.quant_1x128(prob.x)
+    assert np.array_equal(xq, xq_o) and np.array_equal(xs, xs_o)
+    # S2: routing (oracle routes all tokens; cheap relative to the FFNs)
+    ocf = oracle_cfg(oracle_lib, cfg)
+    oi, og, gap, _ = oracle_lib.route(ocf, prob.x, prob.wr, prob.bias)
+    bad, n_exempt = route_sets_match(idx, oi, gap)
+    assert not bad, f"routing differs on {len(bad)} tokens"
+    assert n_exempt <= max(1, T // 1000)
+    assert np.allclose(gate.sum(1), 1.0, atol=2e-6)
+    # S3: counts, offsets, stable expert-contiguous order
+    assert np.array_equal(counts, np.bincount(idx.reshape(-1), minlength=Nr))
+    if n_exempt == 0:
+        assert np.array_equal(counts, oracle_lib.histogram(oi, Nr))
+    off_o, order = oracle_lib.expert_order(idx, Nr)
+    assert np.array_equal(offsets, off_o)
+    pos_o = np.empty(R, np.int64)
+    pos_o[order] = np.arange(R)
+    assert np.array_equal(pos.reshape(-1), pos_o)
+    src_t = order // Kr
+    assert np.array_equal(ap, xq_o[src_t]) and np.array_equal(as_, xs_o[src_t])
+    # weights quantized on the GPU are the oracle's, bit for bit
+    experts = oracle_experts if oracle_experts is not None else {}
+    need = set(int(e) for t in tok for e in idx[t]) | set(int(e) for t in tok for e in oi[t])
+    need |= set(range(Nr, Nr + Ns))
+    for e in sorted(need):
+        if e not in experts:
+            experts[e] = prob.oracle_expert(oracle_lib, e)
+        if check_weights:
+            W13q, s13, W2q, s2 = experts[e]
+            assert np.array_equal(layer.w13[e].cpu().numpy(), W13q)
+            assert np.array_equal(layer.s13[e].cpu().numpy(), s13)
+            assert np.array_equal(layer.w2[e].cpu().numpy(), W2q)
+            assert np.array_equal(layer.s2[e].cpu().numpy(), s2)
+    # S4-S6: per (token, expert) FFN pieces
+    hq_got, hs_got, hq_ref, hs_ref, h_ref, y_got, y_ref = [], [], [], [], [], [], []
+    for t in tok:
+        rows = [(int(pos[t, k]), int(idx[t, k]), float(gate[t, k])) for k in range(Kr)]
+        if Ns:
+            rows.append((R + int(t), Nr, 1.0))
+        for p, e, g in rows:
+            yo, ho, hqo, hso = oracle_lib.expert_ffn(ocf, xq[t:t + 1], xs[t:t + 1], *experts[e], want_h=True)
+            hq_got.append(hq[p])
+            hs_got.append(hs[p])
+            hq_ref.append(hqo[0])
+            hs_ref.append(hso[0])
+            h_ref.append(ho[0])
+            y_got.append(y[p].astype(np.float64))
+            y_ref.append(g * yo[0])
+    check_requantized(oracle_lib, np.stack(hq_got), np.stack(hs_got), np.stack(hq_ref), np.stack(hs_ref),
+                      np.stack(h_ref))
+    assert_close(np.stack(y_got), np.stack(y_ref), what="gate-scaled expert outputs y")
+    # S7: layer output (near-tie tokens may legitimately pick another expert)
+    tok = tok[gap[tok] >= NEAR_TIE]
+    res = oracle_lib.forward(ocf, prob.x, prob.wr, prob.bias,
+                             [experts.get(e) for e in range(Nr + Ns)], tokens=tok)
+    assert np.array_equal(res["idx"], oi[tok])
+    o32 = out32.cpu().numpy()[tok].astype(np.float64)
+    assert_close(o32, res["out"], what="layer output (fp32)")
+    out16 = layer.forward(x_d, out_dtype=m.MOE_DTYPE_BF16)
+    layer.check()
+    o16 = out16.cpu()[torch.as_tensor(tok)]
+    assert_close(bf16_to_f64(o16), res["out"], bf16_out=True, what="layer output (bf16)")
+    assert torch.equal(o16, out32.cpu()[torch.as_tensor(tok)].to(torch.bfloat16))
+    return dict(counts=counts, idx=idx, n_exempt=n_exempt)
+
+
+def check_requantized(oracle_lib, hq, hs, hq_o, hs_o, h_o):
+    """The GPU's 1x128 re-quantization of h against the oracle's: scales
+    agree to FP32 rounding of amax; codes are equal except where the oracle's
+    own quotient h/S sits on the rounding midpoint between the GPU's code and
+    its own (h itself differs in its last bits between the two sides)."""
+    assert np.allclose(hs, hs_o, rtol=2e-6, atol=0), "re-quantization scales"
+    diff = hq != hq_o
+    assert diff.mean() < 1e-3, f"{diff.mean():.2e} of the re-quantized codes differ"
+    if diff.any():
+        dq = oracle_lib.e4m3_decode_table()
+        r, c = np.nonzero(diff)
+        a, b = dq[hq[r, c]], dq[hq_o[r, c]]
+        quot = h_o[r, c].astype(np.float64) / np.repeat(hs_o, 128, axis=1)[r, c]
+        mid = (a + b) / 2
+        # adjacent codes (same sign) and the quotient within 1e-4 of their midpoint
+        assert np.all(np.sign(a) * np.sign(b) >= 0)
+        assert np.all(np.abs(quot - mid) <= 1e-4 * np.maximum(np.abs(mid), 2.0 ** -9)), "code differs off a tie"
+        vals = np.unique(dq[np.isfinite(dq)])
+        assert np.all(np.abs(np.searchsorted(vals, a) - np.searchsorted(vals, b)) == 1), "non-adjacent codes"
+
+
+def test_layer_tiny(m, oracle_lib):
+    prob = Problem(S.TINY, 256, seed=0)
+    check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob))
+
+
+@pytest.mark.parametrize("T", [1, 2, 129])
+def test_layer_tiny_ragged_token_counts(m, oracle_lib, T):
+    prob = Problem(S.TINY, T, seed=T)
+    check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob))
+
+
+def test_layer_no_shared_expert(m, oracle_lib):
+    prob = Problem(dict(S.TINY, Ns=0), 100, seed=3)
+    check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob))
+
+
+def test_layer_all_experts_selected(m, oracle_lib):
+    prob = Problem(dict(S.TINY, Kr=16), 64, seed=4)
+    check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob))
+
+
+def test_layer_group_limited_skewed(m, oracle_lib):
+    prob = Problem(dict(S.TINY, n_groups=4, topk_groups=2), 512, seed=5, x_kind="mixture")
+    r = check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob), tokens=np.arange(0, 512, 7))
+    assert r["counts"].max() > 1.5 * r["counts"].mean()  # the mixture input skews the load
+
+
+def test_layer_wider_hidden_and_many_chunks(m, oracle_lib):
+    # one expert receives > 128 rows (several chunks), H/128 odd (single-block
+    # down-projection tile), I/128 = 3
+    cfg = dict(S.TINY, H=640, I=384, Nr=8, Kr=2)
+    prob = Problem(cfg, 700, seed=6)
+    check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob), tokens=np.arange(0, 700, 11))
+
+
+def test_bias_update_matches_oracle(m, oracle_lib):
+    prob = Problem(S.TINY, 256, seed=7)
+    layer = build_gpu_layer(m, prob)
+    counts = torch.empty(16, dtype=torch.int32, device="cuda")
+    layer.forward(prob.x.cuda(), counts_out=counts)
+    b0 = layer.bias.cpu().numpy().copy()
+    layer.bias_update(counts, 256, 0.001)
+    torch.cuda.synchronize()
+    want = oracle_lib.bias_update(b0, counts.cpu().numpy(), 16, 256 * 4, 0.001)
+    assert np.array_equal(layer.bias.cpu().numpy(), want)
+
+
+def test_forward_rejects_small_workspace(m):
+    prob = Problem(S.TINY, 8, seed=8)
+    layer = build_gpu_layer(m, prob)
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(m.MoeError) as e:
+        m.moe_forward(layer.cfg, layer.weights(), layer.bias, prob.x.cuda(), ws=ws, err=layer.err)
+    assert e.value.status == m.MOE_ERR_WORKSPACE_TOO_SMALL

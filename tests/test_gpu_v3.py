@@ -1,0 +1,68 @@
+"""Full-size parity: the DeepSeek-V3-shaped layer (hidden 7168, intermediate
+2048, 256 routed + 1 shared experts, top-8) in the launch configuration the
+benchmark times.  Quantization, routing, counts, grouping and weights are
+checked over the whole batch; the expert FFNs and the layer output on a seeded
+sample of tokens the double-precision oracle computes one by one."""
+import numpy as np
+import pytest
+import torch
+
+import moe_synth as S
+from _moe_util import Problem
+from test_gpu_layer import check_layer
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def m():
+    import sparse_moe_layer_expert_b200 as pkg
+    return pkg
+
+
+@pytest.fixture(scope="module")
+def v3_layer(m):
+    """One GPU-resident V3 layer (weights generated on the GPU per expert,
+    quantized by the library), shared by the full-size tests."""
+    cfg = dict(S.PREFILL)
+    shape = {k: cfg[k] for k in ("H", "I", "Nr", "Kr", "Ns")}
+    seed = 0
+
+    def gen(e):
+        return S.gen_expert(e, cfg["H"], cfg["I"], seed, device="cuda")
+
+    wr = S.gen_router(cfg["Nr"], cfg["H"], seed, device="cuda")
+    bias = S.gen_bias(cfg["Nr"], seed, "uniform", device="cuda")
+    layer = m.MoeLayer.from_generator(shape, gen, wr, bias)
+    torch.cuda.synchronize()
+    return layer, seed
+
+
+def _problem(cfg, T, seed, layer, bias_kind):
+    prob = Problem(cfg, T, seed=seed, device="cuda")
+    # the layer's weights and router come from seed 0; only x differs per test
+    prob.seed = 0
+    prob.wr = layer.wr
+    prob.bias = layer.bias.clone()
+    if bias_kind == "zero":
+        prob.bias.zero_()
+    layer.bias.copy_(prob.bias)
+    prob.x = S.gen_x(T, cfg["H"], seed, device="cuda")
+    return prob
+
+
+def test_v3_decode_layer(m, oracle_lib, v3_layer):
+    layer, _ = v3_layer
+    prob = _problem(dict(S.DECODE), 64, 11, layer, "zero")
+    r = check_layer(m, oracle_lib, prob, layer, tokens=np.array([0, 9, 31, 63]), check_weights=True)
+    assert r["counts"].sum() == 64 * 8
+
+
+def test_v3_prefill_layer(m, oracle_lib, v3_layer):
+    layer, _ = v3_layer
+    prob = _problem(dict(S.PREFILL), 4096, 12, layer, "uniform")
+    rng = np.random.default_rng(12)
+    toks = np.sort(rng.choice(4096, 4, replace=False))
+    r = check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=False)
+    c = r["counts"]
+    print(f"prefill load: max {c.max()} mean {c.mean():.1f} min {c.min()} empty {(c == 0).sum()}")
