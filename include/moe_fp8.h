@@ -173,6 +173,32 @@ MOE_API int moe_route(const moe_config *cfg, const void *x_dev, const void *wr_d
               int64_t T, int32_t *idx_dev, float *gate_dev, int32_t *counts_dev, void *ws_dev,
               size_t ws_bytes, int32_t *err_flag_dev, void *stream);
 
+/* Allocation-free variant of moe_route (the pages have no counterpart: this
+ * is an interface convenience).  Some callers cannot call cudaMalloc or hand
+ * the library a scratch buffer -- e.g. a host that owns every byte of device
+ * memory through its own planner, or a latency-critical path where an
+ * allocation's implicit device synchronisation is not acceptable.  This entry
+ * point takes the same inputs and outputs as moe_route but keeps the router's
+ * FP32 logit partials in a fixed scratch array inside the library
+ * (MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 16 MiB on every GPU that loads the
+ * library, held until the process exits) and allocates nothing.
+ *   - Limit: the partials moe_route would keep in its workspace must fit,
+ *     i.e. moe_route_workspace_size(cfg, T) - 256 <= 16 MiB (for
+ *     n_routed = 256 every T <= 8192 fits); larger calls return
+ *     MOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
+ *   - The first call on a device looks up the scratch's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Every call shares the one scratch and it keeps the last call's
+ *     contents (each call overwrites every partial it reads, so nothing has
+ *     to start at zero); calls whose execution overlaps on the GPU race on
+ *     it, so serialise them (one stream, or events).
+ * Arguments, outputs and error behaviour are otherwise those of moe_route. */
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (16u << 20)
+MOE_API int moe_route_noalloc(const moe_config *cfg, const void *x_dev, const void *wr_dev,
+                              const float *bias_dev, int64_t T, int32_t *idx_dev, float *gate_dev,
+                              int32_t *counts_dev, int32_t *err_flag_dev, void *stream);
+
 /* ------------------------------------------------------------ full layer */
 /* One DeepSeekMoE layer forward ([P4] Methode 2):
  *   out[t] = u_t + sum_{shared} FFN_s(u_t) + sum_k gate[t, k] FFN_{idx[t,k]}(u_t)

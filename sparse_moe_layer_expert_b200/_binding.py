@@ -39,7 +39,9 @@ EXPORTS = (
     "moe_status_string", "moe_abi_version", "fp8_quant_1x128", "fp8_quant_128x128", "fp8_blockscaled_gemm",
     "moe_route_workspace_size", "moe_route", "moe_workspace_size", "moe_forward", "moe_workspace_layout",
     "moe_bias_update", "moe_check_device_error", "moe_selftest_wait_timeout", "moe_profile_events",
+    "moe_route_noalloc",
 )
+MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 16 << 20
 MOE_PROFILE_EVENTS = 7
 PROFILE_STAGES = ("quantize", "route", "group", "gemm_gate_up", "gemm_down", "combine")
 
@@ -74,6 +76,7 @@ lib.fp8_blockscaled_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, 
 lib.moe_route_workspace_size.restype = _sz
 lib.moe_route_workspace_size.argtypes = [_cfgp, _i64]
 lib.moe_route.argtypes = [_cfgp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
+lib.moe_route_noalloc.argtypes = [_cfgp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp]
 lib.moe_workspace_size.restype = _sz
 lib.moe_workspace_size.argtypes = [_cfgp, _i64]
 lib.moe_forward.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _sz, _vp, _vp]
@@ -167,6 +170,14 @@ def moe_route(cfg: MoeConfig, x, wr, bias, idx=None, gate=None, counts=None, ws=
     err = new_err_flag(dev) if err is None else err
     _check(lib.moe_route(C.byref(cfg), _ptr(x), _ptr(wr), _ptr(bias), T, _ptr(idx), _ptr(gate), _ptr(counts),
                          _ptr(ws), ws.numel(), _ptr(err), _stream(stream)), "moe_route")
+    return idx, gate, counts
+
+
+def moe_route_noalloc(cfg: MoeConfig, x, wr, bias, idx, gate, counts, err, stream=None):
+    """moe_route with the library's fixed scratch; outputs must be supplied
+    (this call is for callers that allocate nothing on the call path)."""
+    _check(lib.moe_route_noalloc(C.byref(cfg), _ptr(x), _ptr(wr), _ptr(bias), x.shape[0], _ptr(idx), _ptr(gate),
+                                 _ptr(counts), _ptr(err), _stream(stream)), "moe_route_noalloc")
     return idx, gate, counts
 
 

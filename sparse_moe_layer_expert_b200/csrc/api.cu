@@ -263,6 +263,34 @@ int moe_route(const moe_config *cfg, const void *x, const void *wr, const float 
   return cuda_status(e);
 }
 
+int moe_route_noalloc(const moe_config *cfg, const void *x, const void *wr, const float *bias, int64_t T,
+                      int32_t *idx, float *gate, int32_t *counts, int32_t *err_flag, void *stream) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
+  if (!counts) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if (const int d = check_device()) return d;
+    return cuda_status(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_routed, st));
+  }
+  if (!x || !wr || !bias || !idx || !gate || !err_flag) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(wr)) return MOE_ERR_INVALID_ARG;
+  const int ks = moe::router_ksplit(T, cfg->n_routed, cfg->hidden);
+  if (static_cast<size_t>(ks) * static_cast<size_t>(T) * cfg->n_routed > moe::kRouteNoAllocScratchFloats)
+    return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (const int d = check_device()) return d;
+  float *partial = nullptr;
+  cudaError_t e = moe::route_static_scratch(&partial);
+  if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_routed, st);
+  if (e == cudaSuccess)
+    e = moe::launch_router_logits(x, wr, T, cfg->n_routed, cfg->hidden, partial, err_flag,
+                                  moe::kDefaultWaitLimitNs, st);
+  if (e == cudaSuccess)
+    e = moe::launch_router_topk(partial, ks, T, cfg->n_routed, cfg->top_k, cfg->n_groups, cfg->topk_groups,
+                                cfg->route_scale, bias, idx, gate, counts, st);
+  return cuda_status(e);
+}
+
 size_t moe_workspace_size(const moe_config *cfg, int64_t T) {
   if (check_cfg(cfg) != MOE_OK || T < 0 || T > kMaxTokens) return 0;
   moe_ws_layout L;

@@ -61,6 +61,9 @@ cudaError_t launch_quant_1x128(const void *x, int64_t rows, int64_t cols, int64_
 cudaError_t launch_quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *s, cudaStream_t st);
 
 int router_ksplit(int64_t T, int Nr, int H);
+// capacity of the fixed router scratch used by moe_route_noalloc (floats)
+constexpr size_t kRouteNoAllocScratchFloats = size_t(4) << 20;
+cudaError_t route_static_scratch(float **ptr);
 cudaError_t launch_router_logits(const void *x, const void *wr, int64_t T, int Nr, int H, float *partial,
                                  int32_t *err, uint64_t limit_ns, cudaStream_t st);
 cudaError_t launch_router_topk(const float *partial, int n_ks, int64_t T, int Nr, int Kr, int n_groups,

@@ -13,6 +13,8 @@
 //  2. router_topk_kernel: one warp per token; each lane holds the experts
 //     lane, lane+32, ... in registers; sigmoid, bias, optional group
 //     pre-selection and K_r rounds of warp-wide argmax.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -293,6 +295,36 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float *__restric
     gate[t * Kr + lane] = route_scale * (sel_s / ssum);
     if (counts && sel_e >= 0 && sel_e < Nr) atomicAdd(&counts[sel_e], 1);
   }
+}
+
+// ------------------------------------------------ fixed scratch (no allocation)
+// Scratch of moe_route_noalloc: the router's FP32 logit partials live in this
+// file-scope array instead of a caller buffer.  Every GPU that loads the
+// library holds it (16 MiB) until the process exits, and all calls share it.
+static __device__ __align__(256) float g_route_scratch[kRouteNoAllocScratchFloats];
+
+namespace {
+std::mutex g_scratch_mu;
+float *g_scratch_ptr[64] = {nullptr};
+}  // namespace
+
+// Device address of g_route_scratch for the current device.  The first call on
+// a device looks it up with cudaGetSymbolAddress (with that device current)
+// and caches it; host code must never pass the array's host-side name itself.
+cudaError_t route_static_scratch(float **ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = static_cast<float *>(p);
+  }
+  *ptr = g_scratch_ptr[dev];
+  return cudaSuccess;
 }
 
 int router_ksplit(int64_t T, int Nr, int H) {
