@@ -234,17 +234,18 @@ typedef struct {
     size_t offsets[2];  /* int32 [N_r + 1]  first row of each expert           */
     size_t pos[2];      /* int32 [T, K_r]   row of (t, k) in expert order      */
     size_t ap[2];       /* E4M3 [R, H]      expert-contiguous copy of xq rows  */
-    size_t as[2];       /* float [R, H/128]                                    */
+    size_t as[2];       /* float [H/128, R + T] scales of every row, transposed */
     size_t row_gate[2]; /* float [R + T*N_s] gate of each row (1 for shared)   */
+    size_t row_src[2];  /* int32 [R]        token of each routed row           */
     size_t hq[2];       /* E4M3 [R + T*N_s, I] re-quantized SwiGLU output      */
-    size_t hs[2];       /* float [R + T*N_s, I/128]                            */
+    size_t hs[2];       /* float [I/128, R + T] its scales, transposed         */
     size_t y[2];        /* float [R + T*N_s, H] gate-scaled expert outputs     */
-    size_t ntiles[2];   /* int32 [4]: tiles of the two grouped GEMMs, rows, chunks */
+    size_t meta[2];     /* int32 [4]: number of chunks, routed rows            */
     size_t logits[2];   /* float [S, T, N_r] router logit partials (S K-splits) */
     size_t blk_hist[2]; /* int32 [ceil(T/128), N_r] per-block expert counts    */
     size_t blk_base[2]; /* int32 [ceil(T/128), N_r] per-block first rows       */
-    size_t tiles1[2];   /* work list of the gate/up GEMM (32-byte entries)     */
-    size_t tiles2[2];   /* work list of the down GEMM                          */
+    size_t chunks[2];   /* int32x4 per chunk: {expert | input flag << 16,
+                           activation row, output row, rows <= 128}            */
     size_t total;
 } moe_ws_layout;
 MOE_API int moe_workspace_layout(const moe_config *cfg, int64_t T, moe_ws_layout *layout);

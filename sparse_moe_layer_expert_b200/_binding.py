@@ -57,8 +57,8 @@ class MoeWeights(C.Structure):
                 ("s2_dev", C.c_void_p), ("wr_dev", C.c_void_p)]
 
 
-_LAYOUT_FIELDS = ("xq", "xs", "idx", "gate", "counts", "offsets", "pos", "ap", "as", "row_gate", "hq", "hs", "y",
-                  "ntiles", "logits", "blk_hist", "blk_base", "tiles1", "tiles2")
+_LAYOUT_FIELDS = ("xq", "xs", "idx", "gate", "counts", "offsets", "pos", "ap", "as", "row_gate", "row_src", "hq",
+                  "hs", "y", "meta", "logits", "blk_hist", "blk_base", "chunks")
 
 
 class MoeWsLayout(C.Structure):

@@ -66,7 +66,6 @@ int sm_count() {
 
 namespace {
 
-using moe::GemmTile;
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -126,17 +125,17 @@ void make_layout(const moe_config *c, int64_t T, moe_ws_layout *L) {
   cv.take(L->offsets, (Nr + 1) * 4);
   cv.take(L->pos, T * Kr * 4);
   cv.take(L->ap, R * H);
-  cv.take(L->as, R * (H / 128) * 4);
+  cv.take(L->as, (H / 128) * (R + T) * 4);
   cv.take(L->row_gate, RS * 4);
+  cv.take(L->row_src, R * 4);
   cv.take(L->hq, RS * I);
-  cv.take(L->hs, RS * (I / 128) * 4);
+  cv.take(L->hs, (I / 128) * (R + T) * 4);
   cv.take(L->y, RS * H * 4);
-  cv.take(L->ntiles, 4 * 4);
+  cv.take(L->meta, 4 * 4);
   cv.take(L->logits, ks * T * Nr * 4);
   cv.take(L->blk_hist, nblk * Nr * 4);
   cv.take(L->blk_base, nblk * Nr * 4);
-  cv.take(L->tiles1, chunks * moe::gemm1_blocks(static_cast<int>(I)) * sizeof(GemmTile));
-  cv.take(L->tiles2, chunks * moe::gemm2_blocks(static_cast<int>(H)) * sizeof(GemmTile));
+  cv.take(L->chunks, chunks * 16);
   L->total = (cv.off + 255) & ~size_t(255);
 }
 
@@ -215,12 +214,14 @@ int fp8_blockscaled_gemm(const uint8_t *A, const float *sA, const uint8_t *B, co
   g.sw = sB;
   g.sa0 = sA;
   g.sa1 = sA;
-  g.tiles = nullptr;
-  g.n_tiles = nullptr;
+  g.sa_transposed = 0;
+  g.chunks = nullptr;
+  g.n_chunks = nullptr;
   g.dense_M = M;
-  const int64_t tiles = ((M + 127) / 128) * ((N / 128 + 1) / 2);
-  if (tiles > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
-  g.max_tiles = static_cast<int>(tiles);
+  g.max_chunks = static_cast<int>((M + 127) / 128);
+  g.nb = static_cast<int>((N / 128 + 1) / 2);
+  g.gate_up = 0;
+  g.rows_per_expert = N;
   g.epi = moe::EPI_BF16;
   g.out = C;
   g.ldo = N;
@@ -340,19 +341,19 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
   int32_t *offsets = at<int32_t *>(ws, L.offsets);
   int32_t *pos = at<int32_t *>(ws, L.pos);
   uint8_t *ap = at<uint8_t *>(ws, L.ap);
-  float *as = at<float *>(ws, L.as);
+  float *as_t = at<float *>(ws, L.as);
   float *row_gate = at<float *>(ws, L.row_gate);
+  int32_t *row_src = at<int32_t *>(ws, L.row_src);
   uint8_t *hq = at<uint8_t *>(ws, L.hq);
-  float *hs = at<float *>(ws, L.hs);
+  float *hs_t = at<float *>(ws, L.hs);
   float *y = at<float *>(ws, L.y);
-  int32_t *ntiles = at<int32_t *>(ws, L.ntiles);
+  int32_t *meta = at<int32_t *>(ws, L.meta);
   float *logits = at<float *>(ws, L.logits);
   int32_t *blk_hist = at<int32_t *>(ws, L.blk_hist);
   int32_t *blk_base = at<int32_t *>(ws, L.blk_base);
-  GemmTile *tiles1 = at<GemmTile *>(ws, L.tiles1);
-  GemmTile *tiles2 = at<GemmTile *>(ws, L.tiles2);
+  int4 *chunks = at<int4 *>(ws, L.chunks);
   const int ks = moe::router_ksplit(T, Nr, H);
-  const int64_t chunks = moe::max_chunks(T, Kr, Nr, Ns);
+  const int64_t max_chunks = moe::max_chunks(T, Kr, Nr, Ns);
 
   cudaError_t e = prof_mark(0, st);
   if (e == cudaSuccess) e = moe::launch_quant_1x128(x, T, H, H, xq, xs, st);
@@ -365,10 +366,9 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
   if (e == cudaSuccess) e = prof_mark(2, st);
   if (e == cudaSuccess) e = moe::launch_hist(idx, T, Kr, Nr, blk_hist, err_flag, st);
   if (e == cudaSuccess)
-    e = moe::launch_build_tiles(blk_hist, T, Kr, Nr, Ns, H, I, counts, offsets, blk_base, tiles1, tiles2, ntiles,
-                                counts_out, st);
-  if (e == cudaSuccess)
-    e = moe::launch_scatter(idx, gate, xq, xs, T, Kr, Nr, Ns, H, blk_base, ap, as, row_gate, pos, st);
+    e = moe::launch_build_chunks(blk_hist, T, Kr, Nr, Ns, counts, offsets, blk_base, chunks, meta, counts_out, st);
+  if (e == cudaSuccess) e = moe::launch_rank(idx, gate, T, Kr, Nr, Ns, blk_base, row_gate, row_src, pos, st);
+  if (e == cudaSuccess) e = moe::launch_copy_rows(xq, xs, row_src, R, T, Ns, H, ap, as_t, st);
   if (e == cudaSuccess) e = prof_mark(3, st);
   if (e == cudaSuccess) {
     // gate/up projection + SwiGLU + 1x128 requantization
@@ -381,19 +381,24 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
     g.a1_rows = T;
     g.K = H;
     g.sw = w->s13_dev;
-    g.sa0 = as;
-    g.sa1 = xs;
-    g.tiles = tiles1;
-    g.n_tiles = ntiles;
-    g.tile_slot = 0;
-    g.max_tiles = static_cast<int>(chunks * moe::gemm1_blocks(I));
+    g.sa0 = as_t;
+    g.sa1 = as_t;
+    g.sa_transposed = 1;
+    g.sa_ld = R + T;
+    g.chunks = chunks;
+    g.n_chunks = meta;
+    g.max_chunks = static_cast<int>(max_chunks);
+    g.nb = moe::gemm1_blocks(I);
+    g.gate_up = 1;
+    g.half = I;
+    g.rows_per_expert = 2 * static_cast<int64_t>(I);
     g.epi = moe::EPI_SWIGLU_Q;
     g.out = hq;
     g.ldo = I;
     g.out_rows = RS;
     g.out_cols = 2 * I;  // block B (up) shares block A's output columns
-    g.out_scale = hs;
-    g.ld_os = I / 128;
+    g.out_scale = hs_t;
+    g.ld_os = R + T;
     g.err = err_flag;
     g.wait_limit_ns = moe::kDefaultWaitLimitNs;
     e = moe::launch_gemm(g, st);
@@ -410,12 +415,17 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
     g.a1_rows = RS;
     g.K = I;
     g.sw = w->s2_dev;
-    g.sa0 = hs;
-    g.sa1 = hs;
-    g.tiles = tiles2;
-    g.n_tiles = ntiles;
-    g.tile_slot = 1;
-    g.max_tiles = static_cast<int>(chunks * moe::gemm2_blocks(H));
+    g.sa0 = hs_t;
+    g.sa1 = hs_t;
+    g.sa_transposed = 1;
+    g.sa_ld = R + T;
+    g.chunks = chunks;
+    g.n_chunks = meta;
+    g.max_chunks = static_cast<int>(max_chunks);
+    g.nb = moe::gemm2_blocks(H);
+    g.gate_up = 0;
+    g.a_is_out_row = 1;
+    g.rows_per_expert = H;
     g.epi = moe::EPI_GATE_F32;
     g.out = y;
     g.ldo = H;

@@ -7,20 +7,18 @@
 
 namespace moe {
 
-// One unit of work of the grouped block-scaled GEMM: a pair of 128-row
-// weight blocks (block B optional) against up to 128 activation rows.
+// One unit of work of the grouped block-scaled GEMM, decoded on the device
+// from a chunk (<= 128 activation rows of one expert) and a weight-block pair.
 struct GemmTile {
   int32_t w_row0;   // first row of weight block A in the weight tensor
   int32_t w_row1;   // first row of weight block B, or -1
-  int32_t sw0;      // 128-row block index of block A in the weight scales
-  int32_t sw1;      // 128-row block index of block B
-  int32_t a_row;    // first activation row
+  int32_t a_row;    // first activation row (in the tensor map the tile reads)
   int32_t n;        // activation rows in this tile, 1..128
-  int32_t out_row;  // first output row
-  int32_t out_col;  // bits 0..23: first output column of block A's outputs;
-                    // bit 24: activations come from the second tensor map
+  int32_t out_row;  // first output row (also the column of the transposed scales)
+  int32_t out_col;  // first output column of block A's outputs
+  int32_t from1;    // activations come from the second tensor map
+  int32_t pad;
 };
-constexpr int32_t kTileFromMap1 = 1 << 24;
 
 enum EpiKind : int { EPI_SWIGLU_Q = 0, EPI_GATE_F32 = 1, EPI_BF16 = 2 };
 
@@ -36,20 +34,26 @@ struct GemmLaunch {
   const float *sw;        // weight scales [w_rows/128, K/128]
   const float *sa0;       // activation scales [a0_rows, K/128]
   const float *sa1;
-  // tiles: either a device list (tiles != null, count at n_tiles[slot]) or
-  // the dense grid of a plain GEMM (dense_M rows x w_rows outputs)
-  const GemmTile *tiles;
-  const int32_t *n_tiles;
-  int tile_slot;
-  int max_tiles;          // host-side upper bound (grid sizing)
+  // work: a chunk table (chunks != null, count at n_chunks[0]) or the dense
+  // grid of a plain GEMM (dense_M rows); nb weight-block pairs per chunk
+  const int4 *chunks;
+  const int32_t *n_chunks;
+  int max_chunks;          // host-side upper bound (grid sizing)
   int64_t dense_M;
+  int nb;                  // weight-block pairs per chunk
+  int gate_up;             // pair block j with block j + half (SwiGLU) instead of 2j, 2j+1
+  int a_is_out_row;        // activation row = the chunk's output row (input is a previous GEMM's output)
+  int64_t half;            // I for the gate/up GEMM
+  int64_t rows_per_expert; // weight rows per expert (2I, H, or N for the dense GEMM)
+  int sa_transposed;       // activation scales stored [K/128][sa_ld] (column = out_row)
+  int64_t sa_ld;
   // epilogue
   int epi;
   void *out;
   int64_t ldo;
   int64_t out_rows;       // rows of `out` (bounds check)
   int64_t out_cols;       // output columns addressable per row (bounds check)
-  float *out_scale;
+  float *out_scale;       // EPI_SWIGLU_Q: transposed scales [I/128][ld_os], column = row
   int64_t ld_os;
   const float *row_gate;
   int32_t *err;
@@ -72,12 +76,13 @@ cudaError_t launch_router_topk(const float *partial, int n_ks, int64_t T, int Nr
 
 cudaError_t launch_hist(const int32_t *idx, int64_t T, int Kr, int Nr, int32_t *blk_hist, int32_t *err,
                         cudaStream_t st);
-cudaError_t launch_build_tiles(const int32_t *blk_hist, int64_t T, int Kr, int Nr, int Ns, int H, int I,
-                               int32_t *counts, int32_t *offsets, int32_t *blk_base, GemmTile *tiles1,
-                               GemmTile *tiles2, int32_t *ntiles, int32_t *counts_out, cudaStream_t st);
-cudaError_t launch_scatter(const int32_t *idx, const float *gate, const uint8_t *xq, const float *xs, int64_t T,
-                           int Kr, int Nr, int Ns, int H, const int32_t *blk_base, uint8_t *ap, float *as,
-                           float *row_gate, int32_t *pos, cudaStream_t st);
+cudaError_t launch_build_chunks(const int32_t *blk_hist, int64_t T, int Kr, int Nr, int Ns, int32_t *counts,
+                                int32_t *offsets, int32_t *blk_base, int4 *chunks, int32_t *meta,
+                                int32_t *counts_out, cudaStream_t st);
+cudaError_t launch_rank(const int32_t *idx, const float *gate, int64_t T, int Kr, int Nr, int Ns,
+                        const int32_t *blk_base, float *row_gate, int32_t *row_src, int32_t *pos, cudaStream_t st);
+cudaError_t launch_copy_rows(const uint8_t *xq, const float *xs, const int32_t *row_src, int64_t R, int64_t T,
+                             int Ns, int H, uint8_t *ap, float *as_t, cudaStream_t st);
 
 cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st);
 
@@ -87,7 +92,7 @@ cudaError_t launch_bias_update(float *bias, const int32_t *counts, int Nr, int64
                                cudaStream_t st);
 cudaError_t launch_wait_selftest(int32_t *err, uint64_t limit_ns, cudaStream_t st);
 
-// tiles per 128-row chunk of activations in each grouped GEMM
+// weight-block pairs (tiles) per chunk of activations in each grouped GEMM
 __host__ __device__ inline int gemm1_blocks(int I) { return I / 128; }
 __host__ __device__ inline int gemm2_blocks(int H) { return (H / 128 + 1) / 2; }
 // upper bound on chunks of <= 128 rows over all experts

@@ -8,11 +8,14 @@
 // slot order.  All of it runs on the device; the host never learns the
 // per-expert counts.
 //
-//  hist_kernel        per 128-token block, per-expert counts
-//  build_tiles_kernel one CTA: totals, exclusive scans, per-block bases, and
-//                     the work lists of both grouped GEMMs
-//  scatter_kernel     per 128-token block: stable ranks (warp match), then
-//                     row copies (16-byte vectors) and per-row gate values
+//  hist_kernel         per 128-token block, per-expert counts
+//  build_chunks_kernel one CTA: totals, exclusive scans, per-block bases and
+//                      the chunk table (<= 128 rows of one expert per chunk)
+//                      from which both grouped GEMMs derive their tiles
+//  rank_kernel         per 128-token block: stable ranks (warp match) ->
+//                      row of every (token, slot), per-row gate and source
+//  copy_rows_kernel    one warp per row: FP8 row copy (16-byte vectors) and
+//                      the row's scales into the transposed scale table
 #include "common.cuh"
 #include "kernels.h"
 
@@ -63,10 +66,11 @@ __device__ int block_excl_scan(int v, int *total) {
   return base + x - v;
 }
 
-__global__ void __launch_bounds__(256) build_tiles_kernel(const int32_t *__restrict__ blk_hist, int64_t T, int Kr,
-                                                           int Nr, int Ns, int H, int I, int32_t *counts,
-                                                           int32_t *offsets, int32_t *blk_base, GemmTile *tiles1,
-                                                           GemmTile *tiles2, int32_t *ntiles, int32_t *counts_out) {
+// Chunk table entry: {expert | from_input << 16, activation row, output row, rows}.
+__global__ void __launch_bounds__(256) build_chunks_kernel(const int32_t *__restrict__ blk_hist, int64_t T, int Kr,
+                                                            int Nr, int Ns, int32_t *counts, int32_t *offsets,
+                                                            int32_t *blk_base, int4 *chunks, int32_t *meta,
+                                                            int32_t *counts_out) {
   const int e = threadIdx.x;
   const int nblk = static_cast<int>((T + kTokBlock - 1) / kTokBlock);
   const int64_t R = T * Kr;
@@ -89,87 +93,31 @@ __global__ void __launch_bounds__(256) build_tiles_kernel(const int32_t *__restr
       run += blk_hist[static_cast<int64_t>(b) * Nr + e];
     }
   }
-  const int nb1 = gemm1_blocks(I), nb2 = gemm2_blocks(H);
-  const int hb = H / 128, ib = I / 128;
+  // shared-expert chunks first (full 128-row chunks: largest work first)
   const int sh_chunks = Ns ? static_cast<int>((T + 127) / 128) : 0;
-  // shared-expert tiles first (full 128-row chunks, largest work first)
-  for (int i = threadIdx.x; i < sh_chunks * nb1; i += blockDim.x) {
-    const int c = i / nb1, rb = i % nb1;
-    const int es = Nr;  // shared expert index
+  for (int c = threadIdx.x; c < sh_chunks; c += blockDim.x) {
     const int n = static_cast<int>((T - c * 128) < 128 ? (T - c * 128) : 128);
-    GemmTile t;
-    t.w_row0 = es * 2 * I + rb * 128;
-    t.w_row1 = es * 2 * I + I + rb * 128;
-    t.sw0 = es * (2 * ib) + rb;
-    t.sw1 = es * (2 * ib) + ib + rb;
-    t.a_row = c * 128;
-    t.n = n;
-    t.out_row = static_cast<int32_t>(R) + c * 128;
-    t.out_col = (rb * 128) | kTileFromMap1;
-    tiles1[rb * sh_chunks + c] = t;
-  }
-  for (int i = threadIdx.x; i < sh_chunks * nb2; i += blockDim.x) {
-    const int c = i / nb2, p = i % nb2;
-    const int es = Nr;
-    const int n = static_cast<int>((T - c * 128) < 128 ? (T - c * 128) : 128);
-    GemmTile t;
-    t.w_row0 = es * H + (2 * p) * 128;
-    t.w_row1 = (2 * p + 1 < hb) ? es * H + (2 * p + 1) * 128 : -1;
-    t.sw0 = es * hb + 2 * p;
-    t.sw1 = es * hb + 2 * p + 1;
-    t.a_row = static_cast<int32_t>(R) + c * 128;
-    t.n = n;
-    t.out_row = t.a_row;
-    t.out_col = 2 * p * 128;
-    tiles2[p * sh_chunks + c] = t;
+    chunks[c] = make_int4(Nr | (1 << 16), c * 128, static_cast<int>(R) + c * 128, n);
   }
   if (e < Nr && nch > 0) {
-    const int sz = (cnt + nch - 1) / nch;  // <= 128
-    const int64_t base1 = static_cast<int64_t>(sh_chunks) * nb1 + static_cast<int64_t>(cbase) * nb1;
-    const int64_t base2 = static_cast<int64_t>(sh_chunks) * nb2 + static_cast<int64_t>(cbase) * nb2;
-    for (int rb = 0; rb < nb1; ++rb) {
-      for (int c = 0; c < nch; ++c) {
-        GemmTile t;
-        t.w_row0 = e * 2 * I + rb * 128;
-        t.w_row1 = e * 2 * I + I + rb * 128;
-        t.sw0 = e * (2 * ib) + rb;
-        t.sw1 = e * (2 * ib) + ib + rb;
-        t.a_row = off + c * sz;
-        t.n = (cnt - c * sz) < sz ? (cnt - c * sz) : sz;
-        t.out_row = t.a_row;
-        t.out_col = rb * 128;
-        tiles1[base1 + rb * nch + c] = t;
-      }
-    }
-    for (int p = 0; p < nb2; ++p) {
-      for (int c = 0; c < nch; ++c) {
-        GemmTile t;
-        t.w_row0 = e * H + (2 * p) * 128;
-        t.w_row1 = (2 * p + 1 < hb) ? e * H + (2 * p + 1) * 128 : -1;
-        t.sw0 = e * hb + 2 * p;
-        t.sw1 = e * hb + 2 * p + 1;
-        t.a_row = off + c * sz;
-        t.n = (cnt - c * sz) < sz ? (cnt - c * sz) : sz;
-        t.out_row = t.a_row;
-        t.out_col = 2 * p * 128;
-        tiles2[base2 + p * nch + c] = t;
-      }
+    const int sz = (cnt + nch - 1) / nch;  // <= 128: rows split evenly over the chunks
+    for (int c = 0; c < nch; ++c) {
+      const int r0 = off + c * sz;
+      const int n = (cnt - c * sz) < sz ? (cnt - c * sz) : sz;
+      chunks[sh_chunks + cbase + c] = make_int4(e, r0, r0, n);
     }
   }
   if (threadIdx.x == 0) {
-    ntiles[0] = (sh_chunks + total_chunks) * nb1;
-    ntiles[1] = (sh_chunks + total_chunks) * nb2;
-    ntiles[2] = total_rows;
-    ntiles[3] = total_chunks;
+    meta[0] = sh_chunks + total_chunks;
+    meta[1] = total_rows;
   }
 }
 
-__global__ void __launch_bounds__(256) scatter_kernel(const int32_t *__restrict__ idx, const float *__restrict__ gate,
-                                                       const uint8_t *__restrict__ xq, const float *__restrict__ xs,
-                                                       int64_t T, int Kr, int Nr, int Ns, int H,
-                                                       const int32_t *__restrict__ blk_base, uint8_t *__restrict__ ap,
-                                                       float *__restrict__ as, float *__restrict__ row_gate,
-                                                       int32_t *__restrict__ pos) {
+__global__ void __launch_bounds__(256) rank_kernel(const int32_t *__restrict__ idx, const float *__restrict__ gate,
+                                                    int64_t T, int Kr, int Nr, int Ns,
+                                                    const int32_t *__restrict__ blk_base,
+                                                    float *__restrict__ row_gate, int32_t *__restrict__ row_src,
+                                                    int32_t *__restrict__ pos) {
   __shared__ int s_cnt[256];
   __shared__ int s_pos[kTokBlock * 16];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -200,20 +148,40 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t *__restrict_
   for (int a = threadIdx.x; a < na; a += blockDim.x) {
     const int p = s_pos[a];
     pos[t0 * Kr + a] = p;
-    if (p >= 0) row_gate[p] = gate[t0 * Kr + a];
+    if (p >= 0) {
+      row_gate[p] = gate[t0 * Kr + a];
+      row_src[p] = static_cast<int32_t>(t0 + a / Kr);
+    }
   }
   if (Ns)
     for (int i = threadIdx.x; i < nt; i += blockDim.x) row_gate[R + t0 + i] = 1.0f;
-  const int hv = H / 16, hs = H / 128;
-  for (int a = warp; a < na; a += blockDim.x / 32) {
-    const int p = s_pos[a];
-    if (p < 0) continue;
-    const int64_t t = t0 + a / Kr;
+}
+
+// Rows [0, R): routed rows, copied from the quantized input row row_src[p];
+// rows [R, R + T): the shared expert's rows (token p - R), scales only (the
+// gate/up GEMM reads their codes from the quantized input directly).
+// Scales go to the transposed table as_t[kb * ld + p], ld = R + T.
+__global__ void __launch_bounds__(256) copy_rows_kernel(const uint8_t *__restrict__ xq, const float *__restrict__ xs,
+                                                         const int32_t *__restrict__ row_src, int64_t R, int64_t T,
+                                                         int Ns, int H, uint8_t *__restrict__ ap,
+                                                         float *__restrict__ as_t) {
+  const int lane = threadIdx.x & 31;
+  const int64_t p = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int64_t rows = R + (Ns ? T : 0);
+  if (p >= rows) return;
+  const int hv = H / 16, kb = H / 128;
+  const int64_t ld = R + T;
+  int64_t t;
+  if (p < R) {
+    t = row_src[p];
+    if (t < 0 || t >= T) return;
     const uint4 *src = reinterpret_cast<const uint4 *>(xq + t * H);
-    uint4 *dst = reinterpret_cast<uint4 *>(ap + static_cast<int64_t>(p) * H);
+    uint4 *dst = reinterpret_cast<uint4 *>(ap + p * H);
     for (int i = lane; i < hv; i += 32) dst[i] = __ldg(src + i);
-    for (int i = lane; i < hs; i += 32) as[static_cast<int64_t>(p) * hs + i] = __ldg(xs + t * hs + i);
+  } else {
+    t = p - R;
   }
+  for (int i = lane; i < kb; i += 32) as_t[i * ld + p] = __ldg(xs + t * kb + i);
 }
 
 cudaError_t launch_hist(const int32_t *idx, int64_t T, int Kr, int Nr, int32_t *blk_hist, int32_t *err,
@@ -224,21 +192,29 @@ cudaError_t launch_hist(const int32_t *idx, int64_t T, int Kr, int Nr, int32_t *
   return cudaGetLastError();
 }
 
-cudaError_t launch_build_tiles(const int32_t *blk_hist, int64_t T, int Kr, int Nr, int Ns, int H, int I,
-                               int32_t *counts, int32_t *offsets, int32_t *blk_base, GemmTile *tiles1,
-                               GemmTile *tiles2, int32_t *ntiles, int32_t *counts_out, cudaStream_t st) {
-  build_tiles_kernel<<<1, 256, 0, st>>>(blk_hist, T, Kr, Nr, Ns, H, I, counts, offsets, blk_base, tiles1, tiles2,
-                                        ntiles, counts_out);
+cudaError_t launch_build_chunks(const int32_t *blk_hist, int64_t T, int Kr, int Nr, int Ns, int32_t *counts,
+                                int32_t *offsets, int32_t *blk_base, int4 *chunks, int32_t *meta,
+                                int32_t *counts_out, cudaStream_t st) {
+  build_chunks_kernel<<<1, 256, 0, st>>>(blk_hist, T, Kr, Nr, Ns, counts, offsets, blk_base, chunks, meta,
+                                         counts_out);
   return cudaGetLastError();
 }
 
-cudaError_t launch_scatter(const int32_t *idx, const float *gate, const uint8_t *xq, const float *xs, int64_t T,
-                           int Kr, int Nr, int Ns, int H, const int32_t *blk_base, uint8_t *ap, float *as,
-                           float *row_gate, int32_t *pos, cudaStream_t st) {
+cudaError_t launch_rank(const int32_t *idx, const float *gate, int64_t T, int Kr, int Nr, int Ns,
+                        const int32_t *blk_base, float *row_gate, int32_t *row_src, int32_t *pos, cudaStream_t st) {
   const int64_t nblk = (T + kTokBlock - 1) / kTokBlock;
   if (nblk == 0) return cudaSuccess;
-  scatter_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(idx, gate, xq, xs, T, Kr, Nr, Ns, H, blk_base, ap,
-                                                               as, row_gate, pos);
+  rank_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(idx, gate, T, Kr, Nr, Ns, blk_base, row_gate, row_src,
+                                                            pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_copy_rows(const uint8_t *xq, const float *xs, const int32_t *row_src, int64_t R, int64_t T,
+                             int Ns, int H, uint8_t *ap, float *as_t, cudaStream_t st) {
+  const int64_t rows = R + (Ns ? T : 0);
+  if (rows == 0) return cudaSuccess;
+  const int64_t blocks = (rows + 7) / 8;
+  copy_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(xq, xs, row_src, R, T, Ns, H, ap, as_t);
   return cudaGetLastError();
 }
 

@@ -51,8 +51,12 @@ def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts
     xq, xs = v("xq", torch.uint8, (T, H)), v("xs", torch.float32, (T, H // 128))
     idx, gate = v("idx", torch.int32, (T, Kr)), v("gate", torch.float32, (T, Kr))
     offsets, pos = v("offsets", torch.int32, (Nr + 1,)), v("pos", torch.int32, (T, Kr))
-    ap, as_ = v("ap", torch.uint8, (R, H)), v("as", torch.float32, (R, H // 128))
-    hq, hs = v("hq", torch.uint8, (R + T * Ns, I)), v("hs", torch.float32, (R + T * Ns, I // 128))
+    ap = v("ap", torch.uint8, (R, H))
+    # scale tables are stored transposed: [K/128, R + T], column = row
+    as_t = v("as", torch.float32, (H // 128, R + T))
+    as_ = np.ascontiguousarray(as_t[:, :R].T)
+    hq = v("hq", torch.uint8, (R + T * Ns, I))
+    hs = np.ascontiguousarray(v("hs", torch.float32, (I // 128, R + T)).T[:R + T * Ns])
     y = v("y", torch.float32, (R + T * Ns, H))
     counts = counts_out.cpu().numpy()
     assert np.array_equal(idx_out.cpu().numpy(), idx)
@@ -79,6 +83,8 @@ def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts
     assert np.array_equal(pos.reshape(-1), pos_o)
     src_t = order // Kr
     assert np.array_equal(ap, xq_o[src_t]) and np.array_equal(as_, xs_o[src_t])
+    if Ns:
+        assert np.array_equal(np.ascontiguousarray(as_t[:, R:].T), xs_o)
     # weights quantized on the GPU are the oracle's, bit for bit
     experts = oracle_experts if oracle_experts is not None else {}
     need = set(int(e) for t in tok for e in idx[t]) | set(int(e) for t in tok for e in oi[t])
