@@ -234,11 +234,12 @@ typedef struct {
     size_t offsets[2];  /* int32 [N_r + 1]  first row of each expert           */
     size_t pos[2];      /* int32 [T, K_r]   row of (t, k) in expert order      */
     size_t ap[2];       /* E4M3 [R, H]      expert-contiguous copy of xq rows  */
-    size_t as[2];       /* float [H/128, R + T] scales of every row, transposed */
+    size_t as[2];       /* float [H/128, P] scales of every row, transposed;
+                           P = R + T rounded up to a multiple of 4          */
     size_t row_gate[2]; /* float [R + T*N_s] gate of each row (1 for shared)   */
     size_t row_src[2];  /* int32 [R]        token of each routed row           */
     size_t hq[2];       /* E4M3 [R + T*N_s, I] re-quantized SwiGLU output      */
-    size_t hs[2];       /* float [I/128, R + T] its scales, transposed         */
+    size_t hs[2];       /* float [I/128, P] its scales, transposed             */
     size_t y[2];        /* float [R + T*N_s, H] gate-scaled expert outputs     */
     size_t meta[2];     /* int32 [4]: number of chunks, routed rows            */
     size_t logits[2];   /* float [S, T, N_r] router logit partials (S K-splits) */

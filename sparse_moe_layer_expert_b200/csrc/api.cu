@@ -125,11 +125,12 @@ void make_layout(const moe_config *c, int64_t T, moe_ws_layout *L) {
   cv.take(L->offsets, (Nr + 1) * 4);
   cv.take(L->pos, T * Kr * 4);
   cv.take(L->ap, R * H);
-  cv.take(L->as, (H / 128) * (R + T) * 4);
+  const int64_t pitch = moe::scale_pitch(R, T);
+  cv.take(L->as, ((H / 128) * pitch + moe::kScaleSlack) * 4);
   cv.take(L->row_gate, RS * 4);
   cv.take(L->row_src, R * 4);
   cv.take(L->hq, RS * I);
-  cv.take(L->hs, (I / 128) * (R + T) * 4);
+  cv.take(L->hs, ((I / 128) * pitch + moe::kScaleSlack) * 4);
   cv.take(L->y, RS * H * 4);
   cv.take(L->meta, 4 * 4);
   cv.take(L->logits, ks * T * Nr * 4);
@@ -368,7 +369,8 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
   if (e == cudaSuccess)
     e = moe::launch_build_chunks(blk_hist, T, Kr, Nr, Ns, counts, offsets, blk_base, chunks, meta, counts_out, st);
   if (e == cudaSuccess) e = moe::launch_rank(idx, gate, T, Kr, Nr, Ns, blk_base, row_gate, row_src, pos, st);
-  if (e == cudaSuccess) e = moe::launch_copy_rows(xq, xs, row_src, R, T, Ns, H, ap, as_t, st);
+  const int64_t pitch = moe::scale_pitch(R, T);
+  if (e == cudaSuccess) e = moe::launch_copy_rows(xq, xs, row_src, R, T, Ns, H, ap, as_t, pitch, st);
   if (e == cudaSuccess) e = prof_mark(3, st);
   if (e == cudaSuccess) {
     // gate/up projection + SwiGLU + 1x128 requantization
@@ -384,7 +386,7 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
     g.sa0 = as_t;
     g.sa1 = as_t;
     g.sa_transposed = 1;
-    g.sa_ld = R + T;
+    g.sa_ld = pitch;
     g.chunks = chunks;
     g.n_chunks = meta;
     g.max_chunks = static_cast<int>(max_chunks);
@@ -398,7 +400,7 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
     g.out_rows = RS;
     g.out_cols = 2 * I;  // block B (up) shares block A's output columns
     g.out_scale = hs_t;
-    g.ld_os = R + T;
+    g.ld_os = pitch;
     g.err = err_flag;
     g.wait_limit_ns = moe::kDefaultWaitLimitNs;
     e = moe::launch_gemm(g, st);
@@ -418,7 +420,7 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
     g.sa0 = hs_t;
     g.sa1 = hs_t;
     g.sa_transposed = 1;
-    g.sa_ld = R + T;
+    g.sa_ld = pitch;
     g.chunks = chunks;
     g.n_chunks = meta;
     g.max_chunks = static_cast<int>(max_chunks);

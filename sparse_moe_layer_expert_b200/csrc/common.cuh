@@ -143,6 +143,16 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// 1D bulk copy global -> shared of `bytes` (multiple of 16; both addresses
+// 16-byte aligned), completing `bytes` on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // -------------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
@@ -270,6 +280,22 @@ __device__ __forceinline__ void setmaxnreg_inc() {
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// a / b rounded to nearest from y = RN(1/b): q0 = RN(a*y), the exact residual
+// r = a - b*q0 (one FMA), then RN(q0 + r*y).  One residual correction of the
+// quotient (Markstein's division by reciprocal, as presented in Muller et al.,
+// "Handbook of Floating-Point Arithmetic", chapter on division) -- used where
+// many values share one divisor; b > 0 normal, a/b far from over/underflow.
+__device__ __forceinline__ float div_by_recip(float a, float b, float y) {
+  const float q0 = a * y;
+  const float r = fmaf(-b, q0, a);
+  return fmaf(r, y, q0);
+}
+
+// Two E4M3 codes (round to nearest even, saturating) packed low = a, high = b.
+__device__ __forceinline__ uint32_t e4m3x2_rn_sat(float a, float b) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
 }
 
 // E4M3 code of v (round to nearest even, saturating at +-448).

@@ -48,12 +48,15 @@ constexpr int G_AB = 128 * 128;           // activation tile: 128 rows x 128 byt
 constexpr int G_WB = 128 * 128;           // one 128x128 weight tile (bytes)
 constexpr int G_STAGE = G_AB + 2 * G_WB;  // 48 KB
 constexpr int G_THREADS = 384;
-constexpr int G_RING = 136;               // floats per scale slot: 128 row scales + 2 weight scales
+// Scale slot (floats): [0, 132) activation scales of the tile's rows starting
+// at row offset [134] (a bulk copy starts on a 16-byte boundary), [132] and
+// [133] the two weight-block scales.
+constexpr int G_RING = 136;
+constexpr int G_SA_SPAN = 132;            // activation scales copied per K block
 constexpr int G_AMAX = 2 * 128;           // floats, SwiGLU amax exchange (per warpgroup, per row)
-constexpr int G_PF = 6;                   // K blocks of scales the scale warp has in flight
-constexpr int G_XSLOTS = G_PF + 2;        // staging slots of raw scales
-constexpr int G_SMEM = 1024 + G_STAGES * G_STAGE + G_SSLOTS * G_RING * 4 + G_AMAX * 4 +
-                       G_XSLOTS * G_RING * 4 + 256;
+constexpr int G_KBMAX = 512;              // K/128 up to 512 (K <= 65536)
+constexpr int G_WSC = 2 * 2 * G_KBMAX;    // floats: weight-scale rows of 2 tiles x 2 blocks
+constexpr int G_SMEM = 1024 + G_STAGES * G_STAGE + G_SSLOTS * G_RING * 4 + G_AMAX * 4 + G_WSC * 4 + 256;
 
 struct GemmArgs {
   const int4 *chunks;        // chunk table, or null for the dense grid
@@ -69,7 +72,7 @@ struct GemmArgs {
   const float *sw;
   const float *sa0;
   const float *sa1;
-  int sa_transposed;
+  int sa_transposed;         // [K/128][sa_ld] tables, sa_ld % 4 == 0, 132 floats of slack
   int64_t sa_ld;
   int KB;
   void *out;
@@ -141,7 +144,7 @@ __device__ __forceinline__ bool tile_ok(const GemmArgs &a, const GemmTile &d) {
   return d.n >= 1 && d.n <= 128 && d.a_row >= 0 && d.a_row + d.n <= arows && d.out_row >= 0 &&
          d.out_row + d.n <= a.out_rows && d.w_row0 >= 0 && d.w_row0 + 128 <= a.w_rows &&
          (!two || d.w_row1 + 128 <= a.w_rows) && d.out_col >= 0 && d.out_col + (two ? 256 : 128) <= a.out_cols &&
-         (!a.sa_transposed || d.out_row + d.n <= a.sa_ld);
+         (!a.sa_transposed || d.out_row + d.n <= a.sa_ld) && a.KB <= G_KBMAX;
 }
 }  // namespace
 
@@ -154,8 +157,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   uint8_t *stages = smem;
   float *sring = reinterpret_cast<float *>(smem + G_STAGES * G_STAGE);
   float *amax_x = sring + G_SSLOTS * G_RING;
-  float *xstage = amax_x + G_AMAX;
-  GemmBars *bars = reinterpret_cast<GemmBars *>(xstage + G_XSLOTS * G_RING);
+  float *wsc = amax_x + G_AMAX;
+  GemmBars *bars = reinterpret_cast<GemmBars *>(wsc + G_WSC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -164,7 +167,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       mbar_init(&bars->empty[i], 1);
     }
     for (int i = 0; i < G_SSLOTS; ++i) {
-      mbar_init(&bars->sfull[i], 1);
+      mbar_init(&bars->sfull[i], 2);  // the bulk copy's expect_tx arrival + the weight scales
       mbar_init(&bars->sempty[i], 8);
     }
     for (int i = 0; i < 2; ++i) {
@@ -209,9 +212,11 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         const uint64_t pol_a = policy_evict_last();
         uint32_t it = 0;
         bool stop = false;
+        GemmTile tn = get_tile(args, blockIdx.x < ntiles ? blockIdx.x : 0);  // next tile, loaded one tile ahead
         for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x) {
           if (*abortp) break;
-          const GemmTile td = get_tile(args, tile);
+          const GemmTile td = tn;
+          if (tile + gridDim.x < ntiles) tn = get_tile(args, tile + gridDim.x);
           if (!tile_ok(args, td)) continue;
           const CUtensorMap *amap = td.from1 ? &map_a1 : &map_a0;
           const bool two = td.w_row1 >= 0;
@@ -242,9 +247,11 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       if (lane == 0) {
         uint32_t it = 0;
         bool stop = false;
+        GemmTile tn = get_tile(args, blockIdx.x < ntiles ? blockIdx.x : 0);  // next tile, loaded one tile ahead
         for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x) {
           if (*abortp) break;
-          const GemmTile td = get_tile(args, tile);
+          const GemmTile td = tn;
+          if (tile + gridDim.x < ntiles) tn = get_tile(args, tile + gridDim.x);
           if (!tile_ok(args, td)) continue;
           const bool two = td.w_row1 >= 0;
           // D[128 activation rows, 256 (or 128) weight rows]
@@ -279,11 +286,13 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       }
     } else if (warp == 2) {
       // -------------------------------------------------------- scale producer
-      // Per K block: the activation scale of each of the tile's rows and the
-      // two weight-block scales, fetched with cp.async into a staging ring
-      // G_PF K blocks ahead (no register holds data in flight), then copied
-      // into the promotion ring when a slot frees up.
+      // Fills one promotion-ring slot per K block: the K block's activation
+      // scales of the tile's rows (one bulk copy from the transposed table,
+      // completing on the slot's barrier) and the two weight-block scales
+      // (from the tile's weight-scale rows, staged in shared memory once per
+      // tile).  The ring runs up to G_SSLOTS K blocks ahead of promotion.
       uint32_t it = 0;
+      int par = 0;
       bool stop = false;
       for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x) {
         if (*abortp) break;
@@ -293,57 +302,49 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           continue;
         }
         const bool two = td.w_row1 >= 0;
-        const float *sa = td.from1 ? args.sa1 : args.sa0;
-        const float *swa = args.sw + static_cast<int64_t>(td.w_row0 / 128) * KB;
-        const float *swb = args.sw + static_cast<int64_t>((two ? td.w_row1 : td.w_row0) / 128) * KB;
-        auto issue = [&](int kb) {
-          if (kb < KB) {
-            float *stg = xstage + (kb % G_XSLOTS) * G_RING;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int j = lane + 32 * i;
-              if (j < td.n) {
-                const int64_t off = args.sa_transposed
-                                        ? static_cast<int64_t>(kb) * args.sa_ld + td.out_row + j
-                                        : static_cast<int64_t>(td.a_row + j) * KB + kb;
-                cp_async4(stg + j, sa + off);
-              }
-            }
-            if (lane == 0) {
-              cp_async4(stg + 128, swa + kb);
-              if (two) cp_async4(stg + 129, swb + kb);
-            }
+        float *wA = wsc + par * (2 * G_KBMAX), *wB = wA + G_KBMAX;
+        par ^= 1;
+        {
+          const float *swa = args.sw + static_cast<int64_t>(td.w_row0 / 128) * KB;
+          const float *swb = args.sw + static_cast<int64_t>((two ? td.w_row1 : td.w_row0) / 128) * KB;
+          for (int i = lane; i < KB; i += 32) {
+            wA[i] = __ldg(swa + i);
+            wB[i] = two ? __ldg(swb + i) : 0.0f;
           }
-          cp_async_commit();  // one group per K block (empty past the end)
-        };
-#pragma unroll 1
-        for (int u = 0; u < G_PF; ++u) issue(u);
-        for (int kb = 0; kb < KB; ++kb) {
-          issue(kb + G_PF);
-          cp_async_wait<G_PF>();  // the group of K block kb has landed
           __syncwarp();
+        }
+        const float *sa = td.from1 ? args.sa1 : args.sa0;
+        const int off = args.sa_transposed ? (td.out_row & 3) : 0;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
           const int slot = it % G_SSLOTS;
           if (!mbar_wait(&bars->sempty[slot], ((it / G_SSLOTS) & 1) ^ 1, ctl)) {
             stop = true;
             break;
           }
-          const float *stg = xstage + (kb % G_XSLOTS) * G_RING;
           float *rs = sring + slot * G_RING;
+          if (args.sa_transposed) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&bars->sfull[slot], G_SA_SPAN * 4);
+              bulk_load(rs, sa + static_cast<int64_t>(kb) * args.sa_ld + (td.out_row - off), G_SA_SPAN * 4,
+                        &bars->sfull[slot]);
+            }
+          } else {
+            // row-major scales [rows, K/128] (plain GEMM): strided loads
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int j = lane + 32 * i;
-            rs[j] = (j < td.n) ? stg[j] : 0.0f;
+            for (int i = 0; i < 4; ++i) {
+              const int j = lane + 32 * i;
+              rs[j] = (j < td.n) ? __ldg(sa + static_cast<int64_t>(td.a_row + j) * KB + kb) : 0.0f;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->sfull[slot]);
           }
           if (lane == 0) {
-            rs[128] = stg[128];
-            rs[129] = two ? stg[129] : 0.0f;
+            rs[132] = wA[kb];
+            rs[133] = wB[kb];
+            rs[134] = __int_as_float(off);
+            mbar_arrive(&bars->sfull[slot]);
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->sfull[slot]);
-          ++it;
         }
-        cp_async_wait<0>();
-        __syncwarp();
       }
     }
   } else {
@@ -373,9 +374,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         if (ok) {
           tc_fence_after();
           const float *rs = sring + slot * G_RING;
-          const float sx = rs[r];
-          const float ca = sx * rs[128];  // promotion scale of block A for this row
-          const float cb = sx * rs[129];  // and of block B
+          const float sx = rs[r + __float_as_int(rs[134])];
+          const float ca = sx * rs[132];  // promotion scale of block A for this row
+          const float cb = sx * rs[133];  // and of block B
           const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * 256 + wg * 64;
           uint32_t p[64];
           tmem_ld64(ta, p);
@@ -401,12 +402,13 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const int64_t orow = static_cast<int64_t>(td.out_row) + r;
       const int c0 = td.out_col + wg * 64;  // first output column of this thread (block A)
       if constexpr (EPI == EPI_SWIGLU_Q) {
-        // h = silu(G) * U in FP32 for this row's 64 channels
+        // h = silu(G) * U in FP32 for this row's 64 channels (fast exp and
+        // divide: a few ulp, far inside the layer's tolerance)
         float amax = 0.0f;
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
           const float g = acc0[j];
-          acc0[j] = (g / (1.0f + expf(-g))) * acc1[j];
+          acc0[j] = __fdividef(g, 1.0f + __expf(-g)) * acc1[j];
           amax = fmaxf(amax, fabsf(acc0[j]));
         }
         // amax over the tile's 128 channels = this warpgroup's 64 + the other's
@@ -416,21 +418,27 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         const float S = amax / 448.0f;
         if (valid) {
           uint8_t *hq = static_cast<uint8_t *>(args.out) + orow * args.ldo + c0;
+          uint4 *hq4 = reinterpret_cast<uint4 *>(hq);
+          if (S != 0.0f) {
+            // quotients h / S share the divisor: correctly rounded through the
+            // reciprocal plus one residual correction
+            const float y = __frcp_rn(S);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t w[4];
+            for (int v = 0; v < 4; ++v) {
+              uint32_t w[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              uint32_t b = 0;
-#pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                const float h = acc0[v * 16 + k * 4 + t];
-                const uint32_t code = (S != 0.0f) ? e4m3_rn_sat(h / S) : 0u;
-                b |= code << (8 * t);
+              for (int k = 0; k < 4; ++k) {
+                const int j = v * 16 + k * 4;
+                const uint32_t lo = e4m3x2_rn_sat(div_by_recip(acc0[j], S, y), div_by_recip(acc0[j + 1], S, y));
+                const uint32_t hi =
+                    e4m3x2_rn_sat(div_by_recip(acc0[j + 2], S, y), div_by_recip(acc0[j + 3], S, y));
+                w[k] = lo | (hi << 16);
               }
-              w[k] = b;
+              hq4[v] = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            reinterpret_cast<uint4 *>(hq)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+          } else {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) hq4[v] = make_uint4(0, 0, 0, 0);
           }
           if (wg == 0) args.out_scale[static_cast<int64_t>(td.out_col / 128) * args.ld_os + orow] = S;
         }

@@ -82,7 +82,12 @@ cudaError_t launch_build_chunks(const int32_t *blk_hist, int64_t T, int Kr, int 
 cudaError_t launch_rank(const int32_t *idx, const float *gate, int64_t T, int Kr, int Nr, int Ns,
                         const int32_t *blk_base, float *row_gate, int32_t *row_src, int32_t *pos, cudaStream_t st);
 cudaError_t launch_copy_rows(const uint8_t *xq, const float *xs, const int32_t *row_src, int64_t R, int64_t T,
-                             int Ns, int H, uint8_t *ap, float *as_t, cudaStream_t st);
+                             int Ns, int H, uint8_t *ap, float *as_t, int64_t ld, cudaStream_t st);
+// Row pitch of the transposed scale tables [K/128][pitch]: R + T rounded up to
+// 4 floats (16-byte aligned rows for bulk copies); the tables carry
+// kScaleSlack floats after their last row so a 132-float copy stays in bounds.
+inline int64_t scale_pitch(int64_t R, int64_t T) { return (R + T + 3) / 4 * 4; }
+constexpr int64_t kScaleSlack = 132;
 
 cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st);
 

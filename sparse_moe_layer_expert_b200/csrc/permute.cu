@@ -160,17 +160,16 @@ __global__ void __launch_bounds__(256) rank_kernel(const int32_t *__restrict__ i
 // Rows [0, R): routed rows, copied from the quantized input row row_src[p];
 // rows [R, R + T): the shared expert's rows (token p - R), scales only (the
 // gate/up GEMM reads their codes from the quantized input directly).
-// Scales go to the transposed table as_t[kb * ld + p], ld = R + T.
+// Scales go to the transposed table as_t[kb * ld + p].
 __global__ void __launch_bounds__(256) copy_rows_kernel(const uint8_t *__restrict__ xq, const float *__restrict__ xs,
                                                          const int32_t *__restrict__ row_src, int64_t R, int64_t T,
                                                          int Ns, int H, uint8_t *__restrict__ ap,
-                                                         float *__restrict__ as_t) {
+                                                         float *__restrict__ as_t, int64_t ld) {
   const int lane = threadIdx.x & 31;
   const int64_t p = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int64_t rows = R + (Ns ? T : 0);
   if (p >= rows) return;
   const int hv = H / 16, kb = H / 128;
-  const int64_t ld = R + T;
   int64_t t;
   if (p < R) {
     t = row_src[p];
@@ -210,11 +209,11 @@ cudaError_t launch_rank(const int32_t *idx, const float *gate, int64_t T, int Kr
 }
 
 cudaError_t launch_copy_rows(const uint8_t *xq, const float *xs, const int32_t *row_src, int64_t R, int64_t T,
-                             int Ns, int H, uint8_t *ap, float *as_t, cudaStream_t st) {
+                             int Ns, int H, uint8_t *ap, float *as_t, int64_t ld, cudaStream_t st) {
   const int64_t rows = R + (Ns ? T : 0);
   if (rows == 0) return cudaSuccess;
   const int64_t blocks = (rows + 7) / 8;
-  copy_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(xq, xs, row_src, R, T, Ns, H, ap, as_t);
+  copy_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(xq, xs, row_src, R, T, Ns, H, ap, as_t, ld);
   return cudaGetLastError();
 }
 

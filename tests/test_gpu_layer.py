@@ -52,11 +52,13 @@ def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts
     idx, gate = v("idx", torch.int32, (T, Kr)), v("gate", torch.float32, (T, Kr))
     offsets, pos = v("offsets", torch.int32, (Nr + 1,)), v("pos", torch.int32, (T, Kr))
     ap = v("ap", torch.uint8, (R, H))
-    # scale tables are stored transposed: [K/128, R + T], column = row
-    as_t = v("as", torch.float32, (H // 128, R + T))
+    # scale tables are stored transposed: [K/128, P], column = row, P = R + T
+    # rounded up to a multiple of 4
+    P = (R + T + 3) // 4 * 4
+    as_t = v("as", torch.float32, (H // 128, P))
     as_ = np.ascontiguousarray(as_t[:, :R].T)
     hq = v("hq", torch.uint8, (R + T * Ns, I))
-    hs = np.ascontiguousarray(v("hs", torch.float32, (I // 128, R + T)).T[:R + T * Ns])
+    hs = np.ascontiguousarray(v("hs", torch.float32, (I // 128, P)).T[:R + T * Ns])
     y = v("y", torch.float32, (R + T * Ns, H))
     counts = counts_out.cpu().numpy()
     assert np.array_equal(idx_out.cpu().numpy(), idx)
@@ -84,7 +86,7 @@ def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts
     src_t = order // Kr
     assert np.array_equal(ap, xq_o[src_t]) and np.array_equal(as_, xs_o[src_t])
     if Ns:
-        assert np.array_equal(np.ascontiguousarray(as_t[:, R:].T), xs_o)
+        assert np.array_equal(np.ascontiguousarray(as_t[:, R:R + T].T), xs_o)
     # weights quantized on the GPU are the oracle's, bit for bit
     experts = oracle_experts if oracle_experts is not None else {}
     need = set(int(e) for t in tok for e in idx[t]) | set(int(e) for t in tok for e in oi[t])
