@@ -293,6 +293,18 @@ __device__ __forceinline__ float div_by_recip(float a, float b, float y) {
   return fmaf(r, y, q0);
 }
 
+// Two independent FP32 fused multiply-adds in one instruction:
+// (lo, hi) <- (p_lo * s + c_lo, p_hi * s + c_hi), each rounded to nearest
+// like fmaf.
+__device__ __forceinline__ void ffma2_scalar(float &c_lo, float &c_hi, float p_lo, float p_hi, float s) {
+  uint64_t c, p, ss;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(c_lo), "f"(c_hi));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(p) : "f"(p_lo), "f"(p_hi));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(s));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(c) : "l"(p), "l"(ss));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(c_lo), "=f"(c_hi) : "l"(c));
+}
+
 // Two E4M3 codes (round to nearest even, saturating) packed low = a, high = b.
 __device__ __forceinline__ uint32_t e4m3x2_rn_sat(float a, float b) {
   return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));

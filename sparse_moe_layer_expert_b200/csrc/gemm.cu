@@ -48,15 +48,19 @@ constexpr int G_AB = 128 * 128;           // activation tile: 128 rows x 128 byt
 constexpr int G_WB = 128 * 128;           // one 128x128 weight tile (bytes)
 constexpr int G_STAGE = G_AB + 2 * G_WB;  // 48 KB
 constexpr int G_THREADS = 384;
-// Scale slot (floats): [0, 132) activation scales of the tile's rows starting
-// at row offset [134] (a bulk copy starts on a 16-byte boundary), [132] and
-// [133] the two weight-block scales.
+// Scale slot (floats): [0, 132) activation scales of the tile's rows, starting
+// at row offset out_row & 3 (a bulk copy starts on a 16-byte boundary);
+// [132] and [133] the two weight-block scales.
 constexpr int G_RING = 136;
 constexpr int G_SA_SPAN = 132;            // activation scales copied per K block
 constexpr int G_AMAX = 2 * 128;           // floats, SwiGLU amax exchange (per warpgroup, per row)
-constexpr int G_KBMAX = 512;              // K/128 up to 512 (K <= 65536)
+constexpr int G_KBMAX = 256;              // K/128 up to 256 (K <= 32768)
 constexpr int G_WSC = 2 * 2 * G_KBMAX;    // floats: weight-scale rows of 2 tiles x 2 blocks
-constexpr int G_SMEM = 1024 + G_STAGES * G_STAGE + G_SSLOTS * G_RING * 4 + G_AMAX * 4 + G_WSC * 4 + 256;
+constexpr int G_OPITCH = 20;              // floats per row of an output transpose buffer (16 + pad)
+constexpr int G_OUTX = 8 * 32 * G_OPITCH; // floats: one 32-row x 16-float buffer per promotion warp
+constexpr int G_SMEM =
+    1024 + G_STAGES * G_STAGE + G_SSLOTS * G_RING * 4 + G_AMAX * 4 + G_WSC * 4 + G_OUTX * 4 + 256;
+static_assert(G_SMEM <= 232448, "shared memory budget");
 
 struct GemmArgs {
   const int4 *chunks;        // chunk table, or null for the dense grid
@@ -158,7 +162,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   float *sring = reinterpret_cast<float *>(smem + G_STAGES * G_STAGE);
   float *amax_x = sring + G_SSLOTS * G_RING;
   float *wsc = amax_x + G_AMAX;
-  GemmBars *bars = reinterpret_cast<GemmBars *>(wsc + G_WSC);
+  float *outx = wsc + G_WSC;
+  GemmBars *bars = reinterpret_cast<GemmBars *>(outx + G_OUTX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -341,7 +346,6 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           if (lane == 0) {
             rs[132] = wA[kb];
             rs[133] = wB[kb];
-            rs[134] = __int_as_float(off);
             mbar_arrive(&bars->sfull[slot]);
           }
         }
@@ -360,6 +364,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const GemmTile td = get_tile(args, tile);
       if (!tile_ok(args, td)) continue;
       const bool two = td.w_row1 >= 0;
+      const int soff = args.sa_transposed ? (td.out_row & 3) : 0;  // row offset inside a scale slot
       float acc0[64], acc1[64];
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
@@ -374,7 +379,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         if (ok) {
           tc_fence_after();
           const float *rs = sring + slot * G_RING;
-          const float sx = rs[r + __float_as_int(rs[134])];
+          const float sx = rs[r + soff];
           const float ca = sx * rs[132];  // promotion scale of block A for this row
           const float cb = sx * rs[133];  // and of block B
           const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * 256 + wg * 64;
@@ -382,12 +387,14 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           tmem_ld64(ta, p);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 64; ++j) acc0[j] = fmaf(__uint_as_float(p[j]), ca, acc0[j]);
+          for (int j = 0; j < 64; j += 2)
+            ffma2_scalar(acc0[j], acc0[j + 1], __uint_as_float(p[j]), __uint_as_float(p[j + 1]), ca);
           if (two) {
             tmem_ld64(ta + 128, p);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 64; ++j) acc1[j] = fmaf(__uint_as_float(p[j]), cb, acc1[j]);
+            for (int j = 0; j < 64; j += 2)
+              ffma2_scalar(acc1[j], acc1[j + 1], __uint_as_float(p[j]), __uint_as_float(p[j + 1]), cb);
           }
           tc_fence_before();
         }
@@ -443,48 +450,60 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           if (wg == 0) args.out_scale[static_cast<int64_t>(td.out_col / 128) * args.ld_os + orow] = S;
         }
         named_bar_sync(1, 256);  // amx is reused by the next tile
-      } else if constexpr (EPI == EPI_GATE_F32) {
-        if (valid) {
-          const float g = __ldg(args.row_gate + orow);
-          float4 *y = reinterpret_cast<float4 *>(static_cast<float *>(args.out) + orow * args.ldo + c0);
-#pragma unroll
-          for (int v = 0; v < 16; ++v)
-            y[v] = make_float4(acc0[4 * v] * g, acc0[4 * v + 1] * g, acc0[4 * v + 2] * g, acc0[4 * v + 3] * g);
-          if (two) {
-            float4 *y1 = y + 32;  // block B starts 128 columns later
-#pragma unroll
-            for (int v = 0; v < 16; ++v)
-              y1[v] =
-                  make_float4(acc1[4 * v] * g, acc1[4 * v + 1] * g, acc1[4 * v + 2] * g, acc1[4 * v + 3] * g);
-          }
-        }
       } else {
-        if (valid) {
-          uint4 *Cv = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(args.out) + orow * args.ldo + c0);
+        // Rows are written through a per-warp 32 x 16-float transpose buffer
+        // so that each 16-byte store instruction covers 8 rows x 64
+        // contiguous bytes instead of 32 scattered rows.
+        float *xb = outx + (warp - 4) * (32 * G_OPITCH);
+        const int rbase = q * 32;  // this warp's first row in the tile
+        const float g = (EPI == EPI_GATE_F32 && valid) ? __ldg(args.row_gate + orow) : 1.0f;
+        auto emit = [&](const float(&acc)[64], int b) {
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            uint32_t w[4];
+          for (int piece = 0; piece < (EPI == EPI_GATE_F32 ? 4 : 2); ++piece) {
+            // stage: this thread's 16 floats (or 32 bf16) of the piece, row = lane
+            float4 *dst = reinterpret_cast<float4 *>(xb + lane * G_OPITCH);
+            if constexpr (EPI == EPI_GATE_F32) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc0[8 * v + 2 * k], acc0[8 * v + 2 * k + 1]);
-              w[k] = *reinterpret_cast<const uint32_t *>(&b2);
-            }
-            Cv[v] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-          if (two) {
-            uint4 *C1 = Cv + 16;  // 128 bf16 later
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              uint32_t w[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc1[8 * v + 2 * k], acc1[8 * v + 2 * k + 1]);
-                w[k] = *reinterpret_cast<const uint32_t *>(&b2);
+              for (int v = 0; v < 4; ++v) {
+                const int j = piece * 16 + 4 * v;
+                dst[v] = make_float4(acc[j] * g, acc[j + 1] * g, acc[j + 2] * g, acc[j + 3] * g);
               }
-              C1[v] = make_uint4(w[0], w[1], w[2], w[3]);
+            } else {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                float f[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const int j = piece * 32 + 8 * v + 2 * k;
+                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[j], acc[j + 1]);
+                  f[k] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&b2));
+                }
+                dst[v] = make_float4(f[0], f[1], f[2], f[3]);
+              }
             }
+            __syncwarp();
+            // drain: lane L stores 16 bytes of row (L / 4 + 8 s), chunk L % 4
+#pragma unroll
+            for (int sgrp = 0; sgrp < 4; ++sgrp) {
+              const int rr = lane / 4 + 8 * sgrp;  // row within the warp's 32
+              if (rbase + rr < td.n) {
+                const float4 val = reinterpret_cast<const float4 *>(xb + rr * G_OPITCH)[lane & 3];
+                const int64_t grow = static_cast<int64_t>(td.out_row) + rbase + rr;
+                if constexpr (EPI == EPI_GATE_F32) {
+                  float *yrow = static_cast<float *>(args.out) + grow * args.ldo + c0 + 128 * b + piece * 16;
+                  reinterpret_cast<float4 *>(yrow)[lane & 3] = val;
+                } else {
+                  __nv_bfloat16 *crow =
+                      static_cast<__nv_bfloat16 *>(args.out) + grow * args.ldo + c0 + 128 * b + piece * 32;
+                  reinterpret_cast<float4 *>(crow)[lane & 3] = val;
+                }
+              }
+            }
+            __syncwarp();
           }
-        }
+        };
+        emit(acc0, 0);
+        if (two) emit(acc1, 1);
       }
     }
   }
