@@ -365,6 +365,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       if (!tile_ok(args, td)) continue;
       const bool two = td.w_row1 >= 0;
       const int soff = args.sa_transposed ? (td.out_row & 3) : 0;  // row offset inside a scale slot
+      // a warp whose 32 rows are all padding (short chunks) skips its TMEM
+      // reads and FMAs; it still takes every wait and arrival of the ring
+      const bool live = q * 32 < td.n;
       float acc0[64], acc1[64];
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
@@ -376,7 +379,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         const int slot = it % G_SSLOTS;
         const bool ok = mbar_wait(&bars->tfull[buf], (it >> 1) & 1, ctl) &&
                         mbar_wait(&bars->sfull[slot], (it / G_SSLOTS) & 1, ctl);
-        if (ok) {
+        if (ok && live) {
           tc_fence_after();
           const float *rs = sring + slot * G_RING;
           const float sx = rs[r + soff];
