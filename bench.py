@@ -71,6 +71,13 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def aggregate(total_ms_max: float, steps: int, world: int, tokens_per_rank: int):
+    """(ms per step, whole-job tokens/s) from the slowest rank's timed region:
+    every rank processes its own batch of `tokens_per_rank` tokens per step."""
+    ms_per_step = total_ms_max / steps
+    return ms_per_step, world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def barrier(world: int, device=None):
     if world > 1:
         import torch.distributed as dist
@@ -304,8 +311,7 @@ def main(argv=None):
     # the timed region is the K back-to-back steps: first start to last end
     total_ms = ev[0][0].elapsed_time(ev[-1][n_ev - 1])
     total_ms = max_over_ranks(total_ms, world, dev)
-    ms_per_step = total_ms / args.steps
-    value = world * T / (ms_per_step / 1e3)
+    ms_per_step, value = aggregate(total_ms, args.steps, world, T)
 
     counts_h = counts.cpu()
     touched = int((counts_h > 0).sum())
