@@ -93,6 +93,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
   }
 }
 
+// Non-blocking probe of phase `parity` (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for two phases.  Both are probed before either result is used, so the
+// two round trips to the barriers overlap when both phases are already
+// complete (the common case on the critical path); otherwise each is waited
+// for in turn with the bounded wait above.
+__device__ __forceinline__ bool mbar_wait2(uint64_t *bar1, uint32_t parity1, uint64_t *bar2, uint32_t parity2,
+                                           const WaitCtl &ctl) {
+  const bool a = mbar_test_wait(bar1, parity1);
+  const bool b = mbar_test_wait(bar2, parity2);
+  if (a && b) return true;
+  return (a || mbar_wait(bar1, parity1, ctl)) && (b || mbar_wait(bar2, parity2, ctl));
+}
+
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

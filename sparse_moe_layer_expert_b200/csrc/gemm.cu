@@ -264,8 +264,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           for (int kb = 0; kb < KB; ++kb, ++it) {
             const int s = it % G_STAGES;
             const uint32_t buf = it & 1;
-            if (!mbar_wait(&bars->tempty[buf], ((it >> 1) & 1) ^ 1, ctl) ||
-                !mbar_wait(&bars->full[s], (it / G_STAGES) & 1, ctl)) {
+            if (!mbar_wait2(&bars->tempty[buf], ((it >> 1) & 1) ^ 1, &bars->full[s], (it / G_STAGES) & 1, ctl)) {
               stop = true;
               break;
             }
@@ -377,8 +376,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const uint32_t buf = it & 1;
         const int slot = it % G_SSLOTS;
-        const bool ok = mbar_wait(&bars->tfull[buf], (it >> 1) & 1, ctl) &&
-                        mbar_wait(&bars->sfull[slot], (it / G_SSLOTS) & 1, ctl);
+        const bool ok = mbar_wait2(&bars->tfull[buf], (it >> 1) & 1, &bars->sfull[slot], (it / G_SSLOTS) & 1, ctl);
         if (ok && live) {
           tc_fence_after();
           const float *rs = sring + slot * G_RING;
