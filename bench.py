@@ -3,10 +3,13 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed]
                     [--impl ours|reference] [--no-cpu-baseline]
 
-One step = one whole layer forward (quantize, route, group, gate/up GEMM +
-SwiGLU + requantize, down GEMM, combine) over T tokens of seeded synthetic
-input with V3 shapes (hidden 7168, intermediate 2048, 256 routed + 1 shared
-experts, top-8), weights resident in HBM.  With N > 1 (launched by torchrun)
+One step = the whole path over T tokens of seeded synthetic input with V3
+shapes (hidden 7168, intermediate 2048, 256 routed + 1 shared experts,
+top-8), weights resident in HBM: the layer forward (quantize, route, group,
+gate/up GEMM + SwiGLU + requantize, down GEMM, combine) and the step's bias
+update.  The update goes to a working copy of the bias, so every step routes
+the batch alike; the line also reports the batch's expert load imbalance
+(max / mean) and the imbalance after one bias update applied for real.  With N > 1 (launched by torchrun)
 every rank runs its own replica of the layer on its own batch: there is no
 data-path collective; timing is the max over ranks.  Rank 0 prints one JSON
 line.
@@ -31,7 +34,8 @@ sys.path.insert(0, ROOT)
 
 WORKLOADS = ("prefill", "decode", "skewed")
 METRIC = "MoE-layer tokens/s and grouped FP8 GEMM TFLOP/s (% of B200 FP8 / HBM roofline)"
-KERNELS_PER_STEP = 9  # quantize, router GEMM, top-k, histogram, work lists, scatter, 2 GEMMs, combine
+KERNELS_PER_STEP = 11  # quantize, router GEMM, top-k, histogram, chunk table, ranks, row copy, 2 GEMMs, combine,
+#                        bias update
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 GEMM_SOURCES = [os.path.join(ROOT, "sparse_moe_layer_expert_b200", "csrc", f) for f in ("gemm.cu", "common.cuh")]
 
@@ -278,17 +282,32 @@ def main(argv=None):
     out = torch.empty((T, cfg["H"]), dtype=torch.bfloat16, device=dev)
     counts = torch.empty(cfg["Nr"], dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # A step is the whole path: the layer forward, then the bias update of
+    # the step (b_i -/+ gamma by the step's expert loads).  The update is
+    # written to a working copy of the bias, so every timed step routes the
+    # batch with the same bias (stationary routing) while doing all of the
+    # update's work.
+    bias_next = layer.bias.clone()
+    total_assign = T * cfg["Kr"]
+
+    def step(x_in):
+        layer.forward(x_in, out=out, counts_out=counts, stream=stream)
+        M.moe_bias_update(bias_next, counts, cfg["Nr"], total_assign, 0.001, stream=stream)
+
     torch.cuda.synchronize(dev)
 
     # ------------------------------------------------ device-timed steps
     for _ in range(args.warmup):
-        layer.forward(x, out=out, counts_out=counts, stream=stream)
+        step(x)
     layer.check(stream)
     n_ev = M.MOE_PROFILE_EVENTS
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    ev_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]  # after each step's bias update
     for row in ev:  # torch creates the CUDA event on first record; the library needs the handles
         for e in row:
             e.record(stream)
+    for e in ev_end:
+        e.record(stream)
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     try:
@@ -299,22 +318,35 @@ def main(argv=None):
     with sampler:
         for k in range(args.steps):
             M.moe_profile_events(ev[k])
-            layer.forward(x, out=out, counts_out=counts, stream=stream)
+            step(x)
+            ev_end[k].record(stream)
         M.moe_profile_events(None)
         torch.cuda.synchronize(dev)
     barrier(world, dev)
     layer.check(stream)
     clocks = sampler.summary()
-    step_ms = [ev[k][0].elapsed_time(ev[k][n_ev - 1]) for k in range(args.steps)]
+    step_ms = [ev[k][0].elapsed_time(ev_end[k]) for k in range(args.steps)]
     stage_ms = {name: sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)) / args.steps
                 for i, name in enumerate(M.PROFILE_STAGES)}
+    stage_ms["bias_update"] = sum(ev[k][n_ev - 1].elapsed_time(ev_end[k]) for k in range(args.steps)) / args.steps
     # the timed region is the K back-to-back steps: first start to last end
-    total_ms = ev[0][0].elapsed_time(ev[-1][n_ev - 1])
+    total_ms = ev[0][0].elapsed_time(ev_end[-1])
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step, value = aggregate(total_ms, args.steps, world, T)
 
     counts_h = counts.cpu()
     touched = int((counts_h > 0).sum())
+    # expert load imbalance of the batch, and after one bias update applied
+    # for real (the same batch routed again with b - gamma * sign(load - mean))
+    mean_load = total_assign / cfg["Nr"]
+    b_upd = layer.bias.clone()
+    M.moe_bias_update(b_upd, counts, cfg["Nr"], total_assign, 0.001, stream=stream)
+    b_keep, layer.bias = layer.bias, b_upd
+    counts_upd = torch.empty_like(counts)
+    layer.forward(x, out=out, counts_out=counts_upd, stream=stream)
+    layer.bias = b_keep
+    load = dict(max_over_mean=round(float(counts_h.max()) / mean_load, 3),
+                after_one_bias_update=round(float(counts_upd.max().item()) / mean_load, 3))
     alg = algorithmic_counts(cfg, T, touched)
     peaks = measured_peaks()
     g1_ms, g2_ms = stage_ms["gemm_gate_up"], stage_ms["gemm_down"]
@@ -346,7 +378,7 @@ def main(argv=None):
         out_h = torch.empty((T, cfg["H"]), dtype=torch.bfloat16).pin_memory()
         for _ in range(max(1, args.warmup // 2)):
             x_d = x_h.to(dev, non_blocking=True)
-            layer.forward(x_d, out=out, stream=stream)
+            step(x_d)
             out_h.copy_(out, non_blocking=True)
         barrier(world, dev)
         torch.cuda.synchronize(dev)
@@ -354,7 +386,7 @@ def main(argv=None):
         e0.record(stream)
         for _ in range(args.steps):
             x_d = x_h.to(dev, non_blocking=True)
-            layer.forward(x_d, out=out, stream=stream)
+            step(x_d)
             out_h.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
@@ -393,6 +425,7 @@ def main(argv=None):
         grouped_gemm_frac_fp8_peak=round(gemm_tflops / fp8_peak, 4),
         layer_weight_gb=round(alg["layer_weight_bytes"] / 1e9, 3),
         experts_touched=touched + cfg.get("Ns", 1),
+        load=load,
         stage_ms={k: round(v, 4) for k, v in stage_ms.items()},
         step_ms_min=round(min(step_ms), 4),
         cpu_baseline=cpu,
