@@ -189,6 +189,38 @@ def test_layer_wider_hidden_and_many_chunks(m, oracle_lib):
     check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob), tokens=np.arange(0, 700, 11))
 
 
+def test_layer_every_token_picks_the_same_experts(m, oracle_lib):
+    # A bias far above the spread of the affinities sends every token to
+    # experts 0..K_r-1: each of them receives all T rows (six 128-row
+    # chunks, the last one ragged) and every other routed expert none.
+    prob = Problem(S.TINY, 700, seed=10)
+    kr = S.TINY["Kr"]
+    prob.bias = prob.bias.clone()
+    prob.bias[:kr] += 1.0
+    r = check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob), tokens=np.arange(0, 700, 13))
+    c = r["counts"]
+    assert (c[:kr] == 700).all() and (c[kr:] == 0).all()
+
+
+def test_layer_empty_batch(m, oracle_lib):
+    # T = 0: nothing to compute; the loads are all zero and the bias update
+    # of an empty step leaves every bias unchanged (load == mean == 0)
+    prob = Problem(S.TINY, 4, seed=9)
+    layer = build_gpu_layer(m, prob)
+    nr = S.TINY["Nr"]
+    x0 = torch.empty((0, S.TINY["H"]), dtype=torch.bfloat16, device="cuda")
+    counts = torch.full((nr,), 7, dtype=torch.int32, device="cuda")
+    out = layer.forward(x0, counts_out=counts)
+    layer.check()
+    assert tuple(out.shape) == (0, S.TINY["H"])
+    assert int(counts.abs().sum()) == 0
+    b0 = layer.bias.cpu().numpy().copy()
+    layer.bias_update(counts, 0)
+    torch.cuda.synchronize()
+    want = oracle_lib.bias_update(b0, np.zeros(nr, np.int32), nr, 0)
+    assert np.array_equal(layer.bias.cpu().numpy(), want) and np.array_equal(want, b0)
+
+
 def test_bias_update_matches_oracle(m, oracle_lib):
     prob = Problem(S.TINY, 256, seed=7)
     layer = build_gpu_layer(m, prob)

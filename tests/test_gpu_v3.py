@@ -66,3 +66,27 @@ def test_v3_prefill_layer(m, oracle_lib, v3_layer):
     r = check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=False)
     c = r["counts"]
     print(f"prefill load: max {c.max()} mean {c.mean():.1f} min {c.min()} empty {(c == 0).sum()}")
+
+
+def test_v3_skewed_layer(m, oracle_lib, v3_layer):
+    """The skewed configuration at full size: 16384 tokens of the centroid-
+    mixture input, group-limited routing (8 groups of 32 experts, top-4
+    groups), zero bias; the V3 weights of the shared fixture, routed through a
+    layer object configured for group-limited routing."""
+    base, _ = v3_layer
+    cfg = dict(S.SKEWED)
+    shape = {k: cfg[k] for k in ("H", "I", "Nr", "Kr", "Ns", "n_groups", "topk_groups")}
+    layer = m.MoeLayer(shape)
+    layer.w13, layer.s13, layer.w2, layer.s2 = base.w13, base.s13, base.w2, base.s2  # same weights, no copy
+    T = cfg["T"]
+    prob = Problem(cfg, T, seed=13, device="cuda")  # mixture input (the configuration's x)
+    prob.seed = 0                                    # weights and router of the fixture (seed 0)
+    prob.wr = base.wr
+    prob.bias = torch.zeros(cfg["Nr"], dtype=torch.float32, device="cuda")
+    layer.set_router(prob.wr, prob.bias)
+    rng = np.random.default_rng(13)
+    toks = np.sort(rng.choice(T, 4, replace=False))
+    r = check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=False)
+    c = r["counts"]
+    print(f"skewed load: max {c.max()} mean {c.mean():.1f} max/mean {c.max() / c.mean():.2f}")
+    assert c.max() >= 4 * c.mean()  # the configuration's imbalance (max/mean load >= 4)
