@@ -41,7 +41,12 @@ def build(force: bool = False) -> str:
 class Cfg(C.Structure):
     _fields_ = [("H", C.c_int32), ("I", C.c_int32), ("Nr", C.c_int32), ("Kr", C.c_int32),
                 ("Ns", C.c_int32), ("n_groups", C.c_int32), ("topk_groups", C.c_int32),
-                ("pad", C.c_int32), ("route_scale", C.c_double)]
+                ("scale_mode", C.c_int32), ("route_scale", C.c_double)]
+
+# scale modes of the quantizers: S = amax/448 (the pages' recipe), or the
+# power-of-two variant (S = the smallest 2^e with amax <= 448 * 2^e)
+SCALE_AMAX = 0
+SCALE_POW2 = 1
 
 
 def _p(a: np.ndarray):
@@ -59,9 +64,9 @@ def lib():
             L.moe_oracle_e4m3_decode.restype = C.c_double
             L.moe_oracle_e4m3_encode.argtypes = [C.c_float]
             L.moe_oracle_e4m3_encode.restype = C.c_uint8
-            L.moe_oracle_quant_1x128_bf16.argtypes = [vp, i64, i64, i64, vp, vp]
-            L.moe_oracle_quant_1x128_f32.argtypes = [vp, i64, i64, vp, vp]
-            L.moe_oracle_quant_128x128.argtypes = [vp, i64, i64, vp, vp]
+            L.moe_oracle_quant_1x128_bf16.argtypes = [vp, i64, i64, i64, vp, vp, C.c_int]
+            L.moe_oracle_quant_1x128_f32.argtypes = [vp, i64, i64, vp, vp, C.c_int]
+            L.moe_oracle_quant_128x128.argtypes = [vp, i64, i64, vp, vp, C.c_int]
             L.moe_oracle_blockscaled_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
             L.moe_oracle_route.argtypes = [C.POINTER(Cfg), vp, i64, vp, vp, vp, vp, vp, vp]
             L.moe_oracle_expert_ffn.argtypes = [C.POINTER(Cfg), vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -78,8 +83,8 @@ def num_threads() -> int:
     return int(lib().moe_oracle_num_threads())
 
 
-def cfg(H, I, Nr, Kr, Ns=1, n_groups=0, topk_groups=0, route_scale=1.0) -> Cfg:
-    return Cfg(H, I, Nr, Kr, Ns, n_groups, topk_groups, 0, route_scale)
+def cfg(H, I, Nr, Kr, Ns=1, n_groups=0, topk_groups=0, route_scale=1.0, scale_mode=SCALE_AMAX) -> Cfg:
+    return Cfg(H, I, Nr, Kr, Ns, n_groups, topk_groups, scale_mode, route_scale)
 
 
 def _f32(a) -> np.ndarray:
@@ -114,7 +119,7 @@ def e4m3_decode_table() -> np.ndarray:
 
 
 # ------------------------------------------------------------- quantizers
-def quant_1x128(x) -> tuple[np.ndarray, np.ndarray]:
+def quant_1x128(x, mode: int = SCALE_AMAX) -> tuple[np.ndarray, np.ndarray]:
     """1x128 activation quantizer: x bf16 [rows, cols] -> (codes u8 [rows,
     cols], scales f32 [rows, cols/128])."""
     xu = _u16(x)
@@ -122,20 +127,20 @@ def quant_1x128(x) -> tuple[np.ndarray, np.ndarray]:
     assert cols % 128 == 0
     q = np.empty((rows, cols), np.uint8)
     s = np.empty((rows, cols // 128), np.float32)
-    lib().moe_oracle_quant_1x128_bf16(_p(xu), rows, cols, cols, _p(q), _p(s))
+    lib().moe_oracle_quant_1x128_bf16(_p(xu), rows, cols, cols, _p(q), _p(s), int(mode))
     return q, s
 
 
-def quant_1x128_f32(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+def quant_1x128_f32(x: np.ndarray, mode: int = SCALE_AMAX) -> tuple[np.ndarray, np.ndarray]:
     x = np.ascontiguousarray(x, dtype=np.float32)
     rows, cols = x.shape
     q = np.empty((rows, cols), np.uint8)
     s = np.empty((rows, cols // 128), np.float32)
-    lib().moe_oracle_quant_1x128_f32(_p(x), rows, cols, _p(q), _p(s))
+    lib().moe_oracle_quant_1x128_f32(_p(x), rows, cols, _p(q), _p(s), int(mode))
     return q, s
 
 
-def quant_128x128(w) -> tuple[np.ndarray, np.ndarray]:
+def quant_128x128(w, mode: int = SCALE_AMAX) -> tuple[np.ndarray, np.ndarray]:
     """128x128 weight quantizer: w bf16 [n, k] -> (codes [n, k], scales f32
     [n/128, k/128])."""
     wu = _u16(w)
@@ -143,7 +148,7 @@ def quant_128x128(w) -> tuple[np.ndarray, np.ndarray]:
     assert n % 128 == 0 and k % 128 == 0
     q = np.empty((n, k), np.uint8)
     s = np.empty((n // 128, k // 128), np.float32)
-    lib().moe_oracle_quant_128x128(_p(wu), n, k, _p(q), _p(s))
+    lib().moe_oracle_quant_128x128(_p(wu), n, k, _p(q), _p(s), int(mode))
     return q, s
 
 

@@ -115,8 +115,25 @@ uint8_t moe_oracle_e4m3_encode(float xf)
 
 /* Shared step of both quantizers: with S = amax/448 in FP32 ([P1]), each
  * element's code is E4M3(x/S) with x/S an IEEE FP32 quotient.  amax == 0 gives
- * S = 0 and all codes 0x00. */
-static float scale_from_amax(float amax) { return amax / 448.0f; }
+ * S = 0 and all codes 0x00.
+ *
+ * Scale mode 1 (not on the pages: the variant whose scales a tensor core can
+ * apply itself, power-of-two "E8M0" scale factors): S = 2^e with e the
+ * smallest integer for which amax <= 448 * 2^e, so the tile's largest
+ * magnitude still fits the E4M3 range and x/S is an exact power-of-two
+ * scaling; e is held at -127 or above (the smallest such scale factor).
+ * amax == 0 again gives S = 0. */
+static float scale_pow2(float amax)
+{
+    if (amax == 0.0f) return 0.0f;
+    const double a = (double)amax;
+    int e = ilogb(a) - 9;                  /* 448 * 2^e < a here */
+    while (ldexp(448.0, e) < a) ++e;       /* exact comparisons in double: the first e that fits */
+    if (e < -127) e = -127;
+    return (float)ldexp(1.0, e);           /* exact: 2^e >= 2^-127 is a float */
+}
+
+static float scale_for(float amax, int mode) { return mode ? scale_pow2(amax) : amax / 448.0f; }
 
 static uint8_t code_of(float x, float S)
 {
@@ -129,7 +146,7 @@ static uint8_t code_of(float x, float S)
  * 128 consecutive columns.  x is bf16 [rows, ldx], q [rows, cols], s [rows,
  * cols/128]. */
 void moe_oracle_quant_1x128_bf16(const uint16_t *x, int64_t rows, int64_t cols, int64_t ldx,
-                                 uint8_t *q, float *s)
+                                 uint8_t *q, float *s, int mode)
 {
     int64_t ng = cols / QBLK;
 #pragma omp parallel for schedule(static)
@@ -141,7 +158,7 @@ void moe_oracle_quant_1x128_bf16(const uint16_t *x, int64_t rows, int64_t cols, 
                 float a = fabsf(bf16_to_float(xr[j]));
                 if (a > amax) amax = a;
             }
-            float S = scale_from_amax(amax);
+            float S = scale_for(amax, mode);
             s[r * ng + g] = S;
             for (int j = 0; j < QBLK; ++j)
                 q[r * cols + g * QBLK + j] = code_of(bf16_to_float(xr[j]), S);
@@ -151,7 +168,7 @@ void moe_oracle_quant_1x128_bf16(const uint16_t *x, int64_t rows, int64_t cols, 
 
 /* Same tiling for an FP32 input (the SwiGLU output h before the down
  * projection, re-quantized along the intermediate dimension). */
-void moe_oracle_quant_1x128_f32(const float *x, int64_t rows, int64_t cols, uint8_t *q, float *s)
+void moe_oracle_quant_1x128_f32(const float *x, int64_t rows, int64_t cols, uint8_t *q, float *s, int mode)
 {
     int64_t ng = cols / QBLK;
     for (int64_t r = 0; r < rows; ++r) {
@@ -162,7 +179,7 @@ void moe_oracle_quant_1x128_f32(const float *x, int64_t rows, int64_t cols, uint
                 float a = fabsf(xr[j]);
                 if (a > amax) amax = a;
             }
-            float S = scale_from_amax(amax);
+            float S = scale_for(amax, mode);
             s[r * ng + g] = S;
             for (int j = 0; j < QBLK; ++j) q[r * cols + g * QBLK + j] = code_of(xr[j], S);
         }
@@ -171,7 +188,7 @@ void moe_oracle_quant_1x128_f32(const float *x, int64_t rows, int64_t cols, uint
 
 /* 128x128 weight blocks ([P4] "Kernideen", [P2]): w bf16 [n, k] (rows = output
  * features, k contiguous), q [n, k], s [n/128, k/128]. */
-void moe_oracle_quant_128x128(const uint16_t *w, int64_t n, int64_t k, uint8_t *q, float *s)
+void moe_oracle_quant_128x128(const uint16_t *w, int64_t n, int64_t k, uint8_t *q, float *s, int mode)
 {
     int64_t nb = n / QBLK, kb = k / QBLK;
 #pragma omp parallel for collapse(2) schedule(static)
@@ -183,7 +200,7 @@ void moe_oracle_quant_128x128(const uint16_t *w, int64_t n, int64_t k, uint8_t *
                     float a = fabsf(bf16_to_float(w[(bi * QBLK + i) * k + bj * QBLK + j]));
                     if (a > amax) amax = a;
                 }
-            float S = scale_from_amax(amax);
+            float S = scale_for(amax, mode);
             s[bi * kb + bj] = S;
             for (int i = 0; i < QBLK; ++i)
                 for (int j = 0; j < QBLK; ++j) {
@@ -256,7 +273,8 @@ void moe_oracle_blockscaled_gemm(const uint8_t *A, const float *sA, const uint8_
  * gap[t] is min over the decision boundaries taken for token t of (last
  * chosen - first rejected) score, so near-ties can be recognised. */
 typedef struct {
-    int32_t H, I, Nr, Kr, Ns, n_groups, topk_groups, pad;
+    int32_t H, I, Nr, Kr, Ns, n_groups, topk_groups;
+    int32_t scale_mode; /* 0: S = amax/448 (the pages); 1: power-of-two S (see scale_pow2) */
     double route_scale;
 } moe_oracle_cfg;
 
@@ -365,7 +383,7 @@ static void expert_ffn(const moe_oracle_cfg *cf, const uint8_t *xq, const float 
         double silu = g / (1.0 + exp(-g));
         h_buf[j] = (float)(silu * (double)U);
     }
-    moe_oracle_quant_1x128_f32(h_buf, 1, I, hq_buf, hs_buf);
+    moe_oracle_quant_1x128_f32(h_buf, 1, I, hq_buf, hs_buf, cf->scale_mode);
     for (int n = 0; n < H; ++n)
         y[n] = scaled_row_dot(hq_buf, hs_buf, W2q + (int64_t)n * I, s2 + (int64_t)(n / QBLK) * ik, I);
 }
@@ -434,7 +452,7 @@ int moe_oracle_forward(const moe_oracle_cfg *cf, const uint16_t *x, const int64_
         for (int64_t r = 0; r < n_tok; ++r) {
             const uint16_t *u = x + tokens[r] * H;
             double *o = out + r * H;
-            moe_oracle_quant_1x128_bf16(u, 1, H, H, xq, xs);
+            moe_oracle_quant_1x128_bf16(u, 1, H, H, xq, xs, cf->scale_mode);
             route_token(u, Wr, bias, cf, idx + r * Kr, gate + r * Kr, gap + r, s_buf, c_buf, ok);
             for (int n = 0; n < H; ++n) o[n] = (double)bf16_to_float(u[n]);
             for (int e = Nr; e < Nr + Ns; ++e) {

@@ -12,24 +12,27 @@ against the identity that makes routing irrelevant (all routed experts equal
 the bias update against its closed form.
 """
 import numpy as np
+import pytest
 import torch
 
 from moe_synth import TINY, gen_bias, gen_expert, gen_router, gen_x
 
 
-def _quant_expert(oracle_lib, e, H, I, seed):
+def _quant_expert(oracle_lib, e, H, I, seed, mode=0):
     w13, w2 = gen_expert(e, H, I, seed)
-    W13q, s13 = oracle_lib.quant_128x128(w13)
-    W2q, s2 = oracle_lib.quant_128x128(w2)
+    W13q, s13 = oracle_lib.quant_128x128(w13, mode)
+    W2q, s2 = oracle_lib.quant_128x128(w2, mode)
     return W13q, s13, W2q, s2
 
 
-def test_ffn_matches_dense_swiglu_of_dequantized(oracle_lib):
+# scale mode 0: S = amax/448 (the pages); 1: power-of-two scales
+@pytest.mark.parametrize("mode", [0, 1])
+def test_ffn_matches_dense_swiglu_of_dequantized(oracle_lib, mode):
     H, I = 512, 256
-    cf = oracle_lib.cfg(H, I, 4, 2)
+    cf = oracle_lib.cfg(H, I, 4, 2, scale_mode=mode)
     x = gen_x(24, H, 0)
-    xq, xs = oracle_lib.quant_1x128(x)
-    W13q, s13, W2q, s2 = _quant_expert(oracle_lib, 0, H, I, 0)
+    xq, xs = oracle_lib.quant_1x128(x, mode)
+    W13q, s13, W2q, s2 = _quant_expert(oracle_lib, 0, H, I, 0, mode)
     y, h, hq, hs = oracle_lib.expert_ffn(cf, xq, xs, W13q, s13, W2q, s2, want_h=True)
     Xd = oracle_lib.dequant(xq, xs, 1)
     W13d = oracle_lib.dequant(W13q, s13, 128)
@@ -38,24 +41,25 @@ def test_ffn_matches_dense_swiglu_of_dequantized(oracle_lib):
     U = GU[:, I:].astype(np.float32).astype(np.float64)
     h_ref = (G / (1.0 + np.exp(-G)) * U).astype(np.float32)
     assert np.allclose(h, h_ref, rtol=2e-7, atol=0)
-    hq_ref, hs_ref = oracle_lib.quant_1x128_f32(h_ref)
+    hq_ref, hs_ref = oracle_lib.quant_1x128_f32(h_ref, mode)
     assert (hq == hq_ref).mean() > 0.9999
     W2d = oracle_lib.dequant(W2q, s2, 128)
     y_ref = oracle_lib.dequant(hq_ref, hs_ref, 1) @ W2d.T
     assert np.allclose(y, y_ref, rtol=0, atol=1e-6 * np.abs(y_ref).max())
 
 
-def test_layer_identity_all_routed_experts_equal(oracle_lib):
+@pytest.mark.parametrize("mode", [0, 1])
+def test_layer_identity_all_routed_experts_equal(oracle_lib, mode):
     c = TINY
     H, I, Nr, Kr = c["H"], c["I"], c["Nr"], c["Kr"]
-    cf = oracle_lib.cfg(H, I, Nr, Kr)
+    cf = oracle_lib.cfg(H, I, Nr, Kr, scale_mode=mode)
     x = gen_x(32, H, 1)
     Wr = gen_router(Nr, H, 1)
     b = gen_bias(Nr, 1)
-    shared = _quant_expert(oracle_lib, Nr, H, I, 1)
-    same = _quant_expert(oracle_lib, 0, H, I, 1)
+    shared = _quant_expert(oracle_lib, Nr, H, I, 1, mode)
+    same = _quant_expert(oracle_lib, 0, H, I, 1, mode)
     res = oracle_lib.forward(cf, x, Wr, b, [same] * Nr + [shared])
-    xq, xs = oracle_lib.quant_1x128(x)
+    xq, xs = oracle_lib.quant_1x128(x, mode)
     y_sh = oracle_lib.expert_ffn(cf, xq, xs, *shared)
     y_w = oracle_lib.expert_ffn(cf, xq, xs, *same)
     want = x.double().numpy() + y_sh + y_w
