@@ -37,7 +37,8 @@ METRIC = "MoE-layer tokens/s and grouped FP8 GEMM TFLOP/s (% of B200 FP8 / HBM r
 KERNELS_PER_STEP = 11  # quantize, router GEMM, top-k, histogram, chunk table, ranks, row copy, 2 GEMMs, combine,
 #                        bias update
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-GEMM_SOURCES = [os.path.join(ROOT, "sparse_moe_layer_expert_b200", "csrc", f) for f in ("gemm.cu", "common.cuh")]
+GEMM_SOURCES = [os.path.join(ROOT, "sparse_moe_layer_expert_b200", "csrc", f)
+                for f in ("gemm.cu", "gemm_tiles.cuh", "common.cuh")]
 
 
 def parse(argv=None):

@@ -330,6 +330,28 @@ __device__ __forceinline__ void ffma2_scalar(float &c_lo, float &c_hi, float p_l
   asm("mov.b64 {%0, %1}, %2;" : "=f"(c_lo), "=f"(c_hi) : "l"(c));
 }
 
+// Power-of-two scale, the variant whose scale factors a tensor core applies
+// itself (block-scaled MMA with 8-bit exponent scale factors): S = 2^e with e
+// the smallest integer for which amax <= 448 * 2^e, held at 2^-127 or above;
+// amax == 0 gives 0.  With amax = 1.m * 2^E and 448 = 1.75 * 2^8, e = E - 8
+// when 1.m <= 1.75 and E - 7 otherwise.  The exponent byte of the returned
+// float is the scale factor's 8-bit code (2^-127 is the float subnormal with
+// exponent byte 0).
+__device__ __forceinline__ float pow2_scale(float amax) {
+  if (!(amax > 0.0f)) return 0.0f;
+  uint32_t b = __float_as_uint(amax);
+  int E = static_cast<int>(b >> 23) - 127;
+  uint32_t m = b & 0x7FFFFFu;
+  if ((b >> 23) == 0) {  // subnormal: amax = m * 2^-149, leading bit at p
+    const int p = 31 - __clz(m);
+    E = p - 149;
+    m = (m << (23 - p)) & 0x7FFFFFu;
+  }
+  int e = (m <= 0x600000u) ? E - 8 : E - 7;
+  if (e < -127) e = -127;
+  return e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
 // Two E4M3 codes (round to nearest even, saturating) packed low = a, high = b.
 __device__ __forceinline__ uint32_t e4m3x2_rn_sat(float a, float b) {
   return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));

@@ -60,9 +60,11 @@ struct GemmLaunch {
   uint64_t wait_limit_ns;
 };
 
+// pow2: power-of-two scales (pow2_scale) instead of S = amax / 448
 cudaError_t launch_quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ldx, uint8_t *q, float *s,
-                               cudaStream_t st);
-cudaError_t launch_quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *s, cudaStream_t st);
+                               cudaStream_t st, bool pow2 = false);
+cudaError_t launch_quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *s, cudaStream_t st,
+                                 bool pow2 = false);
 
 int router_ksplit(int64_t T, int Nr, int H);
 // capacity of the fixed router scratch used by moe_route_noalloc (floats)

@@ -6,6 +6,8 @@
 // paragraph: S = max|X| / 448 and X_FP8 = clip(round(X / S), -448, 448).
 // The quotient X / S is an IEEE FP32 division (this file is compiled without
 // fast-math) and the cast rounds to nearest even, saturating at +-448.
+// POW2 = true: the power-of-two scale variant (pow2_scale in common.cuh),
+// for which X / S is an exact scaling.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,6 +34,7 @@ __device__ __forceinline__ uint2 codes8(const float (&f)[8], float S) {
 }
 
 // 1x128 tiles: 16 lanes per tile, 8 bf16 (one 16-byte load) per lane.
+template <bool POW2>
 __global__ void __launch_bounds__(256) quant_1x128_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
                                                            int64_t cols, int64_t ldx, uint8_t *__restrict__ q,
                                                            float *__restrict__ s) {
@@ -51,7 +54,7 @@ __global__ void __launch_bounds__(256) quant_1x128_kernel(const __nv_bfloat16 *_
   for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float S = amax / 448.0f;
+  const float S = POW2 ? pow2_scale(amax) : amax / 448.0f;
   if (valid) {
     *reinterpret_cast<uint2 *>(q + r * cols + g * 128 + sub * 8) = codes8(f, S);
     if (sub == 0) s[r * groups_per_row + g] = S;
@@ -59,6 +62,7 @@ __global__ void __launch_bounds__(256) quant_1x128_kernel(const __nv_bfloat16 *_
 }
 
 // 128x128 blocks: one CTA of 256 threads per block, 8 x 16-byte chunks each.
+template <bool POW2>
 __global__ void __launch_bounds__(256) quant_128x128_kernel(const __nv_bfloat16 *__restrict__ w, int64_t n,
                                                              int64_t k, uint8_t *__restrict__ q,
                                                              float *__restrict__ s) {
@@ -84,7 +88,7 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(const __nv_bfloat16 
   amax = red[0];
 #pragma unroll
   for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
-  const float S = amax / 448.0f;
+  const float S = POW2 ? pow2_scale(amax) : amax / 448.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int c = i * 256 + tid;
@@ -95,21 +99,28 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(const __nv_bfloat16 
 }
 
 cudaError_t launch_quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ldx, uint8_t *q, float *s,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool pow2) {
   const int64_t groups = rows * (cols / 128);
   if (groups == 0) return cudaSuccess;
   const int64_t threads = groups * 16;
   const int64_t blocks = (threads + 255) / 256;
-  quant_1x128_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16 *>(x), rows, cols, ldx, q, s);
+  const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+  if (pow2)
+    quant_1x128_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(xb, rows, cols, ldx, q, s);
+  else
+    quant_1x128_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(xb, rows, cols, ldx, q, s);
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *s, cudaStream_t st) {
+cudaError_t launch_quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *s, cudaStream_t st,
+                                 bool pow2) {
   const int64_t blocks = (n / 128) * (k / 128);
   if (blocks == 0) return cudaSuccess;
-  quant_128x128_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(w), n,
-                                                                       k, q, s);
+  const auto *wb = static_cast<const __nv_bfloat16 *>(w);
+  if (pow2)
+    quant_128x128_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(wb, n, k, q, s);
+  else
+    quant_128x128_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(wb, n, k, q, s);
   return cudaGetLastError();
 }
 
