@@ -91,7 +91,15 @@ MOE_API int moe_abi_version(void);
  *   n_groups    group-limited routing: 0 = off, else number of equal
  *               contiguous expert groups (divides N_r, <= 32)
  *   topk_groups groups kept per token when n_groups > 0 (1..n_groups)
- *   route_scale factor applied to the normalised gates (1.0 = the pages') */
+ *   route_scale factor applied to the normalised gates (1.0 = the pages')
+ *   scale_mode  MOE_SCALE_AMAX (0, the pages' S = amax / 448, the default of
+ *               a zero-initialised config) or MOE_SCALE_POW2 (1: power-of-two
+ *               scales, see fp8_quant_1x128_pow2; moe_forward then runs the
+ *               expert GEMMs with the scales applied by the tensor core, and
+ *               the weights must have been quantized with the _pow2
+ *               quantizer) */
+#define MOE_SCALE_AMAX 0
+#define MOE_SCALE_POW2 1
 typedef struct {
     int32_t hidden;
     int32_t inter;
@@ -101,6 +109,7 @@ typedef struct {
     int32_t n_groups;
     int32_t topk_groups;
     float route_scale;
+    int32_t scale_mode;
 } moe_config;
 
 /* Quantized layer weights, all device pointers, experts stacked routed
@@ -140,6 +149,17 @@ MOE_API int fp8_quant_1x128(const void *x_dev, int64_t rows, int64_t cols, int64
  *   q_dev       E4M3 [n, k];  scales_dev float [n/128, k/128] */
 MOE_API int fp8_quant_128x128(const void *w_dev, int64_t n, int64_t k, uint8_t *q_dev, float *scales_dev,
                       void *stream);
+
+/* The same two quantizers with power-of-two scales (not on the pages: the
+ * variant whose scales a block-scaled tensor-core MMA applies itself, as
+ * 8-bit exponent codes): S = 2^e with e the smallest integer for which
+ * amax <= 448 * 2^e, held at 2^-127 or above; amax == 0 gives S = 0.  x / S
+ * is then an exact scaling and q = E4M3_RNE_satfinite(x / S).  Arguments,
+ * layouts and errors as above. */
+MOE_API int fp8_quant_1x128_pow2(const void *x_dev, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q_dev,
+                         float *scales_dev, void *stream);
+MOE_API int fp8_quant_128x128_pow2(const void *w_dev, int64_t n, int64_t k, uint8_t *q_dev, float *scales_dev,
+                           void *stream);
 
 /* ---------------------------------------------------------------- GEMM */
 /* Fine-grained block-scaled FP8 GEMM ([P4] Kernideen):

@@ -34,9 +34,12 @@ MOE_DEVERR_TIMEOUT = 1
 MOE_DEVERR_BAD_INDEX = 2
 MOE_DTYPE_BF16 = 0
 MOE_DTYPE_F32 = 1
+MOE_SCALE_AMAX = 0  # S = amax / 448 (the pages)
+MOE_SCALE_POW2 = 1  # power-of-two scales, applied by the tensor core
 
 EXPORTS = (
-    "moe_status_string", "moe_abi_version", "fp8_quant_1x128", "fp8_quant_128x128", "fp8_blockscaled_gemm",
+    "moe_status_string", "moe_abi_version", "fp8_quant_1x128", "fp8_quant_128x128", "fp8_quant_1x128_pow2",
+    "fp8_quant_128x128_pow2", "fp8_blockscaled_gemm",
     "moe_route_workspace_size", "moe_route", "moe_workspace_size", "moe_forward", "moe_workspace_layout",
     "moe_bias_update", "moe_check_device_error", "moe_selftest_wait_timeout", "moe_profile_events",
     "moe_route_noalloc",
@@ -49,7 +52,7 @@ PROFILE_STAGES = ("quantize", "route", "group", "gemm_gate_up", "gemm_down", "co
 class MoeConfig(C.Structure):
     _fields_ = [("hidden", C.c_int32), ("inter", C.c_int32), ("n_routed", C.c_int32), ("top_k", C.c_int32),
                 ("n_shared", C.c_int32), ("n_groups", C.c_int32), ("topk_groups", C.c_int32),
-                ("route_scale", C.c_float)]
+                ("route_scale", C.c_float), ("scale_mode", C.c_int32)]
 
 
 class MoeWeights(C.Structure):
@@ -72,6 +75,8 @@ lib.moe_status_string.argtypes = [C.c_int]
 lib.moe_abi_version.restype = C.c_int
 lib.fp8_quant_1x128.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp]
 lib.fp8_quant_128x128.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
+lib.fp8_quant_1x128_pow2.argtypes = lib.fp8_quant_1x128.argtypes
+lib.fp8_quant_128x128_pow2.argtypes = lib.fp8_quant_128x128.argtypes
 lib.fp8_blockscaled_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]
 lib.moe_route_workspace_size.restype = _sz
 lib.moe_route_workspace_size.argtypes = [_cfgp, _i64]
@@ -111,13 +116,14 @@ def _stream(stream) -> int | None:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def config(hidden, inter, n_routed, top_k, n_shared=1, n_groups=0, topk_groups=0, route_scale=1.0) -> MoeConfig:
-    return MoeConfig(hidden, inter, n_routed, top_k, n_shared, n_groups, topk_groups, route_scale)
+def config(hidden, inter, n_routed, top_k, n_shared=1, n_groups=0, topk_groups=0, route_scale=1.0,
+           scale_mode=MOE_SCALE_AMAX) -> MoeConfig:
+    return MoeConfig(hidden, inter, n_routed, top_k, n_shared, n_groups, topk_groups, route_scale, scale_mode)
 
 
 def config_from(d: dict) -> MoeConfig:
     return config(d["H"], d["I"], d["Nr"], d["Kr"], d.get("Ns", 1), d.get("n_groups", 0), d.get("topk_groups", 0),
-                  d.get("route_scale", 1.0))
+                  d.get("route_scale", 1.0), d.get("scale_mode", MOE_SCALE_AMAX))
 
 
 def new_err_flag(device="cuda") -> torch.Tensor:
@@ -125,23 +131,25 @@ def new_err_flag(device="cuda") -> torch.Tensor:
 
 
 # ------------------------------------------------------------------ calls
-def fp8_quant_1x128(x: torch.Tensor, q=None, scales=None, stream=None):
+def fp8_quant_1x128(x: torch.Tensor, q=None, scales=None, stream=None, pow2: bool = False):
     rows, cols = x.shape
     ld = x.stride(0)
     assert x.stride(1) == 1 and x.dtype == torch.bfloat16
     q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device) if q is None else q
     scales = torch.empty((rows, cols // 128), dtype=torch.float32, device=x.device) if scales is None else scales
-    _check(lib.fp8_quant_1x128(_ptr(x), rows, cols, ld, _ptr(q), _ptr(scales), _stream(stream)), "fp8_quant_1x128")
+    fn = lib.fp8_quant_1x128_pow2 if pow2 else lib.fp8_quant_1x128
+    _check(fn(_ptr(x), rows, cols, ld, _ptr(q), _ptr(scales), _stream(stream)), "fp8_quant_1x128")
     return q, scales
 
 
-def fp8_quant_128x128(w: torch.Tensor, q=None, scales=None, stream=None):
+def fp8_quant_128x128(w: torch.Tensor, q=None, scales=None, stream=None, pow2: bool = False):
     assert w.is_contiguous() and w.dtype == torch.bfloat16
     n, k = w.shape[-2] * (w.numel() // (w.shape[-2] * w.shape[-1])), w.shape[-1]
     q = torch.empty(w.shape, dtype=torch.uint8, device=w.device) if q is None else q
     if scales is None:
         scales = torch.empty(w.shape[:-2] + (w.shape[-2] // 128, k // 128), dtype=torch.float32, device=w.device)
-    _check(lib.fp8_quant_128x128(_ptr(w), n, k, _ptr(q), _ptr(scales), _stream(stream)), "fp8_quant_128x128")
+    fn = lib.fp8_quant_128x128_pow2 if pow2 else lib.fp8_quant_128x128
+    _check(fn(_ptr(w), n, k, _ptr(q), _ptr(scales), _stream(stream)), "fp8_quant_128x128")
     return q, scales
 
 

@@ -92,6 +92,7 @@ int check_cfg(const moe_config *c) {
     if (static_cast<int64_t>(c->topk_groups) * (c->n_routed / c->n_groups) < c->top_k) return MOE_ERR_INVALID_ARG;
   }
   if (!(c->route_scale == c->route_scale)) return MOE_ERR_INVALID_ARG;
+  if (c->scale_mode != MOE_SCALE_AMAX && c->scale_mode != MOE_SCALE_POW2) return MOE_ERR_INVALID_ARG;
   // weight rows must be addressable by 32-bit TMA coordinates
   const int64_t E = static_cast<int64_t>(c->n_routed) + c->n_shared;
   if (E * 2 * c->inter > INT32_MAX || E * c->hidden > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -171,20 +172,32 @@ const char *moe_status_string(int s) {
   }
 }
 
-int moe_abi_version(void) { return 100; }
+int moe_abi_version(void) { return 101; }
 
-int fp8_quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q, float *scales,
-                    void *stream) {
+static int quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q, float *scales,
+                       void *stream, bool pow2) {
   if (rows < 0 || cols <= 0 || ld_x < cols || (ld_x % 8) != 0) return MOE_ERR_INVALID_ARG;
   if (cols % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (rows == 0) return MOE_OK;
   if (!x || !q || !scales || !aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 3))
     return MOE_ERR_INVALID_ARG;
   if (const int d = check_device()) return d;
-  return cuda_status(moe::launch_quant_1x128(x, rows, cols, ld_x, q, scales, static_cast<cudaStream_t>(stream)));
+  return cuda_status(
+      moe::launch_quant_1x128(x, rows, cols, ld_x, q, scales, static_cast<cudaStream_t>(stream), pow2));
 }
 
-int fp8_quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *scales, void *stream) {
+int fp8_quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q, float *scales,
+                    void *stream) {
+  return quant_1x128(x, rows, cols, ld_x, q, scales, stream, false);
+}
+
+int fp8_quant_1x128_pow2(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q, float *scales,
+                         void *stream) {
+  return quant_1x128(x, rows, cols, ld_x, q, scales, stream, true);
+}
+
+static int quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *scales, void *stream,
+                         bool pow2) {
   if (n < 0 || k < 0) return MOE_ERR_INVALID_ARG;
   if (n % 128 || k % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (n == 0 || k == 0) return MOE_OK;
@@ -192,7 +205,15 @@ int fp8_quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *sc
     return MOE_ERR_INVALID_ARG;
   if ((n / 128) * (k / 128) > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (const int d = check_device()) return d;
-  return cuda_status(moe::launch_quant_128x128(w, n, k, q, scales, static_cast<cudaStream_t>(stream)));
+  return cuda_status(moe::launch_quant_128x128(w, n, k, q, scales, static_cast<cudaStream_t>(stream), pow2));
+}
+
+int fp8_quant_128x128(const void *w, int64_t n, int64_t k, uint8_t *q, float *scales, void *stream) {
+  return quant_128x128(w, n, k, q, scales, stream, false);
+}
+
+int fp8_quant_128x128_pow2(const void *w, int64_t n, int64_t k, uint8_t *q, float *scales, void *stream) {
+  return quant_128x128(w, n, k, q, scales, stream, true);
 }
 
 int fp8_blockscaled_gemm(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB, void *C, int64_t M,
@@ -357,7 +378,8 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
   const int64_t max_chunks = moe::max_chunks(T, Kr, Nr, Ns);
 
   cudaError_t e = prof_mark(0, st);
-  if (e == cudaSuccess) e = moe::launch_quant_1x128(x, T, H, H, xq, xs, st);
+  const bool pow2 = cfg->scale_mode == MOE_SCALE_POW2;
+  if (e == cudaSuccess) e = moe::launch_quant_1x128(x, T, H, H, xq, xs, st, pow2);
   if (e == cudaSuccess) e = prof_mark(1, st);
   if (e == cudaSuccess)
     e = moe::launch_router_logits(x, w->wr_dev, T, Nr, H, logits, err_flag, moe::kDefaultWaitLimitNs, st);
@@ -403,7 +425,7 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
     g.ld_os = pitch;
     g.err = err_flag;
     g.wait_limit_ns = moe::kDefaultWaitLimitNs;
-    e = moe::launch_gemm(g, st);
+    e = pow2 ? moe::launch_gemm_mx(g, st) : moe::launch_gemm(g, st);
   }
   if (e == cudaSuccess) e = prof_mark(4, st);
   if (e == cudaSuccess) {
@@ -436,7 +458,7 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
     g.row_gate = row_gate;
     g.err = err_flag;
     g.wait_limit_ns = moe::kDefaultWaitLimitNs;
-    e = moe::launch_gemm(g, st);
+    e = pow2 ? moe::launch_gemm_mx(g, st) : moe::launch_gemm(g, st);
   }
   if (e == cudaSuccess) e = prof_mark(5, st);
   if (e == cudaSuccess) e = moe::launch_combine(x, y, pos, T, H, Kr, R, Ns, out, out_dtype == MOE_DTYPE_F32, st);

@@ -118,6 +118,12 @@ __device__ __forceinline__ bool mbar_wait2(uint64_t *bar1, uint32_t parity1, uin
   return (a || mbar_wait(bar1, parity1, ctl)) && (b || mbar_wait(bar2, parity2, ctl));
 }
 
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy reads of them (TMA, tcgen05.cp, tcgen05.mma operands).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -92,6 +92,10 @@ inline int64_t scale_pitch(int64_t R, int64_t T) { return (R + T + 3) / 4 * 4; }
 constexpr int64_t kScaleSlack = 132;
 
 cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st);
+// The same grouped GEMM with power-of-two scales applied by the tensor core
+// (block-scaled MMA); transposed activation scales, EPI_SWIGLU_Q (with
+// power-of-two requantization) or EPI_GATE_F32 only.
+cudaError_t launch_gemm_mx(const GemmLaunch &g, cudaStream_t st);
 
 cudaError_t launch_combine(const void *x, const float *y, const int32_t *pos, int64_t T, int H, int Kr,
                            int64_t R, int Ns, void *out, int out_f32, cudaStream_t st);

@@ -33,9 +33,11 @@ class MoeLayer:
 
     # -------------------------------------------------------------- weights
     def set_expert(self, e: int, w13_bf16: torch.Tensor, w2_bf16: torch.Tensor, stream=None) -> None:
-        """Quantize expert e's bf16 weights (128x128 blocks) into place."""
-        B.fp8_quant_128x128(w13_bf16.contiguous(), q=self.w13[e], scales=self.s13[e], stream=stream)
-        B.fp8_quant_128x128(w2_bf16.contiguous(), q=self.w2[e], scales=self.s2[e], stream=stream)
+        """Quantize expert e's bf16 weights (128x128 blocks) into place, with
+        the scale rule of the layer's scale mode."""
+        pow2 = self.cfg.scale_mode == B.MOE_SCALE_POW2
+        B.fp8_quant_128x128(w13_bf16.contiguous(), q=self.w13[e], scales=self.s13[e], stream=stream, pow2=pow2)
+        B.fp8_quant_128x128(w2_bf16.contiguous(), q=self.w2[e], scales=self.s2[e], stream=stream, pow2=pow2)
 
     def set_router(self, wr_bf16: torch.Tensor, bias: torch.Tensor) -> None:
         self.wr.copy_(wr_bf16)

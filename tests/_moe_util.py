@@ -61,12 +61,12 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
 
 
 def shape_of(cfg: dict) -> dict:
-    return {k: cfg[k] for k in ("H", "I", "Nr", "Kr", "Ns", "n_groups", "topk_groups") if k in cfg}
+    return {k: cfg[k] for k in ("H", "I", "Nr", "Kr", "Ns", "n_groups", "topk_groups", "scale_mode") if k in cfg}
 
 
 def oracle_cfg(oracle, cfg: dict):
     return oracle.cfg(cfg["H"], cfg["I"], cfg["Nr"], cfg["Kr"], cfg.get("Ns", 1), cfg.get("n_groups", 0),
-                      cfg.get("topk_groups", 0), cfg.get("route_scale", 1.0))
+                      cfg.get("topk_groups", 0), cfg.get("route_scale", 1.0), cfg.get("scale_mode", 0))
 
 
 def route_sets_match(idx_gpu: np.ndarray, idx_ref: np.ndarray, gap: np.ndarray):
@@ -106,6 +106,7 @@ class Problem:
 
     def oracle_expert(self, oracle, e: int):
         w13, w2 = self.expert_bf16(e)
-        W13q, s13 = oracle.quant_128x128(w13)
-        W2q, s2 = oracle.quant_128x128(w2)
+        mode = self.cfg.get("scale_mode", 0)
+        W13q, s13 = oracle.quant_128x128(w13, mode)
+        W2q, s2 = oracle.quant_128x128(w2, mode)
         return W13q, s13, W2q, s2

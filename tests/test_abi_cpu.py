@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported(m):
 
 
 def test_status_strings_and_version(m):
-    assert m.lib.moe_abi_version() == 100
+    assert m.lib.moe_abi_version() == 101
     assert m.lib.moe_status_string(0) == b"ok"
     assert b"128" in m.lib.moe_status_string(m.MOE_ERR_UNSUPPORTED_SHAPE)
     assert m.lib.moe_status_string(12345) == b"unknown status"

@@ -81,3 +81,38 @@ def test_quant_rejects_bad_arguments(m):
     with pytest.raises(m.MoeError) as e:  # misaligned base pointer
         m.fp8_quant_1x128(x.contiguous()[:, :] if False else x)
     assert e.value.status in (m.MOE_ERR_INVALID_ARG, m.MOE_ERR_UNSUPPORTED_SHAPE)
+
+
+# ------------------------------------------------ power-of-two scale rule
+def _check_1x128_pow2(m, oracle_lib, x_cpu):
+    q, s = m.fp8_quant_1x128(x_cpu.cuda(), pow2=True)
+    torch.cuda.synchronize()
+    qo, so = oracle_lib.quant_1x128(x_cpu, 1)
+    assert np.array_equal(s.cpu().numpy(), so)
+    assert np.array_equal(q.cpu().numpy(), qo)
+
+
+def test_1x128_pow2_ragged_outliers(m, oracle_lib):
+    _check_1x128_pow2(m, oracle_lib, S.gen_gemm_a(333, 1024, 4))
+
+
+def test_1x128_pow2_thresholds_and_special_tiles(m, oracle_lib):
+    # tiles whose amax sits exactly on, just above and just below a threshold
+    # 448 * 2^e, an all-zero tile, tiny (bf16-subnormal) and huge magnitudes
+    x = S.gen_x(16, 1024, 5)
+    for g, amax in enumerate([448.0, 450.0, 446.0, 224.0, 1.0, 2.0 ** -120, 3.0e38]):
+        x[g, 128 * g:128 * g + 128] = (x[g, 128 * g:128 * g + 128].float().clamp(-0.5, 0.5) *
+                                       (amax if amax < 1e30 else 1.0)).to(torch.bfloat16)
+        x[g, 128 * g + 7] = amax
+    x[9, 256:384] = 0
+    x[10, :128] = (x[10, :128].float() * 2.0 ** -133).to(torch.bfloat16)
+    _check_1x128_pow2(m, oracle_lib, x)
+
+
+def test_128x128_pow2_blocks(m, oracle_lib):
+    w = S.normal_bf16((384, 640), 0.02, 6)
+    q, s = m.fp8_quant_128x128(w.cuda(), pow2=True)
+    torch.cuda.synchronize()
+    qo, so = oracle_lib.quant_128x128(w, 1)
+    assert np.array_equal(s.cpu().numpy(), so)
+    assert np.array_equal(q.cpu().numpy(), qo)
