@@ -52,6 +52,9 @@ def parse(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=8)
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--scale-mode", choices=("amax", "pow2"), default="amax",
+                   help="amax: S = amax/448 (the pages, default); pow2: power-of-two scales applied by the "
+                        "tensor core (block-scaled MMA)")
     p.add_argument("--tokens", type=int, default=0, help="override T (profiling of smaller cases)")
     p.add_argument("--experts", type=int, default=0, help="override N_r (profiling of smaller cases)")
     return p.parse_args(argv)
@@ -267,6 +270,7 @@ def main(argv=None):
     cfg = workload_shape(args.workload, args)
     T = cfg["T"]
     shape = {k: cfg[k] for k in ("H", "I", "Nr", "Kr", "Ns", "n_groups", "topk_groups")}
+    shape["scale_mode"] = M.MOE_SCALE_POW2 if args.scale_mode == "pow2" else M.MOE_SCALE_AMAX
     seed = args.seed
 
     def expert_bf16(e):
@@ -358,7 +362,8 @@ def main(argv=None):
     fp8_peak = 2.0 * peaks["bf16_sustained"]  # FP8 dense = 2 x bf16 (nominal ratio 4.5 / 2.25 PFLOP/s)
     t_mem = dom_bytes / (peaks["hbm"] * 1e9)
     t_tc = dom_flops / (fp8_peak * 1e12)
-    kernel_name = "gemm_fp8_kernel<0>" if dom == "gemm_gate_up" else "gemm_fp8_kernel<1>"
+    kname = "gemm_mx_kernel" if args.scale_mode == "pow2" else "gemm_fp8_kernel"
+    kernel_name = f"{kname}<0>" if dom == "gemm_gate_up" else f"{kname}<1>"
     if t_mem >= t_tc:
         achieved = dom_bytes / (dom_ms / 1e3) / 1e9
         roofline = dict(bound="hbm", achieved=round(achieved, 1), peak=peaks["hbm"], unit="GB/s",
@@ -420,6 +425,8 @@ def main(argv=None):
                              f"Ns={cfg.get('Ns', 1)} groups={cfg.get('n_groups', 0)}/{cfg.get('topk_groups', 0)}",
                     global_batch=world * T, tokens_per_gpu=T, parallelism=f"replicas x{world} (no collective)",
                     l2="no flush: per-step working set >= 11 GB of expert weights >> 126 MB L2",
+                    scales="amax/448 (FP32 promotion per 128-K block)" if args.scale_mode == "amax" else
+                    "power of two (applied by the tensor core, block-scaled MMA)",
                     seed=seed),
         roofline=roofline,
         grouped_gemm_tflops=round(gemm_tflops, 1),

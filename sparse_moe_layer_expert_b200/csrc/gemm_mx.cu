@@ -23,10 +23,10 @@
 //     of the 128-long K block);
 //   * warp 2 builds those atoms from the FP32 scale tables (the code is the
 //     float's exponent byte), loading two K blocks ahead;
-//   * warp 1's lane 0 copies the atoms into TMEM (tcgen05.cp 32x128b.warpx4:
-//     columns 256.. for A, 260.. for the weight blocks) and issues the four
-//     block-scaled MMAs of the K block, slice k reading scale byte k;
-//   * TMEM: accumulator columns 0..255 + 12 scale-factor columns; the
+//   * warp 1's lane 0 copies the atoms into TMEM (tcgen05.cp 32x128b.warpx4;
+//     two sets of 12 columns from column 256, alternate K blocks) and issues
+//     the four block-scaled MMAs of the K block, slice k reading byte k;
+//   * TMEM: accumulator columns 0..255 + the scale-factor columns; the
 //     epilogue warps copy the accumulator to registers, hand TMEM back to the
 //     tensor core (which starts the next tile) and then run the epilogue.
 #include "common.cuh"
@@ -49,8 +49,11 @@ constexpr int X_OUTX = 8 * 32 * G_OPITCH;
 constexpr int X_SMEM = 1024 + X_STAGES * X_STAGE + X_AMAX * 4 + X_OUTX * 4 + 256;
 static_assert(X_SMEM <= 232448, "shared memory budget");
 static_assert(X_STAGE % 1024 == 0, "stage alignment");
-constexpr uint32_t X_TSFA = 256;                // TMEM column of the activation scale factors
-constexpr uint32_t X_TSFB = 260;                // and of the two weight blocks' (4 columns each)
+// TMEM columns of the scale factors, two sets used by alternate K blocks (a
+// copy into one set does not wait for MMAs still reading the other): A at
+// +0, the two weight blocks at +4 and +8.
+constexpr uint32_t X_TSF = 256;
+constexpr uint32_t X_TSF_SET = 16;
 
 struct XBars {
   uint64_t full[X_STAGES];   // TMA bytes + the scale-factor atoms
@@ -191,7 +194,6 @@ __global__ void __launch_bounds__(X_THREADS, 1)
       if (lane == 0) {
         uint32_t it = 0, tcount = 0;
         bool stop = false;
-        const uint32_t t_sfa = tmem + X_TSFA, t_sfb = tmem + X_TSFB;
         for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x) {
           if (*abortp) break;
           const GemmTile td = get_tile(args, tile);
@@ -210,7 +212,8 @@ __global__ void __launch_bounds__(X_THREADS, 1)
             tc_fence_after();
             const uint32_t base = smem_u32(stages + s * X_STAGE);
             // scale factors of this K block into TMEM (ordered before the MMAs
-            // that read them, and after those of the previous K block)
+            // that read them)
+            const uint32_t t_sfa = tmem + X_TSF + (it & 1) * X_TSF_SET, t_sfb = t_sfa + 4;
             tmem_cp_atom(t_sfa, base + X_SF);
             tmem_cp_atom(t_sfb, base + X_SF + 512);
             if (two) tmem_cp_atom(t_sfb + 4, base + X_SF + 1024);
@@ -247,32 +250,45 @@ __global__ void __launch_bounds__(X_THREADS, 1)
         float a[4];
         float wa, wb;
       };
-      auto load = [&](int t, int kb, Sf &v) {
-        const GemmTile d = get_tile(args, t);
-        const float *col = (d.from1 ? args.sa1 : args.sa0) + static_cast<int64_t>(kb) * args.sa_ld + d.out_row;
+      struct Pos {
+        int t, kb;
+        GemmTile d;  // descriptor of tile t, read once per tile
+      };
+      auto load = [&](const Pos &p, Sf &v) {
+        const float *col =
+            (p.d.from1 ? args.sa1 : args.sa0) + static_cast<int64_t>(p.kb) * args.sa_ld + p.d.out_row;
 #pragma unroll
         for (int i = 0; i < 4; ++i) v.a[i] = __ldg(col + lane + 32 * i);
-        v.wa = __ldg(args.sw + static_cast<int64_t>(d.w_row0 >> 7) * KB + kb);
-        v.wb = d.w_row1 >= 0 ? __ldg(args.sw + static_cast<int64_t>(d.w_row1 >> 7) * KB + kb) : 0.0f;
+        v.wa = __ldg(args.sw + static_cast<int64_t>(p.d.w_row0 >> 7) * KB + p.kb);
+        v.wb = p.d.w_row1 >= 0 ? __ldg(args.sw + static_cast<int64_t>(p.d.w_row1 >> 7) * KB + p.kb) : 0.0f;
       };
-      auto advance = [&](int &t, int &kb) {
-        if (++kb == KB) {
-          kb = 0;
-          t = next_valid_tile(args, t + gridDim.x, ntiles);
-        }
+      auto seek = [&](Pos &p, int t) {  // first valid tile from t
+        p.t = next_valid_tile(args, t, ntiles);
+        p.kb = 0;
+        if (p.t < ntiles) p.d = get_tile(args, p.t);
       };
-      int t0 = next_valid_tile(args, blockIdx.x, ntiles), k0 = 0;  // position being written
-      int t1 = t0, k1 = 0, t2 = t0, k2 = 0;                         // and the two after it
+      auto advance = [&](Pos &p) {
+        if (++p.kb == KB) seek(p, p.t + gridDim.x);
+      };
+      // v0: the K block whose atoms are written next; v1, v2: the two after
+      // it (p is the position of v2's K block)
+      Pos p;
+      seek(p, blockIdx.x);
       Sf v0{}, v1{}, v2{};
-      if (t0 < ntiles) load(t0, 0, v0);
-      if (t0 < ntiles) advance(t1, k1);
-      if (t1 < ntiles) load(t1, k1, v1);
-      t2 = t1;
-      k2 = k1;
-      if (t1 < ntiles) advance(t2, k2);
-      if (t2 < ntiles) load(t2, k2, v2);
+      bool h0 = p.t < ntiles;
+      if (h0) {
+        load(p, v0);
+        advance(p);
+      }
+      bool h1 = h0 && p.t < ntiles;
+      if (h1) {
+        load(p, v1);
+        advance(p);
+      }
+      bool h2 = h1 && p.t < ntiles;
+      if (h2) load(p, v2);
       uint32_t it = 0;
-      while (t0 < ntiles) {
+      while (h0) {
         if (*abortp) break;
         const int s = it % X_STAGES;
         if (!mbar_wait(&bars->empty[s], ((it / X_STAGES) & 1) ^ 1, ctl)) break;
@@ -286,19 +302,17 @@ __global__ void __launch_bounds__(X_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->full[s]);
         ++it;
-        // slide the window: the atom after next starts loading now
-        t0 = t1;
-        k0 = k1;
+        // slide the window: the K block after next starts loading now
         v0 = v1;
-        t1 = t2;
-        k1 = k2;
+        h0 = h1;
         v1 = v2;
-        if (t2 < ntiles) {
-          advance(t2, k2);
-          if (t2 < ntiles) load(t2, k2, v2);
+        h1 = h2;
+        if (h2) {
+          advance(p);
+          h2 = p.t < ntiles;
+          if (h2) load(p, v2);
         }
       }
-      (void)k0;
     }
   } else {
     setmaxnreg_inc<224>();

@@ -90,3 +90,29 @@ def test_v3_skewed_layer(m, oracle_lib, v3_layer):
     c = r["counts"]
     print(f"skewed load: max {c.max()} mean {c.mean():.1f} max/mean {c.max() / c.mean():.2f}")
     assert c.max() >= 4 * c.mean()  # the configuration's imbalance (max/mean load >= 4)
+
+
+@pytest.fixture(scope="module")
+def v3_layer_pow2(m):
+    """The same V3 layer with power-of-two scales (block-scaled GEMM path)."""
+    cfg = dict(S.PREFILL)
+    shape = {k: cfg[k] for k in ("H", "I", "Nr", "Kr", "Ns")}
+    shape["scale_mode"] = m.MOE_SCALE_POW2
+    seed = 0
+
+    def gen(e):
+        return S.gen_expert(e, cfg["H"], cfg["I"], seed, device="cuda")
+
+    wr = S.gen_router(cfg["Nr"], cfg["H"], seed, device="cuda")
+    bias = S.gen_bias(cfg["Nr"], seed, "uniform", device="cuda")
+    layer = m.MoeLayer.from_generator(shape, gen, wr, bias)
+    torch.cuda.synchronize()
+    return layer, seed
+
+
+def test_v3_prefill_layer_pow2(m, oracle_lib, v3_layer_pow2):
+    layer, _ = v3_layer_pow2
+    prob = _problem(dict(S.PREFILL, scale_mode=1), 4096, 12, layer, "uniform")
+    rng = np.random.default_rng(14)
+    toks = np.sort(rng.choice(4096, 4, replace=False))
+    check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=True)
