@@ -38,7 +38,7 @@ KERNELS_PER_STEP = 11  # quantize, router GEMM, top-k, histogram, chunk table, r
 #                        bias update
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 GEMM_SOURCES = [os.path.join(ROOT, "sparse_moe_layer_expert_b200", "csrc", f)
-                for f in ("gemm.cu", "gemm_tiles.cuh", "common.cuh")]
+                for f in ("gemm.cu", "gemm_mx.cu", "gemm_tiles.cuh", "common.cuh")]
 
 
 def parse(argv=None):
