@@ -22,7 +22,9 @@
 //     (row / 32) * 4 + slice, the code repeated for the four 32-long slices
 //     of the 128-long K block);
 //   * warp 2 builds those atoms from the FP32 scale tables (the code is the
-//     float's exponent byte), loading two K blocks ahead;
+//     float's exponent byte); its loads run up to 7 K blocks ahead through a
+//     small cp.async ring in shared memory (their latency under load is as
+//     long as the operand loads', so a shallow look-ahead stalls the ring);
 //   * warp 1's lane 0 copies the atoms into TMEM (tcgen05.cp 32x128b.warpx4;
 //     two sets of 12 columns from column 256, alternate K blocks) and issues
 //     the four block-scaled MMAs of the K block, slice k reading byte k;
@@ -46,7 +48,9 @@ constexpr int X_STAGE = X_SF + 2048;            // 50 KB: keeps every stage 1024
 constexpr int X_THREADS = 384;
 constexpr int X_AMAX = 2 * 128;
 constexpr int X_OUTX = 8 * 32 * G_OPITCH;
-constexpr int X_SMEM = 1024 + X_STAGES * X_STAGE + X_AMAX * 4 + X_OUTX * 4 + 256;
+constexpr int X_SR = 8;                         // K blocks of scales the builder keeps in flight
+constexpr int X_SRING = 136;                    // floats per ring slot: 128 row scales, 2 block scales
+constexpr int X_SMEM = 1024 + X_STAGES * X_STAGE + X_AMAX * 4 + X_OUTX * 4 + X_SR * X_SRING * 4 + 256;
 static_assert(X_SMEM <= 232448, "shared memory budget");
 static_assert(X_STAGE % 1024 == 0, "stage alignment");
 // TMEM columns of the scale factors, two sets used by alternate K blocks (a
@@ -115,7 +119,8 @@ __global__ void __launch_bounds__(X_THREADS, 1)
   uint8_t *stages = smem;
   float *amax_x = reinterpret_cast<float *>(smem + X_STAGES * X_STAGE);
   float *outx = amax_x + X_AMAX;
-  XBars *bars = reinterpret_cast<XBars *>(outx + X_OUTX);
+  float *sring = outx + X_OUTX;  // the scale-factor builder's load ring
+  XBars *bars = reinterpret_cast<XBars *>(sring + X_SR * X_SRING);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -244,23 +249,12 @@ __global__ void __launch_bounds__(X_THREADS, 1)
       // [K/128][sa_ld] (column = output row; the tile's 128 rows, padding rows
       // included, stay inside the table and its slack) and one atom per weight
       // block (its single scale in all 128 rows).  Lane l owns rows l, l+32,
-      // l+64, l+96, i.e. the 16-byte group l of each atom.  The loads run two
-      // K blocks ahead of the atom being written.
-      struct Sf {
-        float a[4];
-        float wa, wb;
-      };
+      // l+64, l+96, i.e. the 16-byte group l of each atom.  The scales come
+      // through a ring of X_SR slots filled by cp.async, one commit group per
+      // K block, X_SR - 1 K blocks ahead of the atoms being written.
       struct Pos {
         int t, kb;
         GemmTile d;  // descriptor of tile t, read once per tile
-      };
-      auto load = [&](const Pos &p, Sf &v) {
-        const float *col =
-            (p.d.from1 ? args.sa1 : args.sa0) + static_cast<int64_t>(p.kb) * args.sa_ld + p.d.out_row;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v.a[i] = __ldg(col + lane + 32 * i);
-        v.wa = __ldg(args.sw + static_cast<int64_t>(p.d.w_row0 >> 7) * KB + p.kb);
-        v.wb = p.d.w_row1 >= 0 ? __ldg(args.sw + static_cast<int64_t>(p.d.w_row1 >> 7) * KB + p.kb) : 0.0f;
       };
       auto seek = [&](Pos &p, int t) {  // first valid tile from t
         p.t = next_valid_tile(args, t, ntiles);
@@ -270,49 +264,52 @@ __global__ void __launch_bounds__(X_THREADS, 1)
       auto advance = [&](Pos &p) {
         if (++p.kb == KB) seek(p, p.t + gridDim.x);
       };
-      // v0: the K block whose atoms are written next; v1, v2: the two after
-      // it (p is the position of v2's K block)
-      Pos p;
+      auto issue = [&](const Pos &p, int slot) {
+        float *dst = sring + slot * X_SRING;
+        const float *col =
+            (p.d.from1 ? args.sa1 : args.sa0) + static_cast<int64_t>(p.kb) * args.sa_ld + p.d.out_row;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cp_async4(dst + lane + 32 * i, col + lane + 32 * i);
+        if (lane == 0) {
+          cp_async4(dst + 128, args.sw + static_cast<int64_t>(p.d.w_row0 >> 7) * KB + p.kb);
+          if (p.d.w_row1 >= 0) cp_async4(dst + 129, args.sw + static_cast<int64_t>(p.d.w_row1 >> 7) * KB + p.kb);
+        }
+      };
+      Pos p;  // the next K block to load
       seek(p, blockIdx.x);
-      Sf v0{}, v1{}, v2{};
-      bool h0 = p.t < ntiles;
-      if (h0) {
-        load(p, v0);
-        advance(p);
+      int loaded = 0;
+      for (int j = 0; j < X_SR - 1; ++j) {
+        if (p.t < ntiles) {
+          issue(p, j);
+          advance(p);
+          ++loaded;
+        }
+        cp_async_commit();  // one group per K block (empty past the end)
       }
-      bool h1 = h0 && p.t < ntiles;
-      if (h1) {
-        load(p, v1);
-        advance(p);
-      }
-      bool h2 = h1 && p.t < ntiles;
-      if (h2) load(p, v2);
-      uint32_t it = 0;
-      while (h0) {
+      for (int it = 0; it < loaded; ++it) {
         if (*abortp) break;
+        if (p.t < ntiles) {
+          issue(p, (it + X_SR - 1) % X_SR);  // the slot K block it - 1 has left
+          advance(p);
+          ++loaded;
+        }
+        cp_async_commit();
+        cp_async_wait<X_SR - 1>();  // K block it's group has landed (this lane's part) ...
+        __syncwarp();               // ... and every lane's
         const int s = it % X_STAGES;
         if (!mbar_wait(&bars->empty[s], ((it / X_STAGES) & 1) ^ 1, ctl)) break;
+        const float *v = sring + (it % X_SR) * X_SRING;
         uint8_t *sf = stages + s * X_STAGE + X_SF;
         reinterpret_cast<uint4 *>(sf)[lane] =
-            make_uint4(sf_word(v0.a[0]), sf_word(v0.a[1]), sf_word(v0.a[2]), sf_word(v0.a[3]));
-        const uint32_t wa = sf_word(v0.wa), wb = sf_word(v0.wb);
+            make_uint4(sf_word(v[lane]), sf_word(v[lane + 32]), sf_word(v[lane + 64]), sf_word(v[lane + 96]));
+        const uint32_t wa = sf_word(v[128]), wb = sf_word(v[129]);
         reinterpret_cast<uint4 *>(sf + 512)[lane] = make_uint4(wa, wa, wa, wa);
         reinterpret_cast<uint4 *>(sf + 1024)[lane] = make_uint4(wb, wb, wb, wb);
         fence_proxy_async_smem();  // generic writes -> the tensor core's copy
-        __syncwarp();
+        __syncwarp();              // (also: every lane has read slot it before it is refilled)
         if (lane == 0) mbar_arrive(&bars->full[s]);
-        ++it;
-        // slide the window: the K block after next starts loading now
-        v0 = v1;
-        h0 = h1;
-        v1 = v2;
-        h1 = h2;
-        if (h2) {
-          advance(p);
-          h2 = p.t < ntiles;
-          if (h2) load(p, v2);
-        }
       }
+      cp_async_wait<0>();  // nothing may land in shared memory after the CTA ends
     }
   } else {
     setmaxnreg_inc<224>();
