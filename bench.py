@@ -37,8 +37,13 @@ METRIC = "MoE-layer tokens/s and grouped FP8 GEMM TFLOP/s (% of B200 FP8 / HBM r
 KERNELS_PER_STEP = 11  # quantize, router GEMM, top-k, histogram, chunk table, ranks, row copy, 2 GEMMs, combine,
 #                        bias update
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-GEMM_SOURCES = [os.path.join(ROOT, "sparse_moe_layer_expert_b200", "csrc", f)
-                for f in ("gemm.cu", "gemm_mx.cu", "gemm_tiles.cuh", "common.cuh")]
+# sources each GEMM kernel is built from (the traffic figures in profiles/
+# hold only while these are unchanged)
+_CSRC = os.path.join(ROOT, "sparse_moe_layer_expert_b200", "csrc")
+GEMM_SOURCES = {
+    "gemm_fp8_kernel": [os.path.join(_CSRC, f) for f in ("gemm.cu", "gemm_tiles.cuh", "common.cuh")],
+    "gemm_mx_kernel": [os.path.join(_CSRC, f) for f in ("gemm_mx.cu", "gemm_tiles.cuh", "common.cuh")],
+}
 
 
 def parse(argv=None):
@@ -135,9 +140,10 @@ def measured_peaks() -> dict:
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
 
 
-def gemm_source_sha() -> str:
+def gemm_source_sha(kernel: str) -> str:
+    """Hash of the sources of a GEMM kernel ("gemm_fp8_kernel<0>" or its base name)."""
     h = hashlib.sha256()
-    for f in GEMM_SOURCES:
+    for f in GEMM_SOURCES[kernel.split("<")[0]]:
         h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
 
@@ -149,7 +155,7 @@ def profiled_traffic(workload: str, kernel: str):
         return None
     d = json.load(open(TRAFFIC_FILE))
     ent = d.get(f"{kernel}:{workload}")
-    if not ent or ent.get("src_sha") != gemm_source_sha():
+    if not ent or ent.get("src_sha") != gemm_source_sha(kernel):
         return None
     return float(ent["bytes_per_launch"])
 
