@@ -23,7 +23,8 @@
 //   * TMEM holds two partial buffers (2 x 256 columns), so the tensor core
 //     fills one while the promotion threads drain the other.
 //
-// Epilogues (after the last K block of a tile), one row per thread:
+// Epilogues (after the last K block of a tile, one row per thread; shared
+// with the block-scaled kernel in gemm_tiles.cuh):
 //   EPI_SWIGLU_Q  block A = gate, block B = up: h = silu(G) * U in FP32, then
 //                 the 1x128 requantization of h over the tile's 128 channels
 //                 (amax of the row's two 64-channel halves exchanged between
