@@ -1,7 +1,8 @@
 """Benchmark of the FP8 DeepSeekMoE layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed]
-                    [--impl ours|reference] [--no-cpu-baseline]
+                    [--scale-mode amax|pow2] [--balance-steps S] [--impl ours|reference]
+                    [--no-cpu-baseline] [--no-e2e]
 
 One step = the whole path over T tokens of seeded synthetic input with V3
 shapes (hidden 7168, intermediate 2048, 256 routed + 1 shared experts,
@@ -9,13 +10,16 @@ top-8), weights resident in HBM: the layer forward (quantize, route, group,
 gate/up GEMM + SwiGLU + requantize, down GEMM, combine) and the step's bias
 update.  The update goes to a working copy of the bias, so every step routes
 the batch alike; the line also reports the batch's expert load imbalance
-(max / mean) and the imbalance after one bias update applied for real.  With N > 1 (launched by torchrun)
-every rank runs its own replica of the layer on its own batch: there is no
-data-path collective; timing is the max over ranks.  Rank 0 prints one JSON
-line.
+(max / mean) and the imbalance after one bias update applied for real, and
+with --balance-steps S the imbalance along S steps with the update fed back.
+With N > 1 (launched by torchrun) every rank runs its own replica of the
+layer on its own batch: there is no data-path collective; timing is the max
+over ranks.  Rank 0 prints one JSON line.
 
-`--impl reference` times the CPU oracle (the slow double-precision reference
-of the same layer) on the host cores, on a bounded sample of the workload.
+--scale-mode pow2 runs the power-of-two scale variant (scales applied by the
+tensor core); the default is the pages' S = amax/448.  `--impl reference`
+times the CPU oracle (the slow double-precision reference of the same layer)
+on the host cores, on a bounded sample of the workload.
 """
 from __future__ import annotations
 
@@ -57,6 +61,9 @@ def parse(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=8)
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--balance-steps", type=int, default=0,
+                   help="after timing, run this many steps with the bias update fed back (the auxiliary-loss-free "
+                        "balancing loop) and report max/mean expert load along the way")
     p.add_argument("--scale-mode", choices=("amax", "pow2"), default="amax",
                    help="amax: S = amax/448 (the pages, default); pow2: power-of-two scales applied by the "
                         "tensor core (block-scaled MMA)")
@@ -408,6 +415,22 @@ def main(argv=None):
                    d2h_bytes_per_step=out_h.numel() * out_h.element_size(), ms_per_step=round(e2e_ms, 4))
         layer.check(stream)
 
+    # ------------------------------------------------ balancing loop (untimed)
+    balance = None
+    if args.balance_steps > 0:
+        b_keep = layer.bias.clone()
+        marks = sorted({0, 1, 2, 5, 10, 20, 50, 100, 200, 500, 1000, args.balance_steps} & set(range(args.balance_steps + 1)))
+        traj = {}
+        for k in range(args.balance_steps + 1):
+            layer.forward(x, out=out, counts_out=counts, stream=stream)
+            if k in marks:
+                traj[k] = round(float(counts.max().item()) / mean_load, 3)
+            if k < args.balance_steps:
+                M.moe_bias_update(layer.bias, counts, cfg["Nr"], total_assign, 0.001, stream=stream)
+        layer.bias.copy_(b_keep)
+        layer.check(stream)
+        balance = dict(gamma=0.001, steps=args.balance_steps, max_over_mean={str(k): v for k, v in traj.items()})
+
     # ------------------------------------------------ CPU oracle baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -440,6 +463,7 @@ def main(argv=None):
         layer_weight_gb=round(alg["layer_weight_bytes"] / 1e9, 3),
         experts_touched=touched + cfg.get("Ns", 1),
         load=load,
+        **({"balance": balance} if balance else {}),
         stage_ms={k: round(v, 4) for k, v in stage_ms.items()},
         step_ms_min=round(min(step_ms), 4),
         cpu_baseline=cpu,
