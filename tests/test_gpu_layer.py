@@ -163,7 +163,14 @@ def check_requantized(oracle_lib, hq, hs, hq_o, hs_o, h_o, mode=0):
         mid = (a + b) / 2
         # adjacent codes (same sign) and the quotient within 1e-4 of their midpoint
         assert np.all(np.sign(a) * np.sign(b) >= 0)
-        assert np.all(np.abs(quot - mid) <= 1e-4 * np.maximum(np.abs(mid), 2.0 ** -9)), "code differs off a tie"
+        rel = np.abs(quot - mid) / np.maximum(np.abs(mid), 2.0 ** -9)
+        print(f"re-quantized codes differing: {int(diff.sum())} of {diff.size}; distance of the oracle quotient "
+              f"from the midpoint (relative): max {rel.max():.2e}")
+        # the band is the rounding of h on the two sides: 1e-4 when each
+        # 128-long partial is formed exactly and added in FP32 (scale mode 0);
+        # 1e-3 when the tensor core adds the whole K range in FP32 (mode 1)
+        band = 1e-3 if mode == 1 else 1e-4
+        assert np.all(rel <= band), "code differs off a tie"
         vals = np.unique(dq[np.isfinite(dq)])
         assert np.all(np.abs(np.searchsorted(vals, a) - np.searchsorted(vals, b)) == 1), "non-adjacent codes"
 

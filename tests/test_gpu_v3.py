@@ -116,3 +116,31 @@ def test_v3_prefill_layer_pow2(m, oracle_lib, v3_layer_pow2):
     rng = np.random.default_rng(14)
     toks = np.sort(rng.choice(4096, 4, replace=False))
     check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=True)
+
+
+def test_v3_decode_layer_pow2(m, oracle_lib, v3_layer_pow2):
+    layer, _ = v3_layer_pow2
+    prob = _problem(dict(S.DECODE, scale_mode=1), 64, 11, layer, "zero")
+    r = check_layer(m, oracle_lib, prob, layer, tokens=np.array([0, 9, 31, 63]), check_weights=False)
+    assert r["counts"].sum() == 64 * 8
+
+
+def test_v3_skewed_layer_pow2(m, oracle_lib, v3_layer_pow2):
+    """The skewed configuration at full size in the power-of-two scale mode
+    (the block-scaled GEMMs on hot experts with thousands of rows)."""
+    base, _ = v3_layer_pow2
+    cfg = dict(S.SKEWED, scale_mode=1)
+    shape = {k: cfg[k] for k in ("H", "I", "Nr", "Kr", "Ns", "n_groups", "topk_groups", "scale_mode")}
+    layer = m.MoeLayer(shape)
+    layer.w13, layer.s13, layer.w2, layer.s2 = base.w13, base.s13, base.w2, base.s2  # same weights, no copy
+    T = cfg["T"]
+    prob = Problem(cfg, T, seed=15, device="cuda")
+    prob.seed = 0
+    prob.wr = base.wr
+    prob.bias = torch.zeros(cfg["Nr"], dtype=torch.float32, device="cuda")
+    layer.set_router(prob.wr, prob.bias)
+    rng = np.random.default_rng(15)
+    toks = np.sort(rng.choice(T, 4, replace=False))
+    r = check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=False)
+    c = r["counts"]
+    assert c.max() >= 4 * c.mean()
