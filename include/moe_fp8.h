@@ -83,8 +83,9 @@ MOE_API int moe_abi_version(void);
 
 /* ----------------------------------------------------------- layer shape */
 /* Shape of one DeepSeekMoE layer ([P4] Methode 2; [P3]).
- *   hidden      H, multiple of 128 (7168 in DeepSeek-V3)
- *   inter       I, expert SwiGLU intermediate size, multiple of 128 (2048)
+ *   hidden      H, multiple of 128, at most 32768 (7168 in DeepSeek-V3)
+ *   inter       I, expert SwiGLU intermediate size, multiple of 128, at
+ *               most 32768 (2048)
  *   n_routed    N_r routed experts, 1..256 (256)
  *   top_k       K_r experts per token, 1..min(N_r, 16) (8)
  *   n_shared    N_s always-active experts, 0 or 1 (1)
@@ -121,7 +122,8 @@ typedef struct {
  *   w2_dev    E4M3 [E, H, I] down projection (K = I contiguous)
  *   s2_dev    float [E, H/128, I/128]
  *   wr_dev    bf16 [N_r, H] router centroids e_i
- * Every pointer must be 16-byte aligned. */
+ * The E4M3 and bf16 pointers must be 16-byte aligned, the scale pointers
+ * 4-byte aligned. */
 typedef struct {
     const uint8_t *w13_dev;
     const float *s13_dev;
@@ -170,7 +172,9 @@ MOE_API int fp8_quant_128x128_pow2(const void *w_dev, int64_t n, int64_t k, uint
  *   B_dev   E4M3 [N, K] K-contiguous (the weight, "Linear" layout);
  *   sB_dev  float [N/128, K/128]
  *   C_dev   bf16 [M, N] (RNE of the FP32 accumulator)
- * M >= 1, N % 128 == 0, K % 128 == 0; all pointers 16-byte aligned. */
+ * M >= 0 (0 enqueues nothing), N % 128 == 0, K % 128 == 0, K <= 32768;
+ * A_dev, B_dev, C_dev 16-byte aligned, sA_dev, sB_dev, err_flag_dev 4-byte
+ * aligned. */
 MOE_API int fp8_blockscaled_gemm(const uint8_t *A_dev, const float *sA_dev, const uint8_t *B_dev,
                          const float *sB_dev, void *C_dev, int64_t M, int64_t N, int64_t K,
                          int32_t *err_flag_dev, void *stream);

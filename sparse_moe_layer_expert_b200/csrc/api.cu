@@ -70,6 +70,11 @@ namespace {
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Longest contraction the GEMM kernels take: each tile keeps the scales of up
+// to 256 K blocks of 128.
+constexpr int64_t kMaxK = 256 * 128;
 
 int check_device() {
   int sms = 0, major = 0;
@@ -82,7 +87,7 @@ int check_cfg(const moe_config *c) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (c->hidden <= 0 || c->inter <= 0 || c->n_routed <= 0 || c->top_k <= 0) return MOE_ERR_INVALID_ARG;
   if (c->hidden % 128 || c->inter % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (c->hidden > 65536 || c->inter > 65536) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (c->hidden > kMaxK || c->inter > kMaxK) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (c->n_routed > 256 || c->top_k > 16 || c->top_k > c->n_routed) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (c->n_shared < 0 || c->n_shared > 1) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (c->n_groups < 0) return MOE_ERR_INVALID_ARG;
@@ -221,9 +226,10 @@ int fp8_blockscaled_gemm(const uint8_t *A, const float *sA, const uint8_t *B, co
   if (M < 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
   if (N % 128 || K % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return MOE_OK;
-  if (M > INT32_MAX - 256 || N > INT32_MAX - 256) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (M > INT32_MAX - 256 || N > INT32_MAX - 256 || K > kMaxK) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!A || !sA || !B || !sB || !C || !err_flag) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C) || !aligned4(sA) || !aligned4(sB) || !aligned4(err_flag))
+    return MOE_ERR_INVALID_ARG;
   if (const int d = check_device()) return d;
   moe::GemmLaunch g{};
   g.w = B;
@@ -272,6 +278,8 @@ int moe_route(const moe_config *cfg, const void *x, const void *wr, const float 
   }
   if (!x || !wr || !bias || !idx || !gate || !ws || !err_flag) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(wr) || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_INVALID_ARG;
+  if (!aligned4(bias) || !aligned4(idx) || !aligned4(gate) || !aligned4(counts) || !aligned4(err_flag))
+    return MOE_ERR_INVALID_ARG;
   if (ws_bytes < moe_route_workspace_size(cfg, T)) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (const int d = check_device()) return d;
   float *partial = static_cast<float *>(ws);
@@ -298,6 +306,8 @@ int moe_route_noalloc(const moe_config *cfg, const void *x, const void *wr, cons
   }
   if (!x || !wr || !bias || !idx || !gate || !err_flag) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(wr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned4(bias) || !aligned4(idx) || !aligned4(gate) || !aligned4(counts) || !aligned4(err_flag))
+    return MOE_ERR_INVALID_ARG;
   const int ks = moe::router_ksplit(T, cfg->n_routed, cfg->hidden);
   if (static_cast<size_t>(ks) * static_cast<size_t>(T) * cfg->n_routed > moe::kRouteNoAllocScratchFloats)
     return MOE_ERR_WORKSPACE_TOO_SMALL;
@@ -346,6 +356,9 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
   if (!w->w13_dev || !w->s13_dev || !w->w2_dev || !w->s2_dev || !w->wr_dev) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(out) || !aligned16(w->w13_dev) || !aligned16(w->w2_dev) || !aligned16(w->wr_dev) ||
       (reinterpret_cast<uintptr_t>(ws) & 255))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned4(w->s13_dev) || !aligned4(w->s2_dev) || !aligned4(bias) || !aligned4(err_flag) ||
+      !aligned4(idx_out) || !aligned4(counts_out))
     return MOE_ERR_INVALID_ARG;
   moe_ws_layout L;
   make_layout(cfg, T, &L);
@@ -484,7 +497,8 @@ int moe_profile_events(void *const *events, int32_t n_events) {
 
 int moe_bias_update(float *bias, const int32_t *counts, int32_t n_routed, int64_t total, float gamma,
                     void *stream) {
-  if (!bias || !counts || n_routed <= 0 || total < 0) return MOE_ERR_INVALID_ARG;
+  if (!bias || !counts || n_routed <= 0 || total < 0 || !aligned4(bias) || !aligned4(counts))
+    return MOE_ERR_INVALID_ARG;
   if (const int d = check_device()) return d;
   return cuda_status(moe::launch_bias_update(bias, counts, n_routed, total, gamma, static_cast<cudaStream_t>(stream)));
 }

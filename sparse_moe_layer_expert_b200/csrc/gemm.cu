@@ -345,13 +345,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 template <int EPI>
 static cudaError_t launch_epi(const CUtensorMap &mw, const CUtensorMap &m0, const CUtensorMap &m1,
                               const GemmArgs &a, int grid, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(gemm_fp8_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (const cudaError_t e = smem_attr_once(gemm_fp8_kernel<EPI>, G_SMEM, attr_done)) return e;
   gemm_fp8_kernel<EPI><<<grid, G_THREADS, G_SMEM, st>>>(mw, m0, m1, a);
   return cudaGetLastError();
 }

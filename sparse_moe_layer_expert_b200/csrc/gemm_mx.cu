@@ -367,13 +367,8 @@ __global__ void __launch_bounds__(X_THREADS, 1)
 template <int EPI>
 static cudaError_t launch_mx(const CUtensorMap &mw, const CUtensorMap &m0, const CUtensorMap &m1,
                              const GemmArgs &a, int grid, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(gemm_mx_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, X_SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (const cudaError_t e = smem_attr_once(gemm_mx_kernel<EPI>, X_SMEM, attr_done)) return e;
   gemm_mx_kernel<EPI><<<grid, X_THREADS, X_SMEM, st>>>(mw, m0, m1, a);
   return cudaGetLastError();
 }

@@ -5,7 +5,25 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace moe {
+
+// Raise a kernel's dynamic shared-memory limit once per device: the attribute
+// belongs to the current device's context, so a process that drives several
+// GPUs sets it on each.  `done` keeps one bit per device ordinal (< 64;
+// higher ordinals set it on every call).
+template <typename Fn>
+inline cudaError_t smem_attr_once(Fn *fn, int bytes, std::atomic<uint64_t> &done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // One unit of work of the grouped block-scaled GEMM, decoded on the device
 // from a chunk (<= 128 activation rows of one expert) and a weight-block pair.

@@ -358,12 +358,8 @@ cudaError_t launch_router_logits(const void *x, const void *wr, int64_t T, int N
   a.partial = partial;
   a.err = err;
   a.limit_ns = limit_ns;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, R_SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (const cudaError_t e = smem_attr_once(router_logits_kernel, R_SMEM, attr_done)) return e;
   const int tiles = a.n_eb * a.n_tb * a.n_ks;
   const int grid = tiles < moe_host::sm_count() ? tiles : moe_host::sm_count();
   router_logits_kernel<<<grid, R_THREADS, R_SMEM, st>>>(mw, mx, a);

@@ -60,6 +60,35 @@ def test_host_validation_without_device(m):
     assert L.fp8_quant_1x128(16, 4, 128, 128, 16, 16, None) == m.MOE_ERR_NO_DEVICE
 
 
+def test_contraction_and_alignment_limits_without_device(m):
+    import ctypes as C
+    L = m.lib
+    # the GEMM kernels keep the scales of at most 256 K blocks per tile
+    for H, I in [(32768, 2048), (7168, 32768)]:
+        assert m.moe_workspace_size(m.config(H, I, 16, 4), 8) > 0
+    for H, I in [(32768 + 128, 2048), (7168, 32768 + 128), (65536, 2048)]:
+        assert m.moe_workspace_size(m.config(H, I, 16, 4), 8) == 0
+    assert L.fp8_blockscaled_gemm(16, 16, 16, 16, 16, 4, 128, 32768 + 128, 16, None) == m.MOE_ERR_UNSUPPORTED_SHAPE
+    # operands 16-byte aligned, scales and the error word 4-byte aligned
+    assert L.fp8_blockscaled_gemm(16, 18, 16, 16, 16, 4, 128, 128, 16, None) == m.MOE_ERR_INVALID_ARG
+    assert L.fp8_blockscaled_gemm(16, 16, 16, 17, 16, 4, 128, 128, 16, None) == m.MOE_ERR_INVALID_ARG
+    assert L.fp8_blockscaled_gemm(16, 16, 16, 16, 16, 4, 128, 128, 18, None) == m.MOE_ERR_INVALID_ARG
+    assert L.fp8_blockscaled_gemm(24, 16, 16, 16, 16, 4, 128, 128, 16, None) == m.MOE_ERR_INVALID_ARG
+    assert L.fp8_blockscaled_gemm(16, 20, 16, 20, 16, 4, 128, 128, 20, None) == m.MOE_ERR_NO_DEVICE
+    assert L.fp8_blockscaled_gemm(16, 16, 16, 16, 16, 4, 128, 32768, 16, None) == m.MOE_ERR_NO_DEVICE
+    assert L.moe_bias_update(18, 16, 16, 64, C.c_float(0.001), None) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_bias_update(16, 16, 16, 64, C.c_float(0.001), None) == m.MOE_ERR_NO_DEVICE
+    # moe_forward: misaligned weight scales are rejected before the device check
+    cfg = m.config(512, 256, 16, 4)
+    for s13, s2, bias in [(18, 16, 16), (16, 18, 16), (16, 16, 18)]:
+        w = m._binding.MoeWeights(16, s13, 16, s2, 16)
+        assert L.moe_forward(C.byref(cfg), C.byref(w), bias, 16, 64, 16, 0, None, None, 256, 1 << 40, 16, None) \
+            == m.MOE_ERR_INVALID_ARG
+    w = m._binding.MoeWeights(16, 16, 16, 16, 16)
+    assert L.moe_forward(C.byref(cfg), C.byref(w), 16, 16, 64, 16, 0, None, None, 256, 1 << 40, 16, None) \
+        == m.MOE_ERR_NO_DEVICE
+
+
 def test_workspace_layout_is_disjoint_and_aligned(m):
     for (H, I, Nr, Kr, T) in [(512, 256, 16, 4, 256), (7168, 2048, 256, 8, 64), (7168, 2048, 256, 8, 4096),
                               (7168, 2048, 256, 8, 16384), (512, 256, 16, 4, 1)]:
