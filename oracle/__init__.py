@@ -3,7 +3,8 @@
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  It wraps ``moe_oracle.c`` (plain C,
 double precision, built with gcc) through ctypes and adds the integer-only
-steps (histogram, expert-contiguous order) in numpy.  It shares no code with
+steps (histogram, expert-contiguous order) and the sequence-wise balance loss
+(a metric of the routing) in numpy.  It shares no code with
 the CUDA library and never calls it.
 
 Sources are cited in ``moe_oracle.c`` (page title and section); the short
@@ -207,6 +208,39 @@ def expert_order(idx: np.ndarray, Nr: int):
     offsets = np.zeros(Nr + 1, np.int64)
     offsets[1:] = np.cumsum(counts)
     return offsets, order.astype(np.int64)
+
+
+def seq_balance_loss(s, idx, Nr: int, Kr: int, seq_len: int, alpha: float = 1e-4) -> np.ndarray:
+    """Sequence-wise balance loss of each run of ``seq_len`` consecutive tokens.
+
+    "DeepSeek-V3 Technischer Bericht", Methode section 2, names a small
+    complementary sequence-wise balance loss with alpha = 0.0001 but prints no
+    formula.  This follows the form the DeepSeek-V3 technical report gives it,
+    for one sequence of L tokens:
+        f_i  = N_r / (K_r L) * (number of tokens of the sequence that select expert i)
+        P_i  = (1 / L) * sum_t s_{i,t} / sum_j s_{j,t}
+        loss = alpha * sum_i f_i P_i
+    where s_{i,t} are the sigmoid affinities of all N_r routed experts and the
+    selection is the routing decision.  s: [T, Nr] doubles, idx: [T, Kr]
+    expert ids; T must be a multiple of seq_len.  Returns one loss per
+    sequence, in double precision.
+    """
+    s = np.asarray(s, np.float64)
+    idx = np.asarray(idx)
+    T = s.shape[0]
+    assert s.shape == (T, Nr) and idx.shape == (T, Kr) and seq_len >= 1 and T % seq_len == 0
+    L = seq_len
+    out = np.empty(T // L, np.float64)
+    for q in range(T // L):
+        seq_s = s[q * L:(q + 1) * L]
+        picks = np.zeros(Nr, np.float64)
+        for row in idx[q * L:(q + 1) * L]:
+            for e in row:
+                picks[int(e)] += 1.0
+        f = Nr / (Kr * L) * picks
+        P = (seq_s / seq_s.sum(axis=1, keepdims=True)).sum(axis=0) / L
+        out[q] = alpha * float(np.dot(f, P))
+    return out
 
 
 # ------------------------------------------------------------ expert FFN
