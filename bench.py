@@ -10,8 +10,10 @@ top-8), weights resident in HBM: the layer forward (quantize, route, group,
 gate/up GEMM + SwiGLU + requantize, down GEMM, combine) and the step's bias
 update.  The update goes to a working copy of the bias, so every step routes
 the batch alike; the line also reports the batch's expert load imbalance
-(max / mean) and the imbalance after one bias update applied for real, and
-with --balance-steps S the imbalance along S steps with the update fed back.
+(max / mean), the imbalance after one bias update applied for real and the
+sequence-wise balance loss (alpha = 1e-4, sequences of gcd(T, 4096) tokens;
+untimed), and with --balance-steps S the imbalance along S steps with the
+update fed back.
 With N > 1 (launched by torchrun) every rank runs its own replica of the
 layer on its own batch: there is no data-path collective; timing is the max
 over ranks.  Rank 0 prints one JSON line.
@@ -354,6 +356,10 @@ def main(argv=None):
 
     counts_h = counts.cpu()
     touched = int((counts_h > 0).sum())
+    # sequence-wise balance loss (alpha = 1e-4) of the batch the timed steps
+    # routed, read from the last forward's workspace before anything reroutes
+    seq_len = math.gcd(T, 4096)
+    seq_loss = layer.seq_balance_loss(T, seq_len, 1e-4, stream=stream).cpu().tolist()
     # expert load imbalance of the batch, and after one bias update applied
     # for real (the same batch routed again with b - gamma * sign(load - mean))
     mean_load = total_assign / cfg["Nr"]
@@ -364,7 +370,9 @@ def main(argv=None):
     layer.forward(x, out=out, counts_out=counts_upd, stream=stream)
     layer.bias = b_keep
     load = dict(max_over_mean=round(float(counts_h.max()) / mean_load, 3),
-                after_one_bias_update=round(float(counts_upd.max().item()) / mean_load, 3))
+                after_one_bias_update=round(float(counts_upd.max().item()) / mean_load, 3),
+                seq_balance_loss=dict(alpha=1e-4, seq_len=seq_len,
+                                      values=[float(f"{v:.6g}") for v in seq_loss[:8]]))
     alg = algorithmic_counts(cfg, T, touched)
     peaks = measured_peaks()
     g1_ms, g2_ms = stage_ms["gemm_gate_up"], stage_ms["gemm_down"]

@@ -295,6 +295,27 @@ MOE_API int moe_profile_events(void *const *events, int32_t n_events);
 MOE_API int moe_bias_update(float *bias_dev, const int32_t *counts_dev, int32_t n_routed,
                     int64_t total_assignments, float gamma, void *stream);
 
+/* Sequence-wise balance loss of the batch the last moe_forward routed ([P4]
+ * Methode 2 names this complementary loss and its weight alpha = 0.0001 but
+ * prints no formula; the form is the DeepSeek-V3 technical report's).  For
+ * each run of seq_len consecutive tokens (L = seq_len):
+ *   f_i  = N_r / (K_r L) * (tokens of the run that select expert i)
+ *   P_i  = (1/L) * sum_t s_{i,t} / sum_j s_{j,t}   (s: sigmoid affinities)
+ *   loss = alpha * sum_i f_i P_i                    (FP32)
+ * It reads the router's logit partials and routing decision that moe_forward
+ * leaves in its workspace, so call it on the same stream, after that
+ * moe_forward, with the same cfg, T and workspace.  A metric of the routing:
+ * nothing in the forward pass depends on it.
+ *   T            tokens of that forward; a multiple of seq_len (else
+ *                MOE_ERR_INVALID_ARG); T == 0 enqueues nothing
+ *   ws_dev       that forward's workspace (256-byte aligned, ws_bytes >=
+ *                moe_workspace_size(cfg, T))
+ *   loss_dev     float [T / seq_len], 4-byte aligned
+ *   err_flag_dev gets MOE_DEVERR_BAD_INDEX if a routed index is out of range */
+MOE_API int moe_seq_balance_loss(const moe_config *cfg, int64_t T, int64_t seq_len, float alpha,
+                                 const void *ws_dev, size_t ws_bytes, float *loss_dev, int32_t *err_flag_dev,
+                                 void *stream);
+
 /* ------------------------------------------------------------ errors */
 /* Synchronises `stream`, copies *err_flag_dev to *host_value (nullable) and
  * returns MOE_OK if it is 0, MOE_ERR_TIMEOUT if the timeout bit is set, else

@@ -12,7 +12,8 @@ from ._binding import (  # noqa: F401
     MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_WORKSPACE_TOO_SMALL, MOE_OK, MOE_SCALE_AMAX, MOE_SCALE_POW2, MoeConfig,
     MoeError, config, config_from,
     fp8_blockscaled_gemm, fp8_quant_128x128, fp8_quant_1x128, lib, moe_bias_update, moe_check_device_error,
-    moe_forward, moe_profile_events, moe_route, moe_route_noalloc, moe_route_workspace_size, moe_selftest_wait_timeout, moe_workspace_layout,
+    moe_forward, moe_profile_events, moe_route, moe_route_noalloc, moe_route_workspace_size, moe_selftest_wait_timeout,
+    moe_seq_balance_loss, moe_workspace_layout,
     moe_workspace_size, new_err_flag, weights_struct, ws_view,
 )
 from .layer import MoeLayer  # noqa: F401

@@ -42,7 +42,7 @@ EXPORTS = (
     "fp8_quant_128x128_pow2", "fp8_blockscaled_gemm",
     "moe_route_workspace_size", "moe_route", "moe_workspace_size", "moe_forward", "moe_workspace_layout",
     "moe_bias_update", "moe_check_device_error", "moe_selftest_wait_timeout", "moe_profile_events",
-    "moe_route_noalloc",
+    "moe_route_noalloc", "moe_seq_balance_loss",
 )
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 16 << 20
 MOE_PROFILE_EVENTS = 7
@@ -87,6 +87,7 @@ lib.moe_workspace_size.argtypes = [_cfgp, _i64]
 lib.moe_forward.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _sz, _vp, _vp]
 lib.moe_workspace_layout.argtypes = [_cfgp, _i64, C.POINTER(MoeWsLayout)]
 lib.moe_bias_update.argtypes = [_vp, _vp, _i32, _i64, _f32, _vp]
+lib.moe_seq_balance_loss.argtypes = [_cfgp, _i64, _i64, _f32, _vp, _sz, _vp, _vp, _vp]
 lib.moe_check_device_error.argtypes = [_vp, C.POINTER(C.c_int32), _vp]
 lib.moe_selftest_wait_timeout.argtypes = [_vp, _i64, _vp]
 lib.moe_profile_events.argtypes = [C.POINTER(_vp), _i32]
@@ -226,6 +227,16 @@ def moe_forward(cfg: MoeConfig, w: dict, bias, x, out=None, out_dtype=MOE_DTYPE_
 def moe_bias_update(bias, counts, n_routed: int, total: int, gamma: float = 0.001, stream=None):
     _check(lib.moe_bias_update(_ptr(bias), _ptr(counts), n_routed, total, gamma, _stream(stream)), "moe_bias_update")
     return bias
+
+
+def moe_seq_balance_loss(cfg: MoeConfig, T: int, seq_len: int, ws, err, loss=None, alpha: float = 1e-4,
+                         stream=None):
+    """Sequence-wise balance loss of each run of seq_len tokens of the batch
+    the last moe_forward on `ws` routed (float32 [T // seq_len])."""
+    loss = torch.empty(max(T // max(seq_len, 1), 1), dtype=torch.float32, device=ws.device) if loss is None else loss
+    _check(lib.moe_seq_balance_loss(C.byref(cfg), T, seq_len, alpha, _ptr(ws), ws.numel(), _ptr(loss), _ptr(err),
+                                    _stream(stream)), "moe_seq_balance_loss")
+    return loss[:T // max(seq_len, 1)]
 
 
 def moe_check_device_error(err, stream=None) -> tuple[int, int]:

@@ -177,7 +177,7 @@ const char *moe_status_string(int s) {
   }
 }
 
-int moe_abi_version(void) { return 101; }
+int moe_abi_version(void) { return 102; }
 
 static int quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q, float *scales,
                        void *stream, bool pow2) {
@@ -479,6 +479,26 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
   if (e == cudaSuccess && idx_out)
     e = cudaMemcpyAsync(idx_out, idx, sizeof(int32_t) * T * Kr, cudaMemcpyDeviceToDevice, st);
   return cuda_status(e);
+}
+
+int moe_seq_balance_loss(const moe_config *cfg, int64_t T, int64_t seq_len, float alpha, const void *ws,
+                         size_t ws_bytes, float *loss, int32_t *err_flag, void *stream) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (T < 0 || T > kMaxTokens || seq_len < 1 || !(alpha == alpha)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (T % seq_len) return MOE_ERR_INVALID_ARG;
+  if (!ws || !loss || !err_flag || (reinterpret_cast<uintptr_t>(ws) & 255) || !aligned4(loss) ||
+      !aligned4(err_flag))
+    return MOE_ERR_INVALID_ARG;
+  moe_ws_layout L;
+  make_layout(cfg, T, &L);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (const int d = check_device()) return d;
+  void *w = const_cast<void *>(ws);
+  const int ks = moe::router_ksplit(T, cfg->n_routed, cfg->hidden);
+  return cuda_status(moe::launch_seq_balance(at<const float *>(w, L.logits), ks, T, cfg->n_routed,
+                                             at<const int32_t *>(w, L.idx), cfg->top_k, seq_len, alpha, loss,
+                                             err_flag, static_cast<cudaStream_t>(stream)));
 }
 
 int moe_profile_events(void *const *events, int32_t n_events) {

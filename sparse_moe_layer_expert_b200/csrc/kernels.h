@@ -94,6 +94,11 @@ cudaError_t launch_router_topk(const float *partial, int n_ks, int64_t T, int Nr
                                int topk_groups, float route_scale, const float *bias, int32_t *idx, float *gate,
                                int32_t *counts, cudaStream_t st);
 
+// Sequence-wise balance loss of each run of seq_len tokens (T % seq_len == 0)
+// from the router's logit partials and routing decision.
+cudaError_t launch_seq_balance(const float *partial, int n_ks, int64_t T, int Nr, const int32_t *idx, int Kr,
+                               int64_t seq_len, float alpha, float *loss, int32_t *err, cudaStream_t st);
+
 cudaError_t launch_hist(const int32_t *idx, int64_t T, int Kr, int Nr, int32_t *blk_hist, int32_t *err,
                         cudaStream_t st);
 cudaError_t launch_build_chunks(const int32_t *blk_hist, int64_t T, int Kr, int Nr, int Ns, int32_t *counts,

@@ -5,7 +5,7 @@
 // s_{i,t} + b_i is among the K_r largest of {s_{j,t} + b_j}; the gate of a
 // chosen expert is s_{i,t} normalised over the chosen set.
 //
-// Two kernels:
+// Three kernels:
 //  1. router_logits_kernel: z = x . e_i for all (token, expert) on the
 //     tensor cores (tcgen05 kind::f16, bf16 operands, FP32 accumulation in
 //     TMEM), split over K so that enough CTAs run; each split writes its own
@@ -13,6 +13,8 @@
 //  2. router_topk_kernel: one warp per token; each lane holds the experts
 //     lane, lane+32, ... in registers; sigmoid, bias, optional group
 //     pre-selection and K_r rounds of warp-wide argmax.
+//  3. seq_balance_kernel: the sequence-wise balance loss of a routed batch
+//     (a metric of the routing, outside the layer step).
 #include <mutex>
 
 #include "common.cuh"
@@ -177,6 +179,16 @@ __global__ void __launch_bounds__(R_THREADS, 1)
 namespace {
 constexpr int EPL = 8;  // experts per lane (N_r <= 256)
 
+// s_{e,t} from the router's logit partials: the K splits are added in split
+// order, then the sigmoid.  Every kernel that needs the affinities computes
+// them here, so they agree bit for bit.
+__device__ __forceinline__ float affinity(const float *__restrict__ partial, int n_ks, int64_t T, int Nr,
+                                          int64_t t, int e) {
+  float z = 0.0f;
+  for (int k = 0; k < n_ks; ++k) z += partial[(static_cast<int64_t>(k) * T + t) * Nr + e];
+  return 1.0f / (1.0f + expf(-z));
+}
+
 __device__ __forceinline__ void warp_argmax(float &v, int &i) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -207,9 +219,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float *__restric
     s[i] = 0.0f;
     c[i] = -INFINITY;
     if (ok[i]) {
-      float z = 0.0f;
-      for (int k = 0; k < n_ks; ++k) z += partial[(static_cast<int64_t>(k) * T + t) * Nr + e];
-      s[i] = 1.0f / (1.0f + expf(-z));
+      s[i] = affinity(partial, n_ks, T, Nr, t, e);
       c[i] = s[i] + bias[e];
     }
   }
@@ -295,6 +305,97 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float *__restric
     gate[t * Kr + lane] = route_scale * (sel_s / ssum);
     if (counts && sel_e >= 0 && sel_e < Nr) atomicAdd(&counts[sel_e], 1);
   }
+}
+
+// ------------------------------------------------ sequence-wise balance loss
+// One CTA per sequence of L tokens (the complementary loss of "DeepSeek-V3
+// Technischer Bericht", Methode section 2, in the technical report's form):
+//   loss = alpha * sum_i f_i P_i,  f_i = N_r / (K_r L) * picks_i,
+//   P_i = (1/L) sum_t s_{i,t} / sum_j s_{j,t}.
+// Warp w takes tokens w, w + BL_WARPS, ... of the sequence; lane l keeps, for
+// the experts l, l+32, ..., the running sums of the normalised affinities and
+// of the picks.  The warps' sums are then added in warp order and the
+// experts' terms in expert order, so the result does not depend on the
+// schedule.  Reads the partials once: HBM-bound, a metric outside the step.
+constexpr int BL_WARPS = 16;
+
+__global__ void __launch_bounds__(BL_WARPS * 32)
+    seq_balance_kernel(const float *__restrict__ partial, int n_ks, int64_t T, int Nr,
+                       const int32_t *__restrict__ idx, int Kr, int64_t seq_len, float alpha,
+                       float *__restrict__ loss, int32_t *err) {
+  __shared__ float p_sh[BL_WARPS][EPL * 32];
+  __shared__ int c_sh[BL_WARPS][EPL * 32];
+  __shared__ float term[EPL * 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * seq_len;
+  float acc[EPL];
+  int cnt[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    acc[i] = 0.0f;
+    cnt[i] = 0;
+  }
+  bool bad = false;
+  for (int64_t t = t0 + warp; t < t0 + seq_len; t += BL_WARPS) {
+    float s[EPL];
+    float sum = 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      s[i] = e < Nr ? affinity(partial, n_ks, T, Nr, t, e) : 0.0f;
+      sum += s[i];
+    }
+    // butterfly: every lane ends with the same total
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) acc[i] += s[i] / sum;
+    for (int k = 0; k < Kr; ++k) {
+      const int e = idx[t * Kr + k];
+      if (e < 0 || e >= Nr) {
+        bad = true;
+        continue;
+      }
+      if ((e & 31) == lane) {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) cnt[i] += (i == (e >> 5)) ? 1 : 0;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    p_sh[warp][lane + 32 * i] = acc[i];
+    c_sh[warp][lane + 32 * i] = cnt[i];
+  }
+  if (bad && lane == 0 && err) atomicOr(err, MOE_DEVERR_BAD_INDEX);
+  __syncthreads();
+  if (threadIdx.x < EPL * 32) {
+    const int e = threadIdx.x;
+    float p = 0.0f;
+    int c = 0;
+    for (int w = 0; w < BL_WARPS; ++w) {
+      p += p_sh[w][e];
+      c += c_sh[w][e];
+    }
+    term[e] = e < Nr ? static_cast<float>(c) * p : 0.0f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.0f;
+    for (int e = 0; e < Nr; ++e) tot += term[e];
+    const float L = static_cast<float>(seq_len);
+    // sum_i f_i P_i = N_r / (K_r L) * sum_i picks_i * (sum_t s'_{i,t}) / L
+    loss[blockIdx.x] = alpha * (static_cast<float>(Nr) / (static_cast<float>(Kr) * L)) * (tot / L);
+  }
+}
+
+cudaError_t launch_seq_balance(const float *partial, int n_ks, int64_t T, int Nr, const int32_t *idx, int Kr,
+                               int64_t seq_len, float alpha, float *loss, int32_t *err, cudaStream_t st) {
+  if (T == 0 || seq_len <= 0) return cudaSuccess;
+  const int64_t n_seq = T / seq_len;
+  seq_balance_kernel<<<static_cast<unsigned>(n_seq), BL_WARPS * 32, 0, st>>>(partial, n_ks, T, Nr, idx, Kr,
+                                                                             seq_len, alpha, loss, err);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------ fixed scratch (no allocation)

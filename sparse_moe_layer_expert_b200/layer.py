@@ -74,6 +74,11 @@ class MoeLayer:
     def bias_update(self, counts: torch.Tensor, T: int, gamma: float = 0.001, stream=None) -> None:
         B.moe_bias_update(self.bias, counts, self.cfg.n_routed, T * self.cfg.top_k, gamma, stream=stream)
 
+    def seq_balance_loss(self, T: int, seq_len: int, alpha: float = 1e-4, stream=None) -> torch.Tensor:
+        """Sequence-wise balance loss of the batch of T tokens this layer's
+        last forward of that size routed, one value per run of seq_len tokens."""
+        return B.moe_seq_balance_loss(self.cfg, T, seq_len, self.workspace(T), self.err, alpha=alpha, stream=stream)
+
     def check(self, stream=None) -> None:
         st, v = B.moe_check_device_error(self.err, stream)
         if st != B.MOE_OK:

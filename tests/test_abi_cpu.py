@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported(m):
 
 
 def test_status_strings_and_version(m):
-    assert m.lib.moe_abi_version() == 101
+    assert m.lib.moe_abi_version() == 102
     assert m.lib.moe_status_string(0) == b"ok"
     assert b"128" in m.lib.moe_status_string(m.MOE_ERR_UNSUPPORTED_SHAPE)
     assert m.lib.moe_status_string(12345) == b"unknown status"
@@ -108,3 +108,21 @@ def test_route_workspace_size(m):
     cfg = m.config(7168, 2048, 256, 8)
     assert m.moe_route_workspace_size(cfg, 4096) >= 4096 * 256 * 4
     assert m.moe_route_workspace_size(cfg, 0) >= 0
+
+
+def test_seq_balance_loss_validation_without_device(m):
+    import ctypes as C
+    L = m.lib
+    cfg = m.config(512, 256, 16, 4)
+    big = 1 << 40
+    a = C.c_float(1e-4)
+    assert L.moe_seq_balance_loss(C.byref(cfg), 0, 8, a, None, 0, None, None, None) == m.MOE_OK
+    assert L.moe_seq_balance_loss(C.byref(cfg), 96, 40, a, 256, big, 16, 16, None) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_seq_balance_loss(C.byref(cfg), 96, 0, a, 256, big, 16, 16, None) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_seq_balance_loss(C.byref(cfg), 96, 32, C.c_float(float("nan")), 256, big, 16, 16, None) == \
+        m.MOE_ERR_INVALID_ARG
+    assert L.moe_seq_balance_loss(C.byref(cfg), 96, 32, a, 128, big, 16, 16, None) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_seq_balance_loss(C.byref(cfg), 96, 32, a, 256, big, 18, 16, None) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_seq_balance_loss(C.byref(cfg), 96, 32, a, 256, 1024, 16, 16, None) == \
+        m.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert L.moe_seq_balance_loss(C.byref(cfg), 96, 32, a, 256, big, 16, 16, None) == m.MOE_ERR_NO_DEVICE

@@ -70,7 +70,7 @@ def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts
     assert np.array_equal(xq, xq_o) and np.array_equal(xs, xs_o)
     # S2: routing (oracle routes all tokens; cheap relative to the FFNs)
     ocf = oracle_cfg(oracle_lib, cfg)
-    oi, og, gap, _ = oracle_lib.route(ocf, prob.x, prob.wr, prob.bias)
+    oi, og, gap, s_o = oracle_lib.route(ocf, prob.x, prob.wr, prob.bias, want_s=True)
     bad, n_exempt = route_sets_match(idx, oi, gap)
     assert not bad, f"routing differs on {len(bad)} tokens"
     assert n_exempt <= max(1, T // 1000)
@@ -131,7 +131,32 @@ def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts
     o16 = out16.cpu()[torch.as_tensor(tok)]
     assert_close(bf16_to_f64(o16), res["out"], bf16_out=True, what="layer output (bf16)")
     assert torch.equal(o16, out32.cpu()[torch.as_tensor(tok)].to(torch.bfloat16))
-    return dict(counts=counts, idx=idx, n_exempt=n_exempt)
+    return dict(counts=counts, idx=idx, n_exempt=n_exempt, idx_ref=oi, s_ref=s_o)
+
+
+def check_balance_loss(oracle_lib, prob: Problem, layer, r: dict, seq_len: int, alpha: float = 1e-4):
+    """The sequence-wise balance loss of the batch the last forward routed
+    (run by check_layer) against the oracle's, from the oracle's own
+    affinities and selection.  Tolerance: each lane adds up to L/16
+    normalised affinities in FP32 (relative error <= L/16 * 2^-24, 1.6e-5 at
+    L = 4096) on affinities from FP32 logits; rtol 1e-4 covers both.  A
+    near-tie token may legitimately be routed to other experts than the
+    oracle's (its selection is exempt from bit-exactness): each expert
+    swapped that way moves sum_i f_i P_i by at most N_r / (K_r L) * max_i P_i,
+    which is added to the bound of its sequence."""
+    T, Nr, Kr = prob.T, prob.cfg["Nr"], prob.cfg["Kr"]
+    L = seq_len
+    got = layer.seq_balance_loss(T, L, alpha).cpu().numpy().astype(np.float64)
+    layer.check()
+    ref = oracle_lib.seq_balance_loss(r["s_ref"], r["idx_ref"], Nr, Kr, L, alpha)
+    swaps = np.array([len(set(a.tolist()) - set(b.tolist())) for a, b in zip(r["idx"], r["idx_ref"])])
+    s_norm = r["s_ref"] / r["s_ref"].sum(axis=1, keepdims=True)
+    p_max = s_norm.reshape(T // L, L, Nr).mean(axis=1).max(axis=1)
+    bound = alpha * Nr / (Kr * L) * swaps.reshape(T // L, L).sum(axis=1) * p_max
+    assert got.shape == ref.shape
+    err = np.abs(got - ref)
+    assert (err <= 1e-4 * np.abs(ref) + bound).all(), (got, ref, bound)
+    return got
 
 
 def check_requantized(oracle_lib, hq, hs, hq_o, hs_o, h_o, mode=0):
@@ -292,6 +317,46 @@ def test_bias_update_matches_oracle(m, oracle_lib):
     torch.cuda.synchronize()
     want = oracle_lib.bias_update(b0, counts.cpu().numpy(), 16, 256 * 4, 0.001)
     assert np.array_equal(layer.bias.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("T,seq_lens", [(512, (512, 128, 1)), (300, (300, 100, 3))])
+def test_seq_balance_loss_matches_oracle(m, oracle_lib, T, seq_lens):
+    prob = Problem(S.TINY, T, seed=31 + T)
+    layer = build_gpu_layer(m, prob)
+    r = check_layer(m, oracle_lib, prob, layer, tokens=np.arange(0, T, 37))
+    for L in seq_lens:
+        check_balance_loss(oracle_lib, prob, layer, r, L)
+
+
+def test_seq_balance_loss_skewed_and_collapsed_routing(m, oracle_lib):
+    # group-limited routing of the mixture input
+    prob = Problem(dict(S.TINY, n_groups=4, topk_groups=2), 512, seed=33, x_kind="mixture")
+    layer = build_gpu_layer(m, prob)
+    r = check_layer(m, oracle_lib, prob, layer, tokens=np.arange(0, 512, 61))
+    check_balance_loss(oracle_lib, prob, layer, r, 256)
+    # every token sent to experts 0..K_r-1: f_i = N_r / K_r there, so the
+    # loss is alpha * N_r / K_r * (their share of the affinity mass)
+    prob = Problem(S.TINY, 384, seed=34)
+    kr, nr = S.TINY["Kr"], S.TINY["Nr"]
+    prob.bias = prob.bias.clone()
+    prob.bias[:kr] += 1.0
+    layer = build_gpu_layer(m, prob)
+    r = check_layer(m, oracle_lib, prob, layer, tokens=np.arange(0, 384, 47))
+    got = check_balance_loss(oracle_lib, prob, layer, r, 384, alpha=1.0)
+    share = (r["s_ref"][:, :kr].sum(1) / r["s_ref"].sum(1)).mean()
+    assert got[0] == pytest.approx(nr / kr * share, rel=1e-4)
+
+
+def test_seq_balance_loss_rejects_ragged_sequences(m):
+    prob = Problem(S.TINY, 96, seed=35)
+    layer = build_gpu_layer(m, prob)
+    layer.forward(prob.x.cuda())
+    with pytest.raises(m.MoeError) as e:
+        layer.seq_balance_loss(96, 40)
+    assert e.value.status == m.MOE_ERR_INVALID_ARG
+    with pytest.raises(m.MoeError) as e:
+        m.moe_seq_balance_loss(layer.cfg, 96, 32, torch.empty(1024, dtype=torch.uint8, device="cuda"), layer.err)
+    assert e.value.status == m.MOE_ERR_WORKSPACE_TOO_SMALL
 
 
 def test_forward_rejects_small_workspace(m):

@@ -9,7 +9,7 @@ import torch
 
 import moe_synth as S
 from _moe_util import Problem
-from test_gpu_layer import check_layer
+from test_gpu_layer import check_balance_loss, check_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -66,6 +66,10 @@ def test_v3_prefill_layer(m, oracle_lib, v3_layer):
     r = check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=False)
     c = r["counts"]
     print(f"prefill load: max {c.max()} mean {c.mean():.1f} min {c.min()} empty {(c == 0).sum()}")
+    # the sequence-wise balance loss: one 4096-token sequence, and four of 1024
+    loss = check_balance_loss(oracle_lib, prob, layer, r, 4096)
+    check_balance_loss(oracle_lib, prob, layer, r, 1024)
+    print(f"prefill sequence-wise balance loss (alpha 1e-4): {loss[0]:.6e}")
 
 
 def test_v3_skewed_layer(m, oracle_lib, v3_layer):
@@ -90,6 +94,8 @@ def test_v3_skewed_layer(m, oracle_lib, v3_layer):
     c = r["counts"]
     print(f"skewed load: max {c.max()} mean {c.mean():.1f} max/mean {c.max() / c.mean():.2f}")
     assert c.max() >= 4 * c.mean()  # the configuration's imbalance (max/mean load >= 4)
+    loss = check_balance_loss(oracle_lib, prob, layer, r, 4096)
+    print(f"skewed sequence-wise balance loss (alpha 1e-4), four 4096-token sequences: {loss}")
 
 
 @pytest.fixture(scope="module")
