@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed]
                     [--scale-mode amax|pow2] [--balance-steps S] [--impl ours|reference]
-                    [--no-cpu-baseline] [--no-e2e]
+                    [--no-cpu-baseline] [--no-e2e] [--e2e-serial]
 
 One step = the whole path over T tokens of seeded synthetic input with V3
 shapes (hidden 7168, intermediate 2048, 256 routed + 1 shared experts,
@@ -17,6 +17,11 @@ update fed back.
 With N > 1 (launched by torchrun) every rank runs its own replica of the
 layer on its own batch: there is no data-path collective; timing is the max
 over ranks.  Rank 0 prints one JSON line.
+
+The end-to-end figure ("e2e") runs the same steps through host buffers:
+every step copies its input in from pinned host memory and reads its output
+back, on two copy streams that overlap the neighbouring steps' compute
+(--e2e-serial: copies in series on the launching stream).
 
 --scale-mode pow2 runs the power-of-two scale variant (scales applied by the
 tensor core); the default is the pages' S = amax/448.  `--impl reference`
@@ -63,6 +68,8 @@ def parse(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=8)
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--e2e-serial", action="store_true",
+                   help="end-to-end leg with its copies in series with the compute (default: pipelined)")
     p.add_argument("--balance-steps", type=int, default=0,
                    help="after timing, run this many steps with the bias update fed back (the auxiliary-loss-free "
                         "balancing loop) and report max/mean expert load along the way")
@@ -231,6 +238,80 @@ def _isnum(s):
         return False
 
 
+# ------------------------------------------------ end to end (host buffers)
+def e2e_serial(step_io, x_h, out_h, stream, dev, steps: int, world: int) -> float:
+    """Steps with their copies in series on the launching stream: each step
+    copies its input in from pinned host memory, runs, and reads its output
+    back.  Returns the device time of `steps` steps in ms (max over ranks)."""
+    import torch
+
+    T, H = x_h.shape
+    x_d = torch.empty((T, H), dtype=x_h.dtype, device=dev)
+    out_d = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            x_d.copy_(x_h, non_blocking=True)
+            step_io(x_d, out_d)
+            out_h.copy_(out_d, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+
+def e2e_pipelined(step_io, x_h, out_h, stream, dev, steps: int, world: int) -> float:
+    """Steps with their copies overlapped, as a serving loop runs them: step
+    k's input is copied in on one copy stream while step k-1 computes, and
+    step k's output is read back on another while step k+1 computes.  Two
+    device buffers each way; events order every reuse (step k waits for its
+    input copy and for the read-back of step k-2's output from the buffer it
+    writes; the input copy of step k waits until step k-2 has finished with
+    its buffer).  The timed region runs on the launching stream from before
+    the first input copy to after the last read-back.  out_h: two pinned
+    host buffers.  Returns the device time of `steps` steps in ms (max over
+    ranks)."""
+    import torch
+
+    T, H = x_h.shape
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    x_d = [torch.empty((T, H), dtype=x_h.dtype, device=dev) for _ in range(2)]
+    out_d = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    x_ready = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    read_back = [torch.cuda.Event() for _ in range(2)]
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    h2d.wait_event(e0)
+    d2h.wait_event(e0)
+    for k in range(steps):
+        b = k % 2
+        with torch.cuda.stream(h2d):
+            if k >= 2:
+                h2d.wait_event(computed[b])
+            x_d[b].copy_(x_h, non_blocking=True)
+            x_ready[b].record(h2d)
+        stream.wait_event(x_ready[b])
+        if k >= 2:
+            stream.wait_event(read_back[b])
+        with torch.cuda.stream(stream):
+            step_io(x_d[b], out_d[b])
+        computed[b].record(stream)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(computed[b])
+            out_h[b].copy_(out_d[b], non_blocking=True)
+            read_back[b].record(d2h)
+    stream.wait_stream(h2d)
+    stream.wait_stream(d2h)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+
 # ---------------------------------------------------------- oracle (CPU)
 def oracle_sample(cfg: dict, n_tok: int, seed: int, x_full, wr, bias, expert_bf16):
     """Prepare the oracle's inputs for the first n_tok tokens of the batch:
@@ -312,6 +393,10 @@ def main(argv=None):
 
     def step(x_in):
         layer.forward(x_in, out=out, counts_out=counts, stream=stream)
+        M.moe_bias_update(bias_next, counts, cfg["Nr"], total_assign, 0.001, stream=stream)
+
+    def step_io(x_in, out_buf):  # the same step, output to a given buffer (end-to-end legs)
+        layer.forward(x_in, out=out_buf, counts_out=counts, stream=stream)
         M.moe_bias_update(bias_next, counts, cfg["Nr"], total_assign, 0.001, stream=stream)
 
     torch.cuda.synchronize(dev)
@@ -402,25 +487,31 @@ def main(argv=None):
     e2e = None
     if not args.no_e2e:
         x_h = x.cpu().pin_memory()
-        out_h = torch.empty((T, cfg["H"]), dtype=torch.bfloat16).pin_memory()
-        for _ in range(max(1, args.warmup // 2)):
-            x_d = x_h.to(dev, non_blocking=True)
-            step(x_d)
-            out_h.copy_(out, non_blocking=True)
-        barrier(world, dev)
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            x_d = x_h.to(dev, non_blocking=True)
-            step(x_d)
-            out_h.copy_(out, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+        out_h = [torch.empty((T, cfg["H"]), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        mode, note = ("serial", "requested") if args.e2e_serial else ("pipelined", None)
+        e2e_ms = None
+        if mode == "pipelined":
+            try:
+                for _ in range(max(1, args.warmup // 2)):
+                    e2e_pipelined(step_io, x_h, out_h, stream, dev, 2, world)
+                e2e_ms = e2e_pipelined(step_io, x_h, out_h, stream, dev, args.steps, world) / args.steps
+                # every step still holds its whole computation: a shorter
+                # step than the device-only one means the loop is broken
+                if e2e_ms < 0.98 * ms_per_step:
+                    mode, note, e2e_ms = "serial", f"pipelined loop measured {e2e_ms:.3f} ms/step < device", None
+            except Exception as exc:  # measure serially instead; the line says why
+                torch.cuda.synchronize(dev)
+                mode, note, e2e_ms = "serial", f"pipelined loop failed: {str(exc).splitlines()[0][:120]}", None
+        if e2e_ms is None:
+            for _ in range(max(1, args.warmup // 2)):
+                e2e_serial(step_io, x_h, out_h[0], stream, dev, 1, world)
+            e2e_ms = e2e_serial(step_io, x_h, out_h[0], stream, dev, args.steps, world) / args.steps
         e2e = dict(value=round(world * T / (e2e_ms / 1e3), 1), unit="tokens/s",
                    h2d_bytes_per_step=x_h.numel() * x_h.element_size(),
-                   d2h_bytes_per_step=out_h.numel() * out_h.element_size(), ms_per_step=round(e2e_ms, 4))
+                   d2h_bytes_per_step=out_h[0].numel() * out_h[0].element_size(), ms_per_step=round(e2e_ms, 4),
+                   copies=mode)
+        if note:
+            e2e["note"] = note
         layer.check(stream)
 
     # ------------------------------------------------ balancing loop (untimed)
