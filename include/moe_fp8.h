@@ -280,7 +280,9 @@ MOE_API int moe_workspace_layout(const moe_config *cfg, int64_t T, moe_ws_layout
  * cudaEvent_t handles) on its stream at the stage boundaries below, so
  * per-stage device time can be read with cudaEventElapsedTime.  Pass NULL/0
  * to turn it off.  Events are recorded, never created or destroyed, by the
- * library; recording adds no kernel launches.
+ * library; recording adds no kernel launches.  The caller keeps the events
+ * alive while the hook is set (turn it off before destroying them: a
+ * destroyed event makes the next moe_forward return MOE_ERR_CUDA).
  *   0 start | 1 after quantize | 2 after routing | 3 after grouping (hist,
  *   work lists, row copies) | 4 after gate/up GEMM (+SwiGLU, requant) |
  *   5 after down GEMM | 6 after combine */
