@@ -19,7 +19,10 @@
  * Conventions for every entry point
  *  - Pointers named *_dev are device pointers (cudaMalloc'd or from a
  *    framework allocator) owned by the caller; the library keeps no reference
- *    after the call returns and allocates no device memory.
+ *    after the call returns (the one exception: the event handles given to
+ *    moe_profile_events, kept until the hook is turned off) and allocates no
+ *    device memory (moe_route_noalloc's fixed scratch is a static array of
+ *    the library image).
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
  *    enqueued asynchronously; no entry point synchronises the stream except
  *    moe_check_device_error.
