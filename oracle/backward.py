@@ -36,7 +36,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import (SCALE_AMAX, _u16, blockscaled_gemm, e4m3_decode_table, quant_1x128, quant_1x128_f32)
+from . import (SCALE_AMAX, _u16, blockscaled_gemm, e4m3_decode_table, quant_1x128, quant_1x128_f32, route)
 
 
 def _pad_rows(a: np.ndarray, mult: int = 128) -> np.ndarray:
@@ -90,10 +90,20 @@ def _f32(v: np.ndarray) -> np.ndarray:
     return np.asarray(v, np.float64).astype(np.float32).astype(np.float64)
 
 
+def _as_f32_values(a) -> np.ndarray:
+    """float32 values of a bf16 tensor, uint16 bf16 bit patterns or a float32
+    array (bf16 -> float32 is exact, so quantizing either gives the same codes)."""
+    if isinstance(a, np.ndarray) and a.dtype == np.float32:
+        return np.ascontiguousarray(a)
+    u = _u16(a).astype(np.uint32) << 16
+    return np.ascontiguousarray(u.view(np.float32))
+
+
 def expert_backward(x, dy, W13q, s13, W2q, s2, mode: int = SCALE_AMAX) -> dict:
     """Backward of one expert FFN under the FP8 recipe above.
 
-    x, dy: bf16 [rows, H] (torch bf16 tensors or uint16 bit patterns);
+    x: bf16 [rows, H] (torch bf16 tensor or uint16 bit patterns); dy: the
+    gradient of the expert's output [rows, H], bf16 as x or float32 values;
     W13q u8 [2I, H] (gate rows 0..I-1, up rows I..2I-1), s13 f32 [2I/128, H/128];
     W2q u8 [H, I], s2 f32 [H/128, I/128].
     Returns FP32-rounded values (as float64 arrays): dx [rows, H],
@@ -113,10 +123,11 @@ def expert_backward(x, dy, W13q, s13, W2q, s2, mode: int = SCALE_AMAX) -> dict:
     silu = G * sig
     h = _f32(silu * U)
     # dgrad of the down projection: dY 1x128 along H, W2^T as [I, H] blocks
-    dyq, dys = quant_1x128(dy, mode)
+    dy = _as_f32_values(dy)
+    dyq, dys = quant_1x128_f32(dy, mode)
     dh = _f32(blockscaled_gemm(dyq, dys, np.ascontiguousarray(W2q.T), np.ascontiguousarray(s2.T)))
     # wgrad of the down projection: dY and h as 128x1 tiles along tokens
-    dyq_c, dys_c = quant_128x1_bf16(dy, mode)
+    dyq_c, dys_c = quant_128x1_f32(dy, mode)
     hq_c, hs_c = quant_128x1_f32(h, mode)
     dW2 = _f32(rows_scaled_gemm(dyq_c.T, dys_c.T, hq_c.T, hs_c.T))
     # SwiGLU backward (double, rounded to FP32)
@@ -137,3 +148,43 @@ def expert_backward(x, dy, W13q, s13, W2q, s2, mode: int = SCALE_AMAX) -> dict:
     dW3 = rows_scaled_gemm(dUq_c.T, dUs_c.T, xq_c.T, xs_c.T)
     dW13 = _f32(np.concatenate([dW1, dW3], axis=0))
     return dict(dx=dx, dW13=dW13, dW2=dW2, dh=dh, dG=dG, dU=dU, G=G, U=U, h=h)
+
+
+def layer_backward(cf, x, Wr, bias, experts, dout, mode: int = SCALE_AMAX) -> dict:
+    """Backward of the layer's FFN part with the routing held fixed:
+        out_t = u_t + FFN_shared(u_t) + sum_k g_{t,k} FFN_{e_{t,k}}(u_t)
+    ("DeepSeek-V3 Technischer Bericht", Methode section 2, layer output
+    equation).  Given dout [T, H] (bf16), each routed expert e receives, for
+    every token t that selected it (slot k), dY = g_{t,k} * dout_t in FP32
+    (the gate rounded to FP32, one FP32 product), the shared expert dY = dout;
+    each runs expert_backward on its tokens in token order.
+        dx_t = dout_t + dx_shared,t + sum_k dx_{e_{t,k}},t    (double, then FP32)
+    The routing (and with it every gate) is the oracle's own; the gradient of
+    the gates themselves (router backward) is not part of this.
+    experts: list indexed by expert id (routed 0..N_r-1, shared N_r) of
+    (W13q, s13, W2q, s2) tuples, None for experts no token uses.
+    Returns dx [T, H], dW13 and dW2 dicts keyed by expert id (FP32 values as
+    double arrays), and the routing (idx, gate, gap)."""
+    idx, gate, gap, _ = route(cf, x, Wr, bias)
+    xu = _u16(x)
+    d = _as_f32_values(dout)
+    T = xu.shape[0]
+    Nr = cf.Nr
+    acc = d.astype(np.float64)
+    dW13, dW2 = {}, {}
+    for e in range(Nr):
+        toks, slots = np.nonzero(idx == e)
+        if toks.size == 0:
+            continue
+        order = np.argsort(toks, kind="stable")
+        toks, slots = toks[order], slots[order]
+        g32 = gate[toks, slots].astype(np.float32)
+        dy = (g32[:, None] * d[toks]).astype(np.float32)
+        r = expert_backward(xu[toks], dy, *experts[e], mode=mode)
+        acc[toks] += r["dx"]
+        dW13[e], dW2[e] = r["dW13"], r["dW2"]
+    if cf.Ns:
+        r = expert_backward(xu, d, *experts[Nr], mode=mode)
+        acc += r["dx"]
+        dW13[Nr], dW2[Nr] = r["dW13"], r["dW2"]
+    return dict(dx=_f32(acc), dW13=dW13, dW2=dW2, idx=idx, gate=gate, gap=gap)

@@ -182,3 +182,68 @@ def test_rows_scaled_gemm_matches_dense_dequantized(oracle_lib, bw):
     A = dec[qa] * np.repeat(sa.astype(np.float64), 128, axis=1)[:, :K]
     B = dec[qb] * np.repeat(sb.astype(np.float64), 128, axis=1)[:, :K]
     np.testing.assert_allclose(got, A @ B.T, rtol=1e-12, atol=1e-9)
+
+
+# ------------------------------------------------------------ layer level
+def _layer_problem(oracle_lib, T=96, seed=0, zero_weights=False):
+    cfg = dict(S.TINY)
+    H, I, Nr, Kr = cfg["H"], cfg["I"], cfg["Nr"], cfg["Kr"]
+    x = S.gen_x(T, H, seed)
+    wr = S.gen_router(Nr, H, seed)
+    bias = S.gen_bias(Nr, seed)
+    dout = S.normal_bf16((T, H), 1.0, seed + 77)
+    experts = []
+    for e in range(Nr + 1):
+        w13, w2 = S.gen_expert(e, H, I, seed)
+        if zero_weights:
+            w13, w2 = torch.zeros_like(w13), torch.zeros_like(w2)
+        a, sa = oracle_lib.quant_128x128(w13)
+        b, sb = oracle_lib.quant_128x128(w2)
+        experts.append((a, sa, b, sb))
+    cf = oracle_lib.cfg(H, I, Nr, Kr)
+    return cf, x, wr, bias, dout, experts
+
+
+def test_layer_backward_residual_path_is_exact(oracle_lib, bw):
+    cf, x, wr, bias, dout, experts = _layer_problem(oracle_lib, zero_weights=True)
+    r = bw.layer_backward(cf, x, wr, bias, experts, dout)
+    assert np.array_equal(r["dx"], dout.double().numpy())
+    assert all(not w.any() for w in list(r["dW13"].values()) + list(r["dW2"].values()))
+
+
+def test_layer_backward_scales_exactly_with_dout(oracle_lib, bw):
+    cf, x, wr, bias, dout, experts = _layer_problem(oracle_lib, seed=1)
+    a = bw.layer_backward(cf, x, wr, bias, experts, dout)
+    b = bw.layer_backward(cf, x, wr, bias, experts, (dout.float() * 0.25).to(torch.bfloat16))
+    # every term (residual, each expert's dx) and the FP32 rounding of their
+    # sum scale exactly by a power of two
+    assert np.array_equal(b["dx"], 0.25 * a["dx"])
+    for e in a["dW13"]:
+        assert np.array_equal(b["dW13"][e], 0.25 * a["dW13"][e]) and np.array_equal(b["dW2"][e], 0.25 * a["dW2"][e])
+
+
+def test_layer_backward_tracks_the_dense_layer_gradient(oracle_lib, bw):
+    cf, x, wr, bias, dout, experts = _layer_problem(oracle_lib, T=128, seed=2)
+    r = bw.layer_backward(cf, x, wr, bias, experts, dout)
+    I, Nr = S.TINY["I"], S.TINY["Nr"]
+    xd, dd = x.double().numpy(), dout.double().numpy()
+
+    def dense(e):
+        W13 = oracle_lib.dequant(experts[e][0], experts[e][1], 128)
+        return W13[:I], W13[I:], oracle_lib.dequant(experts[e][2], experts[e][3], 128)
+
+    dx = dd + dense_backward(xd, dd, *dense(Nr))["dx"]
+    used = sorted(set(r["idx"].reshape(-1).tolist()))
+    assert sorted(k for k in r["dW13"] if k < Nr) == used and Nr in r["dW13"]
+    rel_w = []
+    for e in used:
+        toks, slots = np.nonzero(r["idx"] == e)
+        g = r["gate"][toks, slots][:, None]
+        ref = dense_backward(xd[toks], g * dd[toks], *dense(e))
+        dx[toks] += ref["dx"]
+        rel_w.append(_rel(r["dW2"][e], ref["dW2"]))
+        rel_w.append(_rel(r["dW13"][e], np.concatenate([ref["dW1"], ref["dW3"]])))
+    # residual excluded from the comparison so it does not mask the experts' part
+    rel = _rel(r["dx"] - dd, dx - dd)
+    print(f"layer dx rel-Frobenius {rel:.3f}; weight gradients max {max(rel_w):.3f}")
+    assert rel < 0.12 and max(rel_w) < 0.15
