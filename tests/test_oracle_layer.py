@@ -119,3 +119,27 @@ def test_bias_update_closed_form(oracle_lib):
     # fractional mean: 3 tokens x 1 slot over 2 experts -> 1.5 each
     out2 = oracle_lib.bias_update(np.zeros(2, np.float32), np.array([2, 1], np.int32), 2, 3, 0.001)
     assert out2[0] == -g and out2[1] == g
+
+
+def test_round_bf16_ties_subnormals_and_signs(oracle_lib):
+    """The output rounding (bf16, round to nearest, ties to even) on the cases
+    random outputs never reach: exact midpoints between neighbouring bf16
+    values, values a hair off them, subnormals, signed zeros."""
+    rng = np.random.default_rng(3)
+    # random normal bf16 values b and their upper neighbours
+    bits = rng.integers(0x0080, 0x7F00, size=4000).astype(np.uint16)  # positive normals
+    lo = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    hi = ((bits.astype(np.uint32) + 1) << 16).view(np.float32).astype(np.float64)
+    mid = (lo + hi) / 2  # exact in double
+    even = np.where(bits % 2 == 0, bits, bits + 1).astype(np.uint16)
+    got = oracle_lib.round_bf16(np.concatenate([mid, -mid]))
+    assert np.array_equal(got[:4000], even)
+    assert np.array_equal(got[4000:], even | np.uint16(0x8000))
+    # a hair above / below the midpoint goes to the nearer neighbour
+    up = oracle_lib.round_bf16(np.nextafter(mid, np.inf))
+    down = oracle_lib.round_bf16(np.nextafter(mid, -np.inf))
+    assert np.array_equal(up, (bits + 1).astype(np.uint16)) and np.array_equal(down, bits)
+    # subnormals (below 2^-126) and zeros, against the library cast
+    sub = np.concatenate([rng.uniform(-2.0 ** -126, 2.0 ** -126, 2000), [0.0, -0.0, 2.0 ** -133, -2.0 ** -134]])
+    ref = torch.from_numpy(sub).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle_lib.round_bf16(sub), ref)
