@@ -138,3 +138,21 @@ def test_serial_leg_runs_copies_and_steps_in_series(fake_cuda):
     ms = bench.e2e_serial(lambda xi, ob: calls.append(log.current), x_h, out_h, main, "cpu", 3, 1)
     assert ms == 7.0 and calls == ["main"] * 3
     assert [o[1] for o in log.ops] == ["record", "record"]
+
+
+def test_profiled_traffic_is_used_only_for_the_captured_source(tmp_path, monkeypatch):
+    """bench.py reports a kernel's DRAM traffic from profiles/traffic.json
+    only while the kernel's sources hash to the value stored with it."""
+    import json
+
+    import bench
+    for kernel in ("gemm_fp8_kernel<0>", "gemm_mx_kernel<0>"):
+        assert bench.profiled_traffic("prefill", kernel) is not None, kernel
+        assert bench.profiled_traffic("decode", kernel) is None
+    d = json.load(open(bench.TRAFFIC_FILE))
+    d["gemm_fp8_kernel<0>:prefill"]["src_sha"] = "0" * 16
+    f = tmp_path / "traffic.json"
+    f.write_text(json.dumps(d))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.profiled_traffic("prefill", "gemm_fp8_kernel<0>") is None
+    assert bench.profiled_traffic("prefill", "gemm_mx_kernel<0>") is not None
