@@ -8,6 +8,8 @@ for the read-back of the output two steps earlier (the buffer it overwrites),
 earlier has finished with its buffer, (d) read every step's output back after
 that step, and (e) close the timed region only after both copy streams.
 The serial leg copies in, steps and copies out in series on one stream.
+The stored DRAM traffic of a kernel is reported only for the sources it was
+captured on.
 """
 import contextlib
 import os
@@ -72,10 +74,6 @@ def fake_cuda(monkeypatch):
     return bench, log
 
 
-def _tagged(events_list):
-    return [e.tag for e in events_list]
-
-
 def test_pipelined_leg_orders_copies_and_steps(fake_cuda):
     bench, log = fake_cuda
     main = _Stream(log, "main")
@@ -97,10 +95,6 @@ def test_pipelined_leg_orders_copies_and_steps(fake_cuda):
     assert seen[0] != seen[1] and all(seen[k] == seen[k % 2] for k in range(steps))
     # events in creation order: e0/e1 timing, then x_ready[2], computed[2], read_back[2]
     recs = [(s, t) for s, kind, t in ops if kind == "record"]
-    waits = [(s, t) for s, kind, t in ops if kind == "wait"]
-    by_tag = {}
-    for i, (s, kind, t) in enumerate(ops):
-        by_tag.setdefault(t, []).append((i, s, kind))
     # group each step's records: the h2d stream records x_ready, main records computed, d2h read_back
     x_ready = [t for s, t in recs if s == "h2d"]
     computed = [t for s, t in recs if s == "main"][1:-1]  # drop the timing events e0, e1
@@ -126,7 +120,6 @@ def test_pipelined_leg_orders_copies_and_steps(fake_cuda):
     # the start event precedes every copy: both copy streams wait on it first
     e0 = ops[0]
     assert e0[:2] == ("main", "record") and ops[1:3] == [("h2d", "wait", e0[2]), ("d2h", "wait", e0[2])]
-    assert waits and by_tag
 
 
 def test_serial_leg_runs_copies_and_steps_in_series(fake_cuda):
@@ -141,18 +134,17 @@ def test_serial_leg_runs_copies_and_steps_in_series(fake_cuda):
 
 
 def test_profiled_traffic_is_used_only_for_the_captured_source(tmp_path, monkeypatch):
-    """bench.py reports a kernel's DRAM traffic from profiles/traffic.json
-    only while the kernel's sources hash to the value stored with it."""
     import json
 
     import bench
-    for kernel in ("gemm_fp8_kernel<0>", "gemm_mx_kernel<0>"):
-        assert bench.profiled_traffic("prefill", kernel) is not None, kernel
-        assert bench.profiled_traffic("decode", kernel) is None
-    d = json.load(open(bench.TRAFFIC_FILE))
-    d["gemm_fp8_kernel<0>:prefill"]["src_sha"] = "0" * 16
+    k1, k2 = "gemm_fp8_kernel<0>", "gemm_mx_kernel<0>"
+    d = {f"{k1}:prefill": dict(bytes_per_launch=123.0, src_sha=bench.gemm_source_sha(k1)),
+         f"{k2}:prefill": dict(bytes_per_launch=456.0, src_sha="0" * 16)}
     f = tmp_path / "traffic.json"
     f.write_text(json.dumps(d))
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
-    assert bench.profiled_traffic("prefill", "gemm_fp8_kernel<0>") is None
-    assert bench.profiled_traffic("prefill", "gemm_mx_kernel<0>") is not None
+    assert bench.profiled_traffic("prefill", k1) == 123.0
+    assert bench.profiled_traffic("prefill", k2) is None   # captured on other sources
+    assert bench.profiled_traffic("decode", k1) is None    # never captured
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "absent.json"))
+    assert bench.profiled_traffic("prefill", k1) is None
