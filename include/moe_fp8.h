@@ -93,7 +93,9 @@ MOE_API int moe_abi_version(void);
  *   top_k       K_r experts per token, 1..min(N_r, 16) (8)
  *   n_shared    N_s always-active experts, 0 or 1 (1)
  *   n_groups    group-limited routing: 0 = off, else number of equal
- *               contiguous expert groups (divides N_r, <= 32)
+ *               contiguous expert groups (divides N_r, <= 32, at least two
+ *               experts per group: a group's score is the sum of its two
+ *               best biased scores)
  *   topk_groups groups kept per token when n_groups > 0 (1..n_groups)
  *   route_scale factor applied to the normalised gates (1.0 = the pages')
  *   scale_mode  MOE_SCALE_AMAX (0, the pages' S = amax / 448, the default of
@@ -213,9 +215,11 @@ MOE_API int moe_route(const moe_config *cfg, const void *x_dev, const void *wr_d
  *     i.e. moe_route_workspace_size(cfg, T) - 256 <= 16 MiB (for
  *     n_routed = 256 every T <= 8192 fits); larger calls return
  *     MOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
- *   - The first call on a device looks up the scratch's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *   - Every call looks up the scratch's device address in the current
+ *     device's context (cudaGetSymbolAddress, which allocates nothing), so
+ *     the address stays right after a context is torn down and created
+ *     again.  The first call on a device may load the library's device code
+ *     into that context: make it before any stream capture.
  *   - Every call shares the one scratch and it keeps the last call's
  *     contents (each call overwrites every partial it reads, so nothing has
  *     to start at zero); calls whose execution overlaps on the GPU race on

@@ -85,6 +85,9 @@ def num_threads() -> int:
 
 
 def cfg(H, I, Nr, Kr, Ns=1, n_groups=0, topk_groups=0, route_scale=1.0, scale_mode=SCALE_AMAX) -> Cfg:
+    # group-limited routing scores a group by the sum of its two best biased
+    # scores, which needs at least two experts per group
+    assert n_groups == 0 or (Nr % n_groups == 0 and Nr // n_groups >= 2), "groups need two experts or more"
     return Cfg(H, I, Nr, Kr, Ns, n_groups, topk_groups, scale_mode, route_scale)
 
 

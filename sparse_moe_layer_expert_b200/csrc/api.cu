@@ -93,6 +93,9 @@ int check_cfg(const moe_config *c) {
   if (c->n_groups < 0) return MOE_ERR_INVALID_ARG;
   if (c->n_groups > 0) {
     if (c->n_groups > 32 || c->n_routed % c->n_groups) return MOE_ERR_UNSUPPORTED_SHAPE;
+    // a group's score is the sum of its two best biased scores: it needs two
+    // experts per group
+    if (c->n_routed / c->n_groups < 2) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->topk_groups < 1 || c->topk_groups > c->n_groups) return MOE_ERR_INVALID_ARG;
     if (static_cast<int64_t>(c->topk_groups) * (c->n_routed / c->n_groups) < c->top_k) return MOE_ERR_INVALID_ARG;
   }

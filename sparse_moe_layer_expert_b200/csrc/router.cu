@@ -15,8 +15,6 @@
 //     pre-selection and K_r rounds of warp-wide argmax.
 //  3. seq_balance_kernel: the sequence-wise balance loss of a routed batch
 //     (a metric of the routing, outside the layer step).
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 
@@ -404,27 +402,16 @@ cudaError_t launch_seq_balance(const float *partial, int n_ks, int64_t T, int Nr
 // library holds it (16 MiB) until the process exits, and all calls share it.
 static __device__ __align__(256) float g_route_scratch[kRouteNoAllocScratchFloats];
 
-namespace {
-std::mutex g_scratch_mu;
-float *g_scratch_ptr[64] = {nullptr};
-}  // namespace
-
-// Device address of g_route_scratch for the current device.  The first call on
-// a device looks it up with cudaGetSymbolAddress (with that device current)
-// and caches it; host code must never pass the array's host-side name itself.
+// Device address of g_route_scratch in the current device's context, looked
+// up on every call (cudaGetSymbolAddress allocates nothing and is cheap), so
+// a context torn down and created again (cudaDeviceReset) never leaves a
+// stale address behind.  Host code must never pass the array's host-side
+// name itself.
 cudaError_t route_static_scratch(float **ptr) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void *p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_route_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = static_cast<float *>(p);
-  }
-  *ptr = g_scratch_ptr[dev];
+  *ptr = static_cast<float *>(p);
   return cudaSuccess;
 }
 
@@ -432,7 +419,8 @@ int router_ksplit(int64_t T, int Nr, int H) {
   const int64_t base = ((T + 127) / 128) * ((Nr + 127) / 128);
   const int kb_total = H / 64;
   if (base <= 0) return 1;
-  int64_t ks = (148 + base - 1) / base;
+  const int64_t sms = moe_host::sm_count();
+  int64_t ks = (sms + base - 1) / base;
   if (ks > 16) ks = 16;
   if (ks > kb_total) ks = kb_total;
   if (ks < 1) ks = 1;

@@ -56,6 +56,11 @@ def test_host_validation_without_device(m):
     # too many experts per token / groups that cannot hold top_k
     assert m.moe_workspace_size(m.config(512, 256, 16, 17), 8) == 0
     assert m.moe_workspace_size(m.config(512, 256, 16, 5, 1, 4, 1), 8) == 0
+    # one expert per group: a group score (sum of the two best) is undefined
+    assert m.moe_workspace_size(m.config(512, 256, 16, 4, 1, 16, 4), 8) == 0
+    assert L.moe_forward(C.byref(m.config(512, 256, 16, 4, 1, 16, 4)), None, None, None, 64, None, 0, None, None,
+                         None, 0, None, None) == m.MOE_ERR_UNSUPPORTED_SHAPE
+    assert m.moe_workspace_size(m.config(512, 256, 16, 4, 1, 8, 4), 8) > 0
     # a valid call with non-null pointers reaches the device check
     assert L.fp8_quant_1x128(16, 4, 128, 128, 16, 16, None) == m.MOE_ERR_NO_DEVICE
 

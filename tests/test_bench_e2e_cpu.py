@@ -148,3 +148,18 @@ def test_profiled_traffic_is_used_only_for_the_captured_source(tmp_path, monkeyp
     assert bench.profiled_traffic("decode", k1) is None    # never captured
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "absent.json"))
     assert bench.profiled_traffic("prefill", k1) is None
+
+
+def test_committed_traffic_figures_match_their_sources():
+    """Every DRAM-traffic figure committed under profiles/ names the hash of
+    the kernel sources it was captured on, and that hash is the current one:
+    a figure whose kernel changed since must be recaptured or removed, never
+    re-labelled."""
+    import json
+
+    import bench
+    d = json.load(open(bench.TRAFFIC_FILE))
+    for key, ent in d.items():
+        kernel = key.split(":")[0]
+        assert ent["src_sha"] == bench.gemm_source_sha(kernel), f"{key}: captured on other sources"
+        assert "src_sha_note" not in ent, f"{key}: a hash must come from a capture"
