@@ -54,6 +54,7 @@ _CSRC = os.path.join(ROOT, "sparse_moe_layer_expert_b200", "csrc")
 GEMM_SOURCES = {
     "gemm_fp8_kernel": [os.path.join(_CSRC, f) for f in ("gemm.cu", "gemm_tiles.cuh", "common.cuh")],
     "gemm_mx_kernel": [os.path.join(_CSRC, f) for f in ("gemm_mx.cu", "gemm_tiles.cuh", "common.cuh")],
+    "gemm_pair_kernel": [os.path.join(_CSRC, f) for f in ("gemm_pair.cu", "gemm_tiles.cuh", "common.cuh")],
 }
 
 
@@ -76,6 +77,12 @@ def parse(argv=None):
     p.add_argument("--scale-mode", choices=("amax", "pow2"), default="amax",
                    help="amax: S = amax/448 (the pages, default); pow2: power-of-two scales applied by the "
                         "tensor core (block-scaled MMA)")
+    p.add_argument("--gemm", choices=("auto", "single", "pair"), default="auto",
+                   help="grouped GEMM kernel of the default scale mode: the library's default (auto: single "
+                        "CTAs), single CTAs, or CTA pairs (tcgen05 cta_group::2)")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the other workloads (decode, skewed, standalone GEMM, FP8 ceiling) measured after "
+                        "the headline at N = 1")
     p.add_argument("--tokens", type=int, default=0, help="override T (profiling of smaller cases)")
     p.add_argument("--experts", type=int, default=0, help="override N_r (profiling of smaller cases)")
     return p.parse_args(argv)
@@ -332,18 +339,203 @@ def oracle_sample(cfg: dict, n_tok: int, seed: int, x_full, wr, bias, expert_bf1
         experts[e] = (a, sa, b, sb)
     wr_c, bias_c = wr.cpu(), bias.cpu()
 
-    def run():
+    def run(threads=None):
+        if threads:
+            oracle.set_num_threads(threads)
         return oracle.forward(ocf, x, wr_c, bias_c, experts, tokens=np.arange(n_tok))
 
     return run, oracle.num_threads()
 
 
-def time_oracle(run, n_tok: int, reps: int = 1) -> float:
+def time_oracle(run, n_tok: int, reps: int = 1, threads=None) -> float:
+    if threads:
+        run(threads)  # untimed: sets the thread count (and warms the caches)
     t0 = time.perf_counter()
     for _ in range(reps):
         run()
     dt = (time.perf_counter() - t0) / reps
     return n_tok / dt
+
+
+
+# ------------------------------------------------ other workloads (same run)
+def time_layer_steps(M, torch, layer, x, steps: int, warmup: int, stream, dev, gpu_id: str, bias_update=True):
+    """Device time of `steps` back-to-back layer steps (forward + the step's
+    bias update into a working copy of the bias) after `warmup` untimed ones,
+    with per-stage times from the library's events and the SM clocks sampled
+    meanwhile."""
+    T = x.shape[0]
+    Nr, Kr = layer.cfg.n_routed, layer.cfg.top_k
+    out = torch.empty((T, layer.cfg.hidden), dtype=torch.bfloat16, device=dev)
+    counts = torch.empty(Nr, dtype=torch.int32, device=dev)
+    bias_next = layer.bias.clone()
+
+    def step():
+        layer.forward(x, out=out, counts_out=counts, stream=stream)
+        if bias_update:
+            M.moe_bias_update(bias_next, counts, Nr, T * Kr, 0.001, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    layer.check(stream)
+    n_ev = M.MOE_PROFILE_EVENTS
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
+    ev_end = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    for e in ev_end:
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(gpu_id)
+    with sampler:
+        for k in range(steps):
+            M.moe_profile_events(ev[k])
+            step()
+            ev_end[k].record(stream)
+        M.moe_profile_events(None)
+        torch.cuda.synchronize(dev)
+    layer.check(stream)
+    stage_ms = {name: sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)) / steps
+                for i, name in enumerate(M.PROFILE_STAGES)}
+    total_ms = ev[0][0].elapsed_time(ev_end[-1])
+    return dict(ms_per_step=total_ms / steps, stage_ms=stage_ms, counts=counts.cpu(), clocks=sampler.summary(),
+                timed_ms=total_ms)
+
+
+def fp8_ceiling(torch, dev, gpu_id: str, n: int = 8192, iters: int = 20):
+    """Dense FP8 (E4M3) matmul throughput of the library GEMM torch ships
+    (torch._scaled_mm, per-tensor scales, bf16 out) at n^3: the device's FP8
+    tensor ceiling, measured in this run.  A measurement only: nothing of the
+    layer runs through it."""
+    try:
+        a = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn).t()  # column-major operand
+        one = torch.ones((), device=dev)
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sampler = ClockSampler(gpu_id)
+        with sampler:
+            e0.record()
+            for _ in range(iters):
+                torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / iters
+        del a, b
+        return dict(tflops=round(2.0 * n ** 3 / (ms / 1e3) / 1e12, 1), n=n, ms=round(ms, 4),
+                    how="torch._scaled_mm e4m3 x e4m3 -> bf16, per-tensor scales, %d back-to-back" % iters,
+                    clocks=sampler.summary())
+    except Exception as exc:  # report why instead of failing the bench
+        return dict(tflops=None, error=str(exc).splitlines()[0][:160])
+
+
+def time_blockscaled_gemm(M, torch, S, dev, gpu_id: str, Mrows: int, K: int, N: int, seed: int, steps: int,
+                          warmup: int, copies: int = 8):
+    """The standalone fine-grained block-scaled GEMM (fp8_blockscaled_gemm) at
+    [M, K] x [K, N]: A ~ N(0,1) with 1% outliers x50 quantized 1x128, B ~
+    N(0, 0.02^2) quantized 128x128 (passed as [N, K]); `copies` quantized
+    copies of B are used in turn so that B streams from HBM every call."""
+    a = S.gen_gemm_a(Mrows, K, seed, device=dev)
+    A, sA = M.fp8_quant_1x128(a)
+    bs = []
+    for c in range(copies):
+        bt = S.gen_gemm_b(K, N, seed + 101 * c, device=dev).t().contiguous()
+        bs.append(M.fp8_quant_128x128(bt))
+        del bt
+    C = torch.empty((Mrows, N), dtype=torch.bfloat16, device=dev)
+    err = M.new_err_flag(dev)
+    for i in range(warmup):
+        M.fp8_blockscaled_gemm(A, sA, bs[i % copies][0], bs[i % copies][1], C=C, err=err)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_id)
+    with sampler:
+        e0.record()
+        for i in range(steps):
+            M.fp8_blockscaled_gemm(A, sA, bs[i % copies][0], bs[i % copies][1], C=C, err=err)
+        e1.record()
+        torch.cuda.synchronize(dev)
+    st, v = M.moe_check_device_error(err)
+    if st != M.MOE_OK:
+        raise M.MoeError(st, f"fp8_blockscaled_gemm device error {v:#x}")
+    ms = e0.elapsed_time(e1) / steps
+    flops = 2.0 * Mrows * N * K
+    return dict(ms=round(ms, 4), tflops=round(flops / (ms / 1e3) / 1e12, 1), flops=flops, clocks=sampler.summary(),
+                l2="B rotated over %d quantized copies (%.0f MB)" % (copies, copies * N * K / 1e6))
+
+
+def extra_workloads(M, torch, S, layer, args, seed: int, stream, dev, gpu_id: str, peaks: dict) -> dict:
+    """The other configurations of the workload set, measured in the same
+    process on the same resident expert weights: the decode-shaped layer
+    (T = 64, zero bias), the skewed layer (T = 16384, mixture input,
+    group-limited routing 8 x 32 / top-4 groups, zero bias, then one bias
+    update), the standalone block-scaled GEMM at both shapes and the device's
+    FP8 tensor ceiling."""
+    H, I, Nr, Kr = layer.cfg.hidden, layer.cfg.inter, layer.cfg.n_routed, layer.cfg.top_k
+    res = {}
+    ceil = fp8_ceiling(torch, dev, gpu_id)
+    res["fp8_ceiling"] = ceil
+    fp8_peak = ceil.get("tflops") or 2.0 * peaks["bf16"]
+    fp8_src = "measured in this run (torch._scaled_mm)" if ceil.get("tflops") else \
+        peaks["src"] + " bf16 burst x 2 (nominal FP8/bf16 ratio)"
+    # decode: T = 64, zero bias
+    dec = S.CONFIGS["decode"]
+    zero = torch.zeros(Nr, dtype=torch.float32, device=dev)
+    lay_d = layer.sibling(bias=zero)
+    x_d = S.gen_x(dec["T"], H, seed * 1009 + 7, device=dev)
+    r = time_layer_steps(M, torch, lay_d, x_d, args.steps, args.warmup, stream, dev, gpu_id)
+    touched = int((r["counts"] > 0).sum())
+    alg = algorithmic_counts(dict(dec), dec["T"], touched)
+    layer_bytes = alg["layer_weight_bytes"] + Nr * H * 2 + dec["T"] * H * 2 * 2
+    res["decode"] = dict(
+        workload=f"decode: T={dec['T']} H={H} I={I} Nr={Nr} Kr={Kr} Ns=1, zero bias",
+        ms_per_step=round(r["ms_per_step"], 4), tokens_per_s=round(dec["T"] / (r["ms_per_step"] / 1e3), 1),
+        experts_touched=touched + 1,
+        layer_hbm=dict(algorithmic_bytes=layer_bytes, achieved_gbs=round(layer_bytes / (r["ms_per_step"] / 1e3) / 1e9, 1),
+                       frac=round(layer_bytes / (r["ms_per_step"] / 1e3) / 1e9 / peaks["hbm"], 4),
+                       peak=peaks["hbm"], how="expert weights touched + router weights + x in/out over the whole "
+                                            "step (layer + bias update) / HBM copy peak"),
+        gate_up_hbm_frac=round(alg["g1_bytes"] / (r["stage_ms"]["gemm_gate_up"] / 1e3) / 1e9 / peaks["hbm"], 4),
+        stage_ms={k: round(v, 4) for k, v in r["stage_ms"].items()}, clocks=r["clocks"])
+    del lay_d, x_d
+    # skewed: T = 16384, mixture input, group-limited routing, zero bias
+    sk = S.CONFIGS["skewed"]
+    lay_s = layer.sibling(bias=zero.clone(), n_groups=sk["n_groups"], topk_groups=sk["topk_groups"])
+    x_s, _ = S.gen_mixture_x(sk["T"], H, seed * 1009 + 11, device=dev)
+    r = time_layer_steps(M, torch, lay_s, x_s, args.steps, args.warmup, stream, dev, gpu_id)
+    Ts = sk["T"]
+    mean = Ts * Kr / Nr
+    c0 = r["counts"]
+    lay_s.bias_update(c0.to(dev), Ts)  # one update b_i -/+ 0.001 applied for real
+    c1 = torch.empty(Nr, dtype=torch.int32, device=dev)
+    lay_s.forward(x_s, counts_out=c1, stream=stream)
+    lay_s.check(stream)
+    touched = int((c0 > 0).sum())
+    alg = algorithmic_counts(dict(sk), Ts, touched)
+    g_ms = r["stage_ms"]["gemm_gate_up"] + r["stage_ms"]["gemm_down"]
+    tfl = (alg["g1_flops"] + alg["g2_flops"]) / (g_ms / 1e3) / 1e12
+    res["skewed"] = dict(
+        workload=f"skewed: T={Ts} H={H} I={I} Nr={Nr} Kr={Kr} Ns=1, groups {sk['n_groups']}/{sk['topk_groups']}, "
+                 "32-centroid Zipf(1) mixture input, zero bias",
+        ms_per_step=round(r["ms_per_step"], 4), tokens_per_s=round(Ts / (r["ms_per_step"] / 1e3), 1),
+        load_max_over_mean=round(float(c0.max()) / mean, 3),
+        after_one_bias_update=round(float(c1.max().item()) / mean, 3),
+        grouped_gemm_tflops=round(tfl, 1), grouped_gemm_frac_fp8=round(tfl / fp8_peak, 4), fp8_peak=fp8_peak,
+        fp8_peak_src=fp8_src, frac_of_nominal_4500=round(tfl / 4500.0, 4),
+        stage_ms={k: round(v, 4) for k, v in r["stage_ms"].items()}, clocks=r["clocks"])
+    del lay_s, x_s
+    torch.cuda.empty_cache()
+    # the standalone block-scaled GEMM at both shapes
+    for (Mr, K, N) in S.GEMM_SHAPES:
+        g = time_blockscaled_gemm(M, torch, S, dev, gpu_id, Mr, K, N, seed, args.steps, args.warmup)
+        g.update(frac_fp8=round(g["tflops"] / fp8_peak, 4), fp8_peak=fp8_peak, fp8_peak_src=fp8_src,
+                 frac_of_nominal_4500=round(g["tflops"] / 4500.0, 4))
+        res[f"gemm_M{Mr}_K{K}_N{N}"] = g
+        torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------------ main
@@ -360,6 +552,7 @@ def main(argv=None):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    M.moe_set_gemm_variant({"auto": M.MOE_GEMM_AUTO, "single": M.MOE_GEMM_SINGLE, "pair": M.MOE_GEMM_PAIR}[args.gemm])
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
@@ -465,10 +658,15 @@ def main(argv=None):
     dom_ms = max(g1_ms, g2_ms)
     dom_bytes = alg["g1_bytes"] if dom == "gemm_gate_up" else alg["g2_bytes"]
     dom_flops = alg["g1_flops"] if dom == "gemm_gate_up" else alg["g2_flops"]
-    fp8_peak = 2.0 * peaks["bf16_sustained"]  # FP8 dense = 2 x bf16 (nominal ratio 4.5 / 2.25 PFLOP/s)
+    # FP8 dense = 2 x bf16 (nominal ratio 4.5 / 2.25 PFLOP/s); the burst figure
+    # for a timed region under a second, the sustained one for longer ones
+    sustained = total_ms > 1000.0
+    fp8_peak = 2.0 * (peaks["bf16_sustained"] if sustained else peaks["bf16"])
+    fp8_src = peaks["src"] + (" bf16 sustained x 2" if sustained else " bf16 burst x 2")
     t_mem = dom_bytes / (peaks["hbm"] * 1e9)
     t_tc = dom_flops / (fp8_peak * 1e12)
-    kname = "gemm_mx_kernel" if args.scale_mode == "pow2" else "gemm_fp8_kernel"
+    pair = args.scale_mode != "pow2" and args.gemm == "pair" and (cfg["H"] // 128) % 2 == 0
+    kname = "gemm_mx_kernel" if args.scale_mode == "pow2" else ("gemm_pair_kernel" if pair else "gemm_fp8_kernel")
     kernel_name = f"{kname}<0>" if dom == "gemm_gate_up" else f"{kname}<1>"
     if t_mem >= t_tc:
         achieved = dom_bytes / (dom_ms / 1e3) / 1e9
@@ -479,7 +677,7 @@ def main(argv=None):
         achieved = dom_flops / (dom_ms / 1e3) / 1e12
         roofline = dict(bound="tensor", achieved=round(achieved, 1), peak=round(fp8_peak, 1), unit="TFLOP/s",
                         frac=round(achieved / fp8_peak, 4), traffic=profiled_traffic(args.workload, kernel_name),
-                        kernel=dom, peak_src=peaks["src"] + " (bf16 sustained x 2 for FP8)",
+                        kernel=dom, peak_src=fp8_src,
                         algorithmic_flops=dom_flops)
     gemm_tflops = (alg["g1_flops"] + alg["g2_flops"]) / ((g1_ms + g2_ms) / 1e3) / 1e12
 
@@ -530,16 +728,26 @@ def main(argv=None):
         layer.check(stream)
         balance = dict(gamma=0.001, steps=args.balance_steps, max_over_mean={str(k): v for k, v in traj.items()})
 
+    # ------------------------------------------------ other workloads (N = 1)
+    extras = None
+    if world == 1 and not args.no_extras and args.workload == "prefill" and not args.tokens and not args.experts:
+        extras = extra_workloads(M, torch, S, layer, args, seed, stream, dev, gpu_id, peaks)
+
     # ------------------------------------------------ CPU oracle baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n = args.cpu_sample_tokens
         run, threads = oracle_sample(cfg, n, seed, x, wr, bias, expert_bf16)
+        used = int(min(threads, n))  # the oracle parallelises over tokens
         tps = time_oracle(run, n)
-        cpu = dict(value=round(tps, 4), unit="tokens/s", cores=int(min(threads, n)), kind="oracle",
+        tps1 = time_oracle(run, n, threads=1)
+        run(threads)
+        cpu = dict(value=round(tps, 4), unit="tokens/s", cores=used, kind="oracle", nproc=os.cpu_count(),
+                   threads_used=used, one_thread_value=round(tps1, 4),
                    sample=f"first {n} tokens of the {args.workload} batch: full layer (quantize, route over all "
-                          f"{cfg['Nr']} experts, shared + top-{cfg['Kr']} FP8 FFNs, combine); weight "
-                          f"quantization by the oracle excluded (set-up)")
+                          f"{cfg['Nr']} experts, shared + top-{cfg['Kr']} FP8 FFNs, combine), OpenMP over the "
+                          f"tokens ({used} threads; one_thread_value with 1); weight quantization by the oracle "
+                          f"excluded (set-up)")
 
     if world > 1:
         dist.destroy_process_group()
@@ -555,10 +763,12 @@ def main(argv=None):
                     l2="no flush: per-step working set >= 11 GB of expert weights >> 126 MB L2",
                     scales="amax/448 (FP32 promotion per 128-K block)" if args.scale_mode == "amax" else
                     "power of two (applied by the tensor core, block-scaled MMA)",
+                    gemm_kernel=kname,
                     seed=seed),
         roofline=roofline,
         grouped_gemm_tflops=round(gemm_tflops, 1),
         grouped_gemm_frac_fp8_peak=round(gemm_tflops / fp8_peak, 4),
+        fp8_peak=dict(tflops=fp8_peak, src=fp8_src),
         layer_weight_gb=round(alg["layer_weight_bytes"] / 1e9, 3),
         experts_touched=touched + cfg.get("Ns", 1),
         load=load,
@@ -567,6 +777,7 @@ def main(argv=None):
         step_ms_min=round(min(step_ms), 4),
         cpu_baseline=cpu,
         e2e=e2e,
+        **({"workloads": extras} if extras else {}),
         gpu_launches=KERNELS_PER_STEP * args.steps,
         clocks=clocks,
     )

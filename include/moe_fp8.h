@@ -237,8 +237,9 @@ MOE_API int moe_route_noalloc(const moe_config *cfg, const void *x_dev, const vo
  * GEMM: u quantized 1x128 (fp8_quant_1x128), routed as moe_route, rows
  * grouped per expert (stable: token order, then slot), h = silu(G) * U in FP32
  * re-quantized 1x128 along I before the down projection, the down-projection
- * output scaled by the gate, then summed per token in FP32 in a fixed order
- * (residual, shared expert, slots 0..K_r-1) and written as out_dtype.
+ * output scaled by the gate (in FP32, then stored as bf16), then summed per
+ * token in FP32 in a fixed order (residual, shared expert, slots 0..K_r-1)
+ * and written as out_dtype.
  *   x_dev        bf16 [T, H]
  *   out_dev      [T, H] of MOE_DTYPE_BF16 (RNE) or MOE_DTYPE_F32
  *   idx_out_dev  nullable int32 [T, K_r]: routing decision
@@ -271,13 +272,16 @@ typedef struct {
     size_t row_src[2];  /* int32 [R]        token of each routed row           */
     size_t hq[2];       /* E4M3 [R + T*N_s, I] re-quantized SwiGLU output      */
     size_t hs[2];       /* float [I/128, P] its scales, transposed             */
-    size_t y[2];        /* float [R + T*N_s, H] gate-scaled expert outputs     */
+    size_t y[2];        /* bf16 [R + T*N_s, H] gate-scaled expert outputs
+                           (RNE of the FP32 product of the down projection
+                           and the gate)                                       */
     size_t meta[2];     /* int32 [4]: number of chunks, routed rows            */
     size_t logits[2];   /* float [S, T, N_r] router logit partials (S K-splits) */
     size_t blk_hist[2]; /* int32 [ceil(T/128), N_r] per-block expert counts    */
     size_t blk_base[2]; /* int32 [ceil(T/128), N_r] per-block first rows       */
     size_t chunks[2];   /* int32x4 per chunk: {expert | input flag << 16,
-                           activation row, output row, rows <= 128}            */
+                           activation row, output row, rows <= 128 (single
+                           CTAs) or <= 256 (CTA pairs)}                        */
     size_t total;
 } moe_ws_layout;
 MOE_API int moe_workspace_layout(const moe_config *cfg, int64_t T, moe_ws_layout *layout);
@@ -295,6 +299,98 @@ MOE_API int moe_workspace_layout(const moe_config *cfg, int64_t T, moe_ws_layout
  *   5 after down GEMM | 6 after combine */
 enum { MOE_PROFILE_EVENTS = 7 };
 MOE_API int moe_profile_events(void *const *events, int32_t n_events);
+
+/* ------------------------------------------------- expert parallelism */
+/* The layer with its routed experts spread over W ranks (one GPU each), as
+ * the DeepSeek-V3 pages run it: tokens travel to the GPUs of their experts
+ * and the expert outputs travel back by all-to-all exchanges ([P4] "Problem
+ * und Motivation" item 2 and "Kernideen", DualPipe bullet).  Rank d owns the
+ * routed experts [d*N_r/W, (d+1)*N_r/W) (N_r % W == 0); every rank holds the
+ * router, the shared expert and its own tokens.  The exchanges themselves are
+ * the caller's collectives (e.g. NCCL all-to-all over NVLink); these calls
+ * are the compute on either side of them.  One rank's forward:
+ *   1. fp8_quant_1x128 and moe_route on its tokens (xq, xs, idx, gate);
+ *   2. moe_ep_dispatch: packed rows per destination (send buffer), the row
+ *      counts and offsets per destination, each token's row per destination;
+ *   3. exchange: rows r -> d (all-to-all, send_counts rows of
+ *      moe_ep_row_bytes each);
+ *   4. moe_ep_experts on the received rows with this rank's experts: the
+ *      gate-weighted sum over each row's slots whose experts live here
+ *      (bf16 partial sums, one per received row);
+ *   5. exchange back: the partial sums d -> r (the reverse all-to-all);
+ *   6. moe_ep_experts on self_rows with the shared expert's weights
+ *      (n_routed = 1, gate 1) gives y_shared; moe_ep_combine adds u_t,
+ *      y_shared and the returned partial sums (destinations in ascending
+ *      order) in FP32.
+ * Packed row (moe_ep_row_bytes bytes, a multiple of 16): the token's H E4M3
+ * codes, its H/128 FP32 scales, K_r int32 local expert ids (-1: the slot's
+ * expert lives elsewhere) and K_r FP32 gates (0 where -1).
+ * The result equals moe_forward's up to the order of the FP32 additions and
+ * the bf16 rounding of the partial sums. */
+MOE_API int64_t moe_ep_row_bytes(const moe_config *cfg);
+
+/* Dispatch of one rank's T routed tokens (step 2).
+ *   cfg           the whole layer's shape (n_routed = all routed experts)
+ *   world         W, 1..64, dividing n_routed
+ *   xq_dev, xs_dev the tokens quantized 1x128 (E4M3 [T, H], float [T, H/128])
+ *   idx_dev, gate_dev routing decision [T, K_r] (moe_route's outputs)
+ *   send_rows_dev packed rows [send_cap_rows, moe_ep_row_bytes], grouped by
+ *                 destination (rank order), token order within a
+ *                 destination; send_cap_rows >= T * min(W, K_r)
+ *   send_counts_dev int32 [W]: rows for each destination (device; copy it
+ *                 to the host to size the exchange)
+ *   send_offsets_dev int32 [W + 1]: first row of each destination, total
+ *   row_of_dev    int32 [T, W]: row of token t for destination d, or -1
+ *   self_rows_dev nullable [T, moe_ep_row_bytes]: every token packed for the
+ *                 shared expert (slot 0 = expert 0, gate 1)
+ *   ws_dev        moe_ep_dispatch_workspace_size() bytes, 256-byte aligned
+ * err_flag_dev gets MOE_DEVERR_BAD_INDEX for an expert index out of range. */
+MOE_API size_t moe_ep_dispatch_workspace_size(const moe_config *cfg, int32_t world, int64_t T);
+MOE_API int moe_ep_dispatch(const moe_config *cfg, int32_t world, const uint8_t *xq_dev, const float *xs_dev,
+                            const int32_t *idx_dev, const float *gate_dev, int64_t T, uint8_t *send_rows_dev,
+                            int64_t send_cap_rows, int32_t *send_counts_dev, int32_t *send_offsets_dev,
+                            int32_t *row_of_dev, uint8_t *self_rows_dev, void *ws_dev, size_t ws_bytes,
+                            int32_t *err_flag_dev, void *stream);
+
+/* The experts of one rank over received packed rows (steps 4 and 6).
+ *   cfg_local     n_routed = the rank's experts (N_r / W, or 1 for the
+ *                 shared expert), top_k = the layer's K_r, n_shared = 0,
+ *                 other fields as the layer's
+ *   w_local       those experts' weights (layout of moe_weights; wr_dev unused)
+ *   rows_dev      n_rows packed rows, row_bytes = moe_ep_row_bytes(cfg_local)
+ *   partial_out_dev bf16 [n_rows, H]: per row, the sum over its slots of
+ *                 gate * FFN_expert(row) in FP32 (slot order), rounded to bf16
+ *   ws_dev        moe_ep_experts_workspace_size() bytes, 256-byte aligned */
+MOE_API size_t moe_ep_experts_workspace_size(const moe_config *cfg_local, int64_t n_rows);
+MOE_API int moe_ep_experts(const moe_config *cfg_local, const moe_weights *w_local, const uint8_t *rows_dev,
+                           int64_t n_rows, int64_t row_bytes, void *partial_out_dev, void *ws_dev, size_t ws_bytes,
+                           int32_t *err_flag_dev, void *stream);
+
+/* Combine on the sending rank (step 6): out[t] = u_t + y_shared[t] (if given)
+ * + sum over d = 0..W-1 with row_of[t, d] >= 0 of back[row_of[t, d]], in FP32,
+ * written as out_dtype.
+ *   x_dev         bf16 [T, H] (the layer input u_t)
+ *   row_of_dev    moe_ep_dispatch's int32 [T, W]
+ *   back_dev      bf16 [send rows, H]: the partial sums returned by the
+ *                 destinations, in the send buffer's row order
+ *   y_shared_dev  nullable bf16 [T, H] */
+MOE_API int moe_ep_combine(const moe_config *cfg, int32_t world, const void *x_dev, int64_t T,
+                           const int32_t *row_of_dev, const void *back_dev, const void *y_shared_dev, void *out_dev,
+                           int32_t out_dtype, void *stream);
+
+/* Kernel choice of the grouped expert GEMMs in the default scale mode
+ * (process-wide; a tuning and testing switch, the arithmetic is the same):
+ *   MOE_GEMM_AUTO   (default) the measured-fastest choice: single CTAs
+ *   MOE_GEMM_SINGLE one CTA per tile: <= 128 rows of one expert per pass over
+ *                   a weight-block pair
+ *   MOE_GEMM_PAIR   a pair of CTAs on two SMs per tile (<= 256 rows per
+ *                   weight pass, one tcgen05.mma.cta_group::2 per K step)
+ *                   when the down projection's 128-row weight blocks pair up
+ *                   (hidden a multiple of 256), else single CTAs
+ * Returns MOE_ERR_INVALID_ARG for any other value.  Takes effect for the
+ * next moe_forward on any thread; not synchronised with calls in flight. */
+enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SINGLE = 1, MOE_GEMM_PAIR = 2 };
+MOE_API int moe_set_gemm_variant(int32_t variant);
 
 /* --------------------------------------------------------- bias update */
 /* Auxiliary-loss-free balancing step ([P4] Methode 2; [P1]): with

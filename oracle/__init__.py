@@ -76,12 +76,18 @@ def lib():
             L.moe_oracle_bias_update.argtypes = [vp, vp, C.c_int, i64, f32]
             L.moe_oracle_round_bf16.argtypes = [vp, i64, vp]
             L.moe_oracle_num_threads.restype = C.c_int
+            L.moe_oracle_set_num_threads.argtypes = [C.c_int]
             _lib = L
     return _lib
 
 
 def num_threads() -> int:
     return int(lib().moe_oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's later parallel loops (OpenMP), from this thread."""
+    lib().moe_oracle_set_num_threads(int(n))
 
 
 def cfg(H, I, Nr, Kr, Ns=1, n_groups=0, topk_groups=0, route_scale=1.0, scale_mode=SCALE_AMAX) -> Cfg:

@@ -504,3 +504,14 @@ int moe_oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Threads of the following parallel regions started from the calling thread
+ * (timing of the oracle with a chosen thread count). */
+void moe_oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

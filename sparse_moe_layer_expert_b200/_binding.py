@@ -42,8 +42,13 @@ EXPORTS = (
     "fp8_quant_128x128_pow2", "fp8_blockscaled_gemm",
     "moe_route_workspace_size", "moe_route", "moe_workspace_size", "moe_forward", "moe_workspace_layout",
     "moe_bias_update", "moe_check_device_error", "moe_selftest_wait_timeout", "moe_profile_events",
-    "moe_route_noalloc", "moe_seq_balance_loss",
+    "moe_route_noalloc", "moe_seq_balance_loss", "moe_set_gemm_variant",
+    "moe_ep_row_bytes", "moe_ep_dispatch_workspace_size", "moe_ep_dispatch", "moe_ep_experts_workspace_size",
+    "moe_ep_experts", "moe_ep_combine",
 )
+MOE_GEMM_AUTO = 0
+MOE_GEMM_SINGLE = 1
+MOE_GEMM_PAIR = 2
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 16 << 20
 MOE_PROFILE_EVENTS = 7
 PROFILE_STAGES = ("quantize", "route", "group", "gemm_gate_up", "gemm_down", "combine")
@@ -91,8 +96,20 @@ lib.moe_seq_balance_loss.argtypes = [_cfgp, _i64, _i64, _f32, _vp, _sz, _vp, _vp
 lib.moe_check_device_error.argtypes = [_vp, C.POINTER(C.c_int32), _vp]
 lib.moe_selftest_wait_timeout.argtypes = [_vp, _i64, _vp]
 lib.moe_profile_events.argtypes = [C.POINTER(_vp), _i32]
+lib.moe_set_gemm_variant.argtypes = [_i32]
+lib.moe_ep_row_bytes.restype = _i64
+lib.moe_ep_row_bytes.argtypes = [_cfgp]
+lib.moe_ep_dispatch_workspace_size.restype = _sz
+lib.moe_ep_dispatch_workspace_size.argtypes = [_cfgp, _i32, _i64]
+lib.moe_ep_dispatch.argtypes = [_cfgp, _i32, _vp, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
+                                _vp]
+lib.moe_ep_experts_workspace_size.restype = _sz
+lib.moe_ep_experts_workspace_size.argtypes = [_cfgp, _i64]
+lib.moe_ep_experts.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _i64, _i64, _vp, _vp, _sz, _vp, _vp]
+lib.moe_ep_combine.argtypes = [_cfgp, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _i32, _vp]
 for _name in EXPORTS:
-    if _name not in ("moe_status_string", "moe_route_workspace_size", "moe_workspace_size"):
+    if _name not in ("moe_status_string", "moe_route_workspace_size", "moe_workspace_size", "moe_ep_row_bytes",
+                     "moe_ep_dispatch_workspace_size", "moe_ep_experts_workspace_size"):
         getattr(lib, _name).restype = C.c_int
 
 
@@ -257,6 +274,50 @@ def moe_profile_events(events) -> None:
         return
     arr = (_vp * len(events))(*[ev.cuda_event for ev in events])
     _check(lib.moe_profile_events(arr, len(events)), "moe_profile_events")
+
+
+def moe_set_gemm_variant(variant: int) -> None:
+    """Kernel choice of the grouped expert GEMMs (MOE_GEMM_AUTO, _SINGLE,
+    _PAIR), process-wide."""
+    _check(lib.moe_set_gemm_variant(variant), "moe_set_gemm_variant")
+
+
+# ---------------------------------------------------- expert parallelism
+def moe_ep_row_bytes(cfg: MoeConfig) -> int:
+    return int(lib.moe_ep_row_bytes(C.byref(cfg)))
+
+
+def moe_ep_dispatch(cfg: MoeConfig, world: int, xq, xs, idx, gate, send_rows, send_counts, send_offsets, row_of,
+                    self_rows=None, ws=None, err=None, stream=None):
+    T = xq.shape[0]
+    dev = xq.device
+    if ws is None:
+        ws = torch.empty(max(int(lib.moe_ep_dispatch_workspace_size(C.byref(cfg), world, T)), 256), dtype=torch.uint8,
+                         device=dev)
+    err = new_err_flag(dev) if err is None else err
+    _check(lib.moe_ep_dispatch(C.byref(cfg), world, _ptr(xq), _ptr(xs), _ptr(idx), _ptr(gate), T, _ptr(send_rows),
+                               send_rows.shape[0], _ptr(send_counts), _ptr(send_offsets), _ptr(row_of),
+                               _ptr(self_rows), _ptr(ws), ws.numel(), _ptr(err), _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_experts(cfg_local: MoeConfig, w_local: dict, rows, partial_out, ws=None, err=None, stream=None):
+    n = rows.shape[0]
+    dev = rows.device
+    if ws is None:
+        ws = torch.empty(max(int(lib.moe_ep_experts_workspace_size(C.byref(cfg_local), n)), 256), dtype=torch.uint8,
+                         device=dev)
+    err = new_err_flag(dev) if err is None else err
+    wst = MoeWeights(_ptr(w_local["w13"]), _ptr(w_local["s13"]), _ptr(w_local["w2"]), _ptr(w_local["s2"]), None)
+    _check(lib.moe_ep_experts(C.byref(cfg_local), C.byref(wst), _ptr(rows), n, rows.shape[1] if n else
+                              moe_ep_row_bytes(cfg_local), _ptr(partial_out), _ptr(ws), ws.numel(), _ptr(err),
+                              _stream(stream)), "moe_ep_experts")
+    return partial_out
+
+
+def moe_ep_combine(cfg: MoeConfig, world: int, x, row_of, back, y_shared, out, out_dtype=MOE_DTYPE_BF16, stream=None):
+    _check(lib.moe_ep_combine(C.byref(cfg), world, _ptr(x), x.shape[0], _ptr(row_of), _ptr(back), _ptr(y_shared),
+                              _ptr(out), out_dtype, _stream(stream)), "moe_ep_combine")
+    return out
 
 
 def ws_view(ws: torch.Tensor, layout: dict, name: str, dtype, shape) -> torch.Tensor:

@@ -3,6 +3,7 @@
 // encoding and the launch sequence of the layer forward.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -109,6 +110,16 @@ int check_cfg(const moe_config *c) {
 
 constexpr int64_t kMaxTokens = 1 << 20;
 
+// The grouped GEMMs of the default scale mode run on single CTAs; with
+// moe_set_gemm_variant(MOE_GEMM_PAIR) on CTA pairs (256 rows per weight pass)
+// when the down projection's weight blocks pair up (H a multiple of 256).
+std::atomic<int> g_gemm_variant{MOE_GEMM_AUTO};
+
+bool use_pair_gemm(int64_t H) {
+  if ((H / 128) % 2 != 0) return false;
+  return g_gemm_variant.load(std::memory_order_relaxed) == MOE_GEMM_PAIR;
+}
+
 struct Carve {
   size_t off = 0;
   void take(size_t (&slot)[2], size_t bytes) {
@@ -140,7 +151,7 @@ void make_layout(const moe_config *c, int64_t T, moe_ws_layout *L) {
   cv.take(L->row_src, R * 4);
   cv.take(L->hq, RS * I);
   cv.take(L->hs, ((I / 128) * pitch + moe::kScaleSlack) * 4);
-  cv.take(L->y, RS * H * 4);
+  cv.take(L->y, RS * H * 2);
   cv.take(L->meta, 4 * 4);
   cv.take(L->logits, ks * T * Nr * 4);
   cv.take(L->blk_hist, nblk * Nr * 4);
@@ -180,7 +191,13 @@ const char *moe_status_string(int s) {
   }
 }
 
-int moe_abi_version(void) { return 102; }
+int moe_abi_version(void) { return 103; }
+
+int moe_set_gemm_variant(int32_t variant) {
+  if (variant != MOE_GEMM_AUTO && variant != MOE_GEMM_SINGLE && variant != MOE_GEMM_PAIR) return MOE_ERR_INVALID_ARG;
+  g_gemm_variant.store(variant, std::memory_order_relaxed);
+  return MOE_OK;
+}
 
 static int quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q, float *scales,
                        void *stream, bool pow2) {
@@ -250,6 +267,7 @@ int fp8_blockscaled_gemm(const uint8_t *A, const float *sA, const uint8_t *B, co
   g.n_chunks = nullptr;
   g.dense_M = M;
   g.max_chunks = static_cast<int>((M + 127) / 128);
+  g.chunk_rows = 128;
   g.nb = static_cast<int>((N / 128 + 1) / 2);
   g.gate_up = 0;
   g.rows_per_expert = N;
@@ -341,6 +359,143 @@ int moe_workspace_layout(const moe_config *cfg, int64_t T, moe_ws_layout *layout
   return MOE_OK;
 }
 
+// Grouping, both grouped GEMMs and the combine of one forward, from rows
+// already quantized (xq rows xq_ld bytes apart, xs [T, H/128] contiguous) and
+// routed (idx, gate [T, K_r]; with allow_empty, -1 marks an unused slot).
+// out[t] = x_resid[t] (if given) + shared expert (if N_s) + sum_k g y.
+struct ExpertPath {
+  const moe_config *cfg;
+  const moe_weights *w;
+  int64_t T;
+  const uint8_t *xq;
+  int64_t xq_ld;
+  const float *xs;
+  const int32_t *idx;
+  const float *gate;
+  int allow_empty;
+  const void *x_resid;
+  void *out;
+  int out_f32;
+  int32_t *counts_out;
+  const moe_ws_layout *L;
+  void *ws;
+  int32_t *err;
+  cudaStream_t st;
+};
+
+static cudaError_t run_expert_path(const ExpertPath &P) {
+  const moe_config *cfg = P.cfg;
+  const moe_weights *w = P.w;
+  const moe_ws_layout &L = *P.L;
+  void *ws = P.ws;
+  cudaStream_t st = P.st;
+  int32_t *err_flag = P.err;
+  const int64_t T = P.T;
+  const int H = cfg->hidden, I = cfg->inter, Nr = cfg->n_routed, Kr = cfg->top_k, Ns = cfg->n_shared;
+  const int64_t R = T * Kr, RS = R + T * Ns;
+  const int64_t E = static_cast<int64_t>(Nr) + Ns;
+  int32_t *counts = at<int32_t *>(ws, L.counts);
+  int32_t *offsets = at<int32_t *>(ws, L.offsets);
+  int32_t *pos = at<int32_t *>(ws, L.pos);
+  uint8_t *ap = at<uint8_t *>(ws, L.ap);
+  float *as_t = at<float *>(ws, L.as);
+  float *row_gate = at<float *>(ws, L.row_gate);
+  int32_t *row_src = at<int32_t *>(ws, L.row_src);
+  uint8_t *hq = at<uint8_t *>(ws, L.hq);
+  float *hs_t = at<float *>(ws, L.hs);
+  __nv_bfloat16 *y = at<__nv_bfloat16 *>(ws, L.y);
+  int32_t *meta = at<int32_t *>(ws, L.meta);
+  int32_t *blk_hist = at<int32_t *>(ws, L.blk_hist);
+  int32_t *blk_base = at<int32_t *>(ws, L.blk_base);
+  int4 *chunks = at<int4 *>(ws, L.chunks);
+  const int64_t max_chunks = moe::max_chunks(T, Kr, Nr, Ns);
+  const bool pow2 = cfg->scale_mode == MOE_SCALE_POW2;
+  const bool pair = !pow2 && use_pair_gemm(H);
+  const int chunk_rows = pair ? 256 : 128;
+
+  cudaError_t e = moe::launch_hist(P.idx, T, Kr, Nr, P.allow_empty, blk_hist, err_flag, st);
+  if (e == cudaSuccess)
+    e = moe::launch_build_chunks(blk_hist, T, Kr, Nr, Ns, chunk_rows, counts, offsets, blk_base, chunks, meta,
+                                 P.counts_out, st);
+  if (e == cudaSuccess) e = moe::launch_rank(P.idx, P.gate, T, Kr, Nr, Ns, blk_base, row_gate, row_src, pos, st);
+  const int64_t pitch = moe::scale_pitch(R, T);
+  if (e == cudaSuccess) e = moe::launch_copy_rows(P.xq, P.xq_ld, P.xs, row_src, R, T, Ns, H, ap, as_t, pitch, st);
+  if (e == cudaSuccess) e = prof_mark(3, st);
+  if (e == cudaSuccess) {
+    // gate/up projection + SwiGLU + 1x128 requantization
+    moe::GemmLaunch g{};
+    g.w = w->w13_dev;
+    g.w_rows = E * 2 * I;
+    g.a0 = ap;
+    g.a0_rows = R;
+    g.a1 = Ns ? P.xq : ap;  // the shared expert's rows are the quantized input itself
+    g.a1_rows = Ns ? T : R;
+    g.a1_ld = Ns ? P.xq_ld : H;
+    g.K = H;
+    g.sw = w->s13_dev;
+    g.sa0 = as_t;
+    g.sa1 = as_t;
+    g.sa_transposed = 1;
+    g.sa_ld = pitch;
+    g.chunks = chunks;
+    g.n_chunks = meta;
+    g.max_chunks = static_cast<int>(max_chunks);
+    g.chunk_rows = chunk_rows;
+    g.nb = moe::gemm1_blocks(I);
+    g.gate_up = 1;
+    g.half = I;
+    g.rows_per_expert = 2 * static_cast<int64_t>(I);
+    g.epi = moe::EPI_SWIGLU_Q;
+    g.out = hq;
+    g.ldo = I;
+    g.out_rows = RS;
+    g.out_cols = 2 * I;  // block B (up) shares block A's output columns
+    g.out_scale = hs_t;
+    g.ld_os = pitch;
+    g.err = err_flag;
+    g.wait_limit_ns = moe::kDefaultWaitLimitNs;
+    e = pow2 ? moe::launch_gemm_mx(g, st) : pair ? moe::launch_gemm_pair(g, st) : moe::launch_gemm(g, st);
+  }
+  if (e == cudaSuccess) e = prof_mark(4, st);
+  if (e == cudaSuccess) {
+    // down projection, scaled by the gate of each row
+    moe::GemmLaunch g{};
+    g.w = w->w2_dev;
+    g.w_rows = E * H;
+    g.a0 = hq;
+    g.a0_rows = RS;
+    g.a1 = hq;
+    g.a1_rows = RS;
+    g.K = I;
+    g.sw = w->s2_dev;
+    g.sa0 = hs_t;
+    g.sa1 = hs_t;
+    g.sa_transposed = 1;
+    g.sa_ld = pitch;
+    g.chunks = chunks;
+    g.n_chunks = meta;
+    g.max_chunks = static_cast<int>(max_chunks);
+    g.chunk_rows = chunk_rows;
+    g.nb = moe::gemm2_blocks(H);
+    g.gate_up = 0;
+    g.a_is_out_row = 1;
+    g.rows_per_expert = H;
+    g.epi = moe::EPI_GATE_BF16;
+    g.out = y;
+    g.ldo = H;
+    g.out_rows = RS;
+    g.out_cols = H;
+    g.row_gate = row_gate;
+    g.err = err_flag;
+    g.wait_limit_ns = moe::kDefaultWaitLimitNs;
+    e = pow2 ? moe::launch_gemm_mx(g, st) : pair ? moe::launch_gemm_pair(g, st) : moe::launch_gemm(g, st);
+  }
+  if (e == cudaSuccess) e = prof_mark(5, st);
+  if (e == cudaSuccess) e = moe::launch_combine(P.x_resid, y, pos, T, H, Kr, R, Ns, P.out, P.out_f32, st);
+  if (e == cudaSuccess) e = prof_mark(6, st);
+  return e;
+}
+
 int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, const void *x, int64_t T, void *out,
                 int32_t out_dtype, int32_t *idx_out, int32_t *counts_out, void *ws, size_t ws_bytes,
                 int32_t *err_flag, void *stream) {
@@ -368,30 +523,13 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (const int d = check_device()) return d;
 
-  const int H = cfg->hidden, I = cfg->inter, Nr = cfg->n_routed, Kr = cfg->top_k, Ns = cfg->n_shared;
-  const int64_t R = T * Kr, RS = R + T * Ns;
-  const int64_t E = static_cast<int64_t>(Nr) + Ns;
+  const int H = cfg->hidden, Nr = cfg->n_routed, Kr = cfg->top_k;
   uint8_t *xq = at<uint8_t *>(ws, L.xq);
   float *xs = at<float *>(ws, L.xs);
   int32_t *idx = at<int32_t *>(ws, L.idx);
   float *gate = at<float *>(ws, L.gate);
-  int32_t *counts = at<int32_t *>(ws, L.counts);
-  int32_t *offsets = at<int32_t *>(ws, L.offsets);
-  int32_t *pos = at<int32_t *>(ws, L.pos);
-  uint8_t *ap = at<uint8_t *>(ws, L.ap);
-  float *as_t = at<float *>(ws, L.as);
-  float *row_gate = at<float *>(ws, L.row_gate);
-  int32_t *row_src = at<int32_t *>(ws, L.row_src);
-  uint8_t *hq = at<uint8_t *>(ws, L.hq);
-  float *hs_t = at<float *>(ws, L.hs);
-  float *y = at<float *>(ws, L.y);
-  int32_t *meta = at<int32_t *>(ws, L.meta);
   float *logits = at<float *>(ws, L.logits);
-  int32_t *blk_hist = at<int32_t *>(ws, L.blk_hist);
-  int32_t *blk_base = at<int32_t *>(ws, L.blk_base);
-  int4 *chunks = at<int4 *>(ws, L.chunks);
   const int ks = moe::router_ksplit(T, Nr, H);
-  const int64_t max_chunks = moe::max_chunks(T, Kr, Nr, Ns);
 
   cudaError_t e = prof_mark(0, st);
   const bool pow2 = cfg->scale_mode == MOE_SCALE_POW2;
@@ -403,85 +541,149 @@ int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, 
     e = moe::launch_router_topk(logits, ks, T, Nr, Kr, cfg->n_groups, cfg->topk_groups, cfg->route_scale, bias,
                                 idx, gate, nullptr, st);
   if (e == cudaSuccess) e = prof_mark(2, st);
-  if (e == cudaSuccess) e = moe::launch_hist(idx, T, Kr, Nr, blk_hist, err_flag, st);
-  if (e == cudaSuccess)
-    e = moe::launch_build_chunks(blk_hist, T, Kr, Nr, Ns, counts, offsets, blk_base, chunks, meta, counts_out, st);
-  if (e == cudaSuccess) e = moe::launch_rank(idx, gate, T, Kr, Nr, Ns, blk_base, row_gate, row_src, pos, st);
-  const int64_t pitch = moe::scale_pitch(R, T);
-  if (e == cudaSuccess) e = moe::launch_copy_rows(xq, xs, row_src, R, T, Ns, H, ap, as_t, pitch, st);
-  if (e == cudaSuccess) e = prof_mark(3, st);
   if (e == cudaSuccess) {
-    // gate/up projection + SwiGLU + 1x128 requantization
-    moe::GemmLaunch g{};
-    g.w = w->w13_dev;
-    g.w_rows = E * 2 * I;
-    g.a0 = ap;
-    g.a0_rows = R;
-    g.a1 = xq;
-    g.a1_rows = T;
-    g.K = H;
-    g.sw = w->s13_dev;
-    g.sa0 = as_t;
-    g.sa1 = as_t;
-    g.sa_transposed = 1;
-    g.sa_ld = pitch;
-    g.chunks = chunks;
-    g.n_chunks = meta;
-    g.max_chunks = static_cast<int>(max_chunks);
-    g.nb = moe::gemm1_blocks(I);
-    g.gate_up = 1;
-    g.half = I;
-    g.rows_per_expert = 2 * static_cast<int64_t>(I);
-    g.epi = moe::EPI_SWIGLU_Q;
-    g.out = hq;
-    g.ldo = I;
-    g.out_rows = RS;
-    g.out_cols = 2 * I;  // block B (up) shares block A's output columns
-    g.out_scale = hs_t;
-    g.ld_os = pitch;
-    g.err = err_flag;
-    g.wait_limit_ns = moe::kDefaultWaitLimitNs;
-    e = pow2 ? moe::launch_gemm_mx(g, st) : moe::launch_gemm(g, st);
+    ExpertPath P{};
+    P.cfg = cfg;
+    P.w = w;
+    P.T = T;
+    P.xq = xq;
+    P.xq_ld = H;
+    P.xs = xs;
+    P.idx = idx;
+    P.gate = gate;
+    P.allow_empty = 0;
+    P.x_resid = x;
+    P.out = out;
+    P.out_f32 = out_dtype == MOE_DTYPE_F32;
+    P.counts_out = counts_out;
+    P.L = &L;
+    P.ws = ws;
+    P.err = err_flag;
+    P.st = st;
+    e = run_expert_path(P);
   }
-  if (e == cudaSuccess) e = prof_mark(4, st);
-  if (e == cudaSuccess) {
-    // down projection, scaled by the gate of each row
-    moe::GemmLaunch g{};
-    g.w = w->w2_dev;
-    g.w_rows = E * H;
-    g.a0 = hq;
-    g.a0_rows = RS;
-    g.a1 = hq;
-    g.a1_rows = RS;
-    g.K = I;
-    g.sw = w->s2_dev;
-    g.sa0 = hs_t;
-    g.sa1 = hs_t;
-    g.sa_transposed = 1;
-    g.sa_ld = pitch;
-    g.chunks = chunks;
-    g.n_chunks = meta;
-    g.max_chunks = static_cast<int>(max_chunks);
-    g.nb = moe::gemm2_blocks(H);
-    g.gate_up = 0;
-    g.a_is_out_row = 1;
-    g.rows_per_expert = H;
-    g.epi = moe::EPI_GATE_F32;
-    g.out = y;
-    g.ldo = H;
-    g.out_rows = RS;
-    g.out_cols = H;
-    g.row_gate = row_gate;
-    g.err = err_flag;
-    g.wait_limit_ns = moe::kDefaultWaitLimitNs;
-    e = pow2 ? moe::launch_gemm_mx(g, st) : moe::launch_gemm(g, st);
-  }
-  if (e == cudaSuccess) e = prof_mark(5, st);
-  if (e == cudaSuccess) e = moe::launch_combine(x, y, pos, T, H, Kr, R, Ns, out, out_dtype == MOE_DTYPE_F32, st);
-  if (e == cudaSuccess) e = prof_mark(6, st);
   if (e == cudaSuccess && idx_out)
     e = cudaMemcpyAsync(idx_out, idx, sizeof(int32_t) * T * Kr, cudaMemcpyDeviceToDevice, st);
   return cuda_status(e);
+}
+
+// ------------------------------------------------------ expert parallelism
+int64_t moe_ep_row_bytes(const moe_config *cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  const int64_t H = cfg->hidden, Kr = cfg->top_k;
+  return (H + 4 * (H / 128) + 8 * Kr + 15) / 16 * 16;
+}
+
+static void ep_dispatch_layout(int32_t world, int64_t T, size_t *cnt_off, size_t *base_off, size_t *total) {
+  const int64_t nblk = (T + 255) / 256;
+  Carve cv;
+  size_t a[2], b[2];
+  cv.take(a, static_cast<size_t>(nblk) * world * 4);
+  cv.take(b, static_cast<size_t>(nblk) * world * 4);
+  *cnt_off = a[0];
+  *base_off = b[0];
+  *total = (cv.off + 255) & ~size_t(255);
+}
+
+size_t moe_ep_dispatch_workspace_size(const moe_config *cfg, int32_t world, int64_t T) {
+  if (check_cfg(cfg) != MOE_OK || world < 1 || world > 64 || T < 0 || T > kMaxTokens) return 0;
+  size_t c, b, tot;
+  ep_dispatch_layout(world, T, &c, &b, &tot);
+  return tot < 256 ? 256 : tot;
+}
+
+int moe_ep_dispatch(const moe_config *cfg, int32_t world, const uint8_t *xq, const float *xs, const int32_t *idx,
+                    const float *gate, int64_t T, uint8_t *send_rows, int64_t send_cap_rows, int32_t *send_counts,
+                    int32_t *send_offsets, int32_t *row_of, uint8_t *self_rows, void *ws, size_t ws_bytes,
+                    int32_t *err_flag, void *stream) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (world < 1 || world > 64 || cfg->n_routed % world) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
+  const int64_t Kr = cfg->top_k;
+  if (send_cap_rows < T * (world < Kr ? world : Kr)) return MOE_ERR_INVALID_ARG;
+  if (!send_counts || !send_offsets || !ws || !err_flag) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!xq || !xs || !idx || !gate || !send_rows || !row_of)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(send_rows) || !aligned16(self_rows) || !aligned4(xs) || !aligned4(idx) ||
+      !aligned4(gate) || !aligned4(send_counts) || !aligned4(send_offsets) || !aligned4(row_of) ||
+      !aligned4(err_flag) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_ep_dispatch_workspace_size(cfg, world, T)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (const int d = check_device()) return d;
+  size_t c_off, b_off, tot;
+  ep_dispatch_layout(world, T, &c_off, &b_off, &tot);
+  auto *w8 = static_cast<uint8_t *>(ws);
+  return cuda_status(moe::launch_ep_dispatch(
+      xq, xs, idx, gate, T, cfg->hidden, cfg->top_k, cfg->n_routed, world, reinterpret_cast<int32_t *>(w8 + c_off),
+      reinterpret_cast<int32_t *>(w8 + b_off), send_counts, send_offsets, row_of, send_rows, moe_ep_row_bytes(cfg),
+      self_rows, err_flag, static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_ep_experts_workspace_size(const moe_config *cfg_local, int64_t n_rows) {
+  if (check_cfg(cfg_local) != MOE_OK || cfg_local->n_shared != 0 || n_rows < 0 || n_rows > kMaxTokens) return 0;
+  moe_ws_layout L;
+  make_layout(cfg_local, n_rows, &L);
+  return L.total < 256 ? 256 : L.total;
+}
+
+int moe_ep_experts(const moe_config *cfg_local, const moe_weights *w_local, const uint8_t *rows, int64_t n_rows,
+                   int64_t row_bytes, void *partial_out, void *ws, size_t ws_bytes, int32_t *err_flag, void *stream) {
+  if (const int c = check_cfg(cfg_local)) return c;
+  if (cfg_local->n_shared != 0) return MOE_ERR_INVALID_ARG;
+  if (n_rows < 0 || n_rows > kMaxTokens) return MOE_ERR_INVALID_ARG;
+  if (row_bytes != moe_ep_row_bytes(cfg_local)) return MOE_ERR_INVALID_ARG;
+  if (n_rows == 0) return MOE_OK;
+  if (!w_local || !rows || !partial_out || !ws || !err_flag) return MOE_ERR_INVALID_ARG;
+  if (!w_local->w13_dev || !w_local->s13_dev || !w_local->w2_dev || !w_local->s2_dev) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(rows) || !aligned16(partial_out) || !aligned16(w_local->w13_dev) || !aligned16(w_local->w2_dev) ||
+      !aligned4(w_local->s13_dev) || !aligned4(w_local->s2_dev) || !aligned4(err_flag) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255))
+    return MOE_ERR_INVALID_ARG;
+  moe_ws_layout L;
+  make_layout(cfg_local, n_rows, &L);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (const int d = check_device()) return d;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t *idx = at<int32_t *>(ws, L.idx);
+  float *gate = at<float *>(ws, L.gate);
+  float *xs = at<float *>(ws, L.xs);
+  cudaError_t e = moe::launch_ep_unpack(rows, n_rows, row_bytes, cfg_local->hidden, cfg_local->top_k,
+                                        cfg_local->n_routed, idx, gate, xs, err_flag, st);
+  if (e == cudaSuccess) {
+    ExpertPath P{};
+    P.cfg = cfg_local;
+    P.w = w_local;
+    P.T = n_rows;
+    P.xq = rows;
+    P.xq_ld = row_bytes;
+    P.xs = xs;
+    P.idx = idx;
+    P.gate = gate;
+    P.allow_empty = 1;
+    P.x_resid = nullptr;
+    P.out = partial_out;
+    P.out_f32 = 0;
+    P.counts_out = nullptr;
+    P.L = &L;
+    P.ws = ws;
+    P.err = err_flag;
+    P.st = st;
+    e = run_expert_path(P);
+  }
+  return cuda_status(e);
+}
+
+int moe_ep_combine(const moe_config *cfg, int32_t world, const void *x, int64_t T, const int32_t *row_of,
+                   const void *back, const void *y_shared, void *out, int32_t out_dtype, void *stream) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (world < 1 || world > 64 || T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
+  if (out_dtype != MOE_DTYPE_BF16 && out_dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !row_of || !back || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(back) || !aligned16(y_shared) || !aligned16(out) || !aligned4(row_of))
+    return MOE_ERR_INVALID_ARG;
+  if (const int d = check_device()) return d;
+  return cuda_status(moe::launch_ep_combine(x, y_shared, back, row_of, T, world, cfg->hidden, out,
+                                            out_dtype == MOE_DTYPE_F32, static_cast<cudaStream_t>(stream)));
 }
 
 int moe_seq_balance_loss(const moe_config *cfg, int64_t T, int64_t seq_len, float alpha, const void *ws,

@@ -3,8 +3,8 @@
 // "DeepSeek-V3 Technischer Bericht" (xyznot.com/de), Methode section 2:
 //   h'_t = u_t + sum_{i<=N_s} FFN^(s)_i(u_t) + sum_{i<=N_r} g_{i,t} FFN^(r)_i(u_t).
 // The routed outputs arrive already multiplied by their gate (down-projection
-// epilogue), so the combine is a plain FP32 sum per token in a fixed order:
-// residual, shared expert, then the K_r slots in selection order.
+// epilogue, stored as bf16), so the combine is a plain FP32 sum per token in a
+// fixed order: residual, shared expert, then the K_r slots in selection order.
 //
 // Bias update (same section): an overloaded expert gets b_i -= gamma, an
 // underloaded one b_i += gamma, once per step.
@@ -13,50 +13,50 @@
 
 namespace moe {
 
+// bf16 x 8 (one 16-byte word) added to eight FP32 accumulators
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 &v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] += __uint_as_float(w[i] << 16);
+    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// One CTA per token, 8 channels (16-byte loads of x and of every y row) per
+// thread and step.  y rows are bf16: the gate-scaled output of each routed
+// expert, the shared expert's at row R + t.
 template <bool OUT_F32>
-__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ y,
+__global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                       const __nv_bfloat16 *__restrict__ y,
                                                        const int32_t *__restrict__ pos, int H, int Kr, int64_t R,
                                                        int Ns, void *__restrict__ out) {
   const int64_t t = blockIdx.x;
   int p[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) p[k] = (k < Kr) ? pos[t * Kr + k] : 0;
-  const int hv = H / 4;
-  const uint2 *xr = reinterpret_cast<const uint2 *>(x + t * H);
-  const float4 *ysh = reinterpret_cast<const float4 *>(y + (R + t) * H);
+  for (int k = 0; k < 16; ++k) p[k] = (k < Kr) ? pos[t * Kr + k] : -1;
+  const int hv = H / 8;
+  const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * H);
+  const uint4 *ysh = reinterpret_cast<const uint4 *>(y + (R + t) * H);
   for (int v = threadIdx.x; v < hv; v += blockDim.x) {
-    const uint2 xv = __ldg(xr + v);
-    float4 acc;
-    acc.x = __uint_as_float(xv.x << 16);
-    acc.y = __uint_as_float(xv.x & 0xFFFF0000u);
-    acc.z = __uint_as_float(xv.y << 16);
-    acc.w = __uint_as_float(xv.y & 0xFFFF0000u);
-    if (Ns) {
-      const float4 s = __ldg(ysh + v);
-      acc.x += s.x;
-      acc.y += s.y;
-      acc.z += s.z;
-      acc.w += s.w;
-    }
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (x) add_bf16x8(acc, __ldg(xr + v));  // residual u_t
+    if (Ns) add_bf16x8(acc, __ldg(ysh + v));
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      if (k < Kr && p[k] >= 0) {
-        const float4 s = __ldg(reinterpret_cast<const float4 *>(y + static_cast<int64_t>(p[k]) * H) + v);
-        acc.x += s.x;
-        acc.y += s.y;
-        acc.z += s.z;
-        acc.w += s.w;
-      }
-    }
+    for (int k = 0; k < 16; ++k)
+      if (k < Kr && p[k] >= 0) add_bf16x8(acc, __ldg(reinterpret_cast<const uint4 *>(y + static_cast<int64_t>(p[k]) * H) + v));
     if (OUT_F32) {
-      reinterpret_cast<float4 *>(static_cast<float *>(out) + t * H)[v] = acc;
+      float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + t * H) + 2 * v;
+      o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     } else {
-      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-      uint2 o;
-      o.x = *reinterpret_cast<uint32_t *>(&lo);
-      o.y = *reinterpret_cast<uint32_t *>(&hi);
-      reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(out) + t * H)[v] = o;
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t *>(&b2);
+      }
+      reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + t * H)[v] = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 }
@@ -89,15 +89,15 @@ __global__ void wait_selftest_kernel(int32_t *err, uint64_t limit_ns) {
   }
 }
 
-cudaError_t launch_combine(const void *x, const float *y, const int32_t *pos, int64_t T, int H, int Kr, int64_t R,
+cudaError_t launch_combine(const void *x, const void *y, const int32_t *pos, int64_t T, int H, int Kr, int64_t R,
                            int Ns, void *out, int out_f32, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
+  const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+  const auto *yb = static_cast<const __nv_bfloat16 *>(y);
   if (out_f32)
-    combine_kernel<true><<<static_cast<unsigned>(T), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), y, pos,
-                                                                    H, Kr, R, Ns, out);
+    combine_kernel<true><<<static_cast<unsigned>(T), 128, 0, st>>>(xb, yb, pos, H, Kr, R, Ns, out);
   else
-    combine_kernel<false><<<static_cast<unsigned>(T), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), y, pos,
-                                                                     H, Kr, R, Ns, out);
+    combine_kernel<false><<<static_cast<unsigned>(T), 128, 0, st>>>(xb, yb, pos, H, Kr, R, Ns, out);
   return cudaGetLastError();
 }
 

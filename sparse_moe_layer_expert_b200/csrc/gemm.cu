@@ -30,7 +30,7 @@
 //                 (amax of the row's two 64-channel halves exchanged between
 //                 the warpgroups, S = amax / 448, E4M3 RNE), 64 codes per
 //                 thread stored as 16-byte vectors -> hq, scale -> hs
-//   EPI_GATE_F32  y = acc * gate[row] as FP32 (down projection)
+//   EPI_GATE_BF16 y = bf16(acc * gate[row]) (down projection)
 //   EPI_BF16      C = bf16(acc) (plain GEMM)
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
@@ -359,7 +359,8 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st) {
     return cudaErrorInvalidValue;
   if (moe_host::encode_tmap_2d(&m0, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a0, K, g.a0_rows, K, 128, 128) != 0)
     return cudaErrorInvalidValue;
-  if (moe_host::encode_tmap_2d(&m1, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a1, K, g.a1_rows, K, 128, 128) != 0)
+  if (moe_host::encode_tmap_2d(&m1, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a1, K, g.a1_rows,
+                               g.a1_ld ? static_cast<uint64_t>(g.a1_ld) : K, 128, 128) != 0)
     return cudaErrorInvalidValue;
   GemmArgs a = make_args(g);
   const int sms = moe_host::sm_count();
@@ -367,7 +368,7 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st) {
   const int grid = static_cast<int>(max_tiles < sms ? max_tiles : sms);
   switch (g.epi) {
     case EPI_SWIGLU_Q: return launch_epi<EPI_SWIGLU_Q>(mw, m0, m1, a, grid, st);
-    case EPI_GATE_F32: return launch_epi<EPI_GATE_F32>(mw, m0, m1, a, grid, st);
+    case EPI_GATE_BF16: return launch_epi<EPI_GATE_BF16>(mw, m0, m1, a, grid, st);
     default: return launch_epi<EPI_BF16>(mw, m0, m1, a, grid, st);
   }
 }

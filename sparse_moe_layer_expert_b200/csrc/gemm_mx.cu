@@ -377,7 +377,7 @@ static cudaError_t launch_mx(const CUtensorMap &mw, const CUtensorMap &m0, const
 // the activation scales stored transposed (the layer's tables).
 cudaError_t launch_gemm_mx(const GemmLaunch &g, cudaStream_t st) {
   if (g.max_chunks <= 0 || g.nb <= 0) return cudaSuccess;
-  if (!g.sa_transposed || !g.chunks || (g.epi != EPI_SWIGLU_Q && g.epi != EPI_GATE_F32))
+  if (!g.sa_transposed || !g.chunks || (g.epi != EPI_SWIGLU_Q && g.epi != EPI_GATE_BF16))
     return cudaErrorInvalidValue;
   CUtensorMap mw, m0, m1;
   const uint64_t K = static_cast<uint64_t>(g.K);
@@ -385,14 +385,15 @@ cudaError_t launch_gemm_mx(const GemmLaunch &g, cudaStream_t st) {
     return cudaErrorInvalidValue;
   if (moe_host::encode_tmap_2d(&m0, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a0, K, g.a0_rows, K, 128, 128) != 0)
     return cudaErrorInvalidValue;
-  if (moe_host::encode_tmap_2d(&m1, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a1, K, g.a1_rows, K, 128, 128) != 0)
+  if (moe_host::encode_tmap_2d(&m1, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a1, K, g.a1_rows,
+                               g.a1_ld ? static_cast<uint64_t>(g.a1_ld) : K, 128, 128) != 0)
     return cudaErrorInvalidValue;
   const GemmArgs a = make_args(g);
   const int sms = moe_host::sm_count();
   const int64_t max_tiles = static_cast<int64_t>(g.max_chunks) * g.nb;
   const int grid = static_cast<int>(max_tiles < sms ? max_tiles : sms);
   return g.epi == EPI_SWIGLU_Q ? launch_mx<EPI_SWIGLU_Q>(mw, m0, m1, a, grid, st)
-                               : launch_mx<EPI_GATE_F32>(mw, m0, m1, a, grid, st);
+                               : launch_mx<EPI_GATE_BF16>(mw, m0, m1, a, grid, st);
 }
 
 }  // namespace moe

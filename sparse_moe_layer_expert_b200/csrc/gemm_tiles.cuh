@@ -15,6 +15,7 @@ struct GemmArgs {
   const int4 *chunks;        // chunk table, or null for the dense grid
   const int32_t *n_chunks;   // device count of chunks
   int max_chunks;
+  int chunk_rows;            // most activation rows per chunk: 128 (one CTA) or 256 (a CTA pair)
   int dense_chunks;
   int64_t dense_M;
   int nb;                    // weight-block pairs per chunk
@@ -54,9 +55,9 @@ __device__ __forceinline__ GemmTile get_tile(const GemmArgs &a, int t) {
   } else {
     e = 0;
     d.from1 = 0;
-    d.a_row = c * 128;
-    const int64_t rem = a.dense_M - static_cast<int64_t>(c) * 128;
-    d.n = rem < 128 ? static_cast<int32_t>(rem) : 128;
+    d.a_row = c * a.chunk_rows;
+    const int64_t rem = a.dense_M - static_cast<int64_t>(c) * a.chunk_rows;
+    d.n = rem < a.chunk_rows ? static_cast<int32_t>(rem) : a.chunk_rows;
     d.out_row = d.a_row;
   }
   if (a.a_is_out_row) {
@@ -82,7 +83,7 @@ __device__ __forceinline__ GemmTile get_tile(const GemmArgs &a, int t) {
 __device__ __forceinline__ bool tile_ok(const GemmArgs &a, const GemmTile &d) {
   const int64_t arows = d.from1 ? a.a_rows1 : a.a_rows0;
   const bool two = d.w_row1 >= 0;
-  return d.n >= 1 && d.n <= 128 && d.a_row >= 0 && d.a_row + d.n <= arows && d.out_row >= 0 &&
+  return d.n >= 1 && d.n <= a.chunk_rows && d.a_row >= 0 && d.a_row + d.n <= arows && d.out_row >= 0 &&
          d.out_row + d.n <= a.out_rows && d.w_row0 >= 0 && d.w_row0 + 128 <= a.w_rows &&
          (!two || d.w_row1 + 128 <= a.w_rows) && d.out_col >= 0 && d.out_col + (two ? 256 : 128) <= a.out_cols &&
          (!a.sa_transposed || d.out_row + d.n <= a.sa_ld) && a.KB <= G_KBMAX;
@@ -97,7 +98,8 @@ __device__ __forceinline__ bool tile_ok(const GemmArgs &a, const GemmTile &d) {
 //                 the warpgroups through amx; S = amax / 448, or the power-of-
 //                 two scale when POW2; E4M3 RNE), 64 codes per thread stored
 //                 as 16-byte vectors -> hq, scale -> hs
-//   EPI_GATE_F32  y = acc * gate[row] as FP32 (down projection)
+//   EPI_GATE_BF16 y = bf16(acc * gate[row]) (down projection; the product in
+//                 FP32, rounded to nearest even)
 //   EPI_BF16      C = bf16(acc) (plain GEMM)
 // Both warpgroups take the named barrier 1 (256 threads) twice per tile in
 // EPI_SWIGLU_Q.
@@ -161,30 +163,23 @@ __device__ __forceinline__ void tile_epilogue(const GemmArgs &args, const GemmTi
     // contiguous bytes instead of 32 scattered rows.
     float *xb = outx + (warp - 4) * (32 * G_OPITCH);
     const int rbase = q * 32;  // this warp's first row in the tile
-    const float g = (EPI == EPI_GATE_F32 && valid) ? __ldg(args.row_gate + orow) : 1.0f;
+    const float g = (EPI == EPI_GATE_BF16 && valid) ? __ldg(args.row_gate + orow) : 1.0f;
     auto emit = [&](const float(&acc)[64], int b) {
 #pragma unroll
-      for (int piece = 0; piece < (EPI == EPI_GATE_F32 ? 4 : 2); ++piece) {
-        // stage: this thread's 16 floats (or 32 bf16) of the piece, row = lane
+      for (int piece = 0; piece < 2; ++piece) {
+        // stage: this thread's 32 bf16 of the piece, row = lane
         float4 *dst = reinterpret_cast<float4 *>(xb + lane * G_OPITCH);
-        if constexpr (EPI == EPI_GATE_F32) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int j = piece * 16 + 4 * v;
-            dst[v] = make_float4(acc[j] * g, acc[j + 1] * g, acc[j + 2] * g, acc[j + 3] * g);
+        for (int v = 0; v < 4; ++v) {
+          float f[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int j = piece * 32 + 8 * v + 2 * k;
+            const __nv_bfloat162 b2 = EPI == EPI_GATE_BF16 ? __floats2bfloat162_rn(acc[j] * g, acc[j + 1] * g)
+                                                           : __floats2bfloat162_rn(acc[j], acc[j + 1]);
+            f[k] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&b2));
           }
-        } else {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            float f[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int j = piece * 32 + 8 * v + 2 * k;
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[j], acc[j + 1]);
-              f[k] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&b2));
-            }
-            dst[v] = make_float4(f[0], f[1], f[2], f[3]);
-          }
+          dst[v] = make_float4(f[0], f[1], f[2], f[3]);
         }
         __syncwarp();
         // drain: lane L stores 16 bytes of row (L / 4 + 8 s), chunk L % 4
@@ -194,14 +189,9 @@ __device__ __forceinline__ void tile_epilogue(const GemmArgs &args, const GemmTi
           if (rbase + rr < td.n) {
             const float4 val = reinterpret_cast<const float4 *>(xb + rr * G_OPITCH)[lane & 3];
             const int64_t grow = static_cast<int64_t>(td.out_row) + rbase + rr;
-            if constexpr (EPI == EPI_GATE_F32) {
-              float *yrow = static_cast<float *>(args.out) + grow * args.ldo + c0 + 128 * b + piece * 16;
-              reinterpret_cast<float4 *>(yrow)[lane & 3] = val;
-            } else {
-              __nv_bfloat16 *crow =
-                  static_cast<__nv_bfloat16 *>(args.out) + grow * args.ldo + c0 + 128 * b + piece * 32;
-              reinterpret_cast<float4 *>(crow)[lane & 3] = val;
-            }
+            __nv_bfloat16 *crow =
+                static_cast<__nv_bfloat16 *>(args.out) + grow * args.ldo + c0 + 128 * b + piece * 32;
+            reinterpret_cast<float4 *>(crow)[lane & 3] = val;
           }
         }
         __syncwarp();
@@ -219,7 +209,8 @@ inline GemmArgs make_args(const GemmLaunch &g) {
   a.n_chunks = g.n_chunks;
   a.max_chunks = g.max_chunks;
   a.dense_M = g.dense_M;
-  a.dense_chunks = g.chunks ? 0 : static_cast<int>((g.dense_M + 127) / 128);
+  a.chunk_rows = g.chunk_rows == 256 ? 256 : 128;
+  a.dense_chunks = g.chunks ? 0 : static_cast<int>((g.dense_M + a.chunk_rows - 1) / a.chunk_rows);
   a.nb = g.nb;
   a.gate_up = g.gate_up;
   a.a_is_out_row = g.a_is_out_row;

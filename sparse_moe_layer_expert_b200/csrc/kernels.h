@@ -31,14 +31,14 @@ struct GemmTile {
   int32_t w_row0;   // first row of weight block A in the weight tensor
   int32_t w_row1;   // first row of weight block B, or -1
   int32_t a_row;    // first activation row (in the tensor map the tile reads)
-  int32_t n;        // activation rows in this tile, 1..128
+  int32_t n;        // activation rows in this tile, 1..128 (one CTA) or 1..256 (a CTA pair)
   int32_t out_row;  // first output row (also the column of the transposed scales)
   int32_t out_col;  // first output column of block A's outputs
   int32_t from1;    // activations come from the second tensor map
   int32_t pad;
 };
 
-enum EpiKind : int { EPI_SWIGLU_Q = 0, EPI_GATE_F32 = 1, EPI_BF16 = 2 };
+enum EpiKind : int { EPI_SWIGLU_Q = 0, EPI_GATE_BF16 = 1, EPI_BF16 = 2 };
 
 struct GemmLaunch {
   // tensor operands
@@ -48,6 +48,7 @@ struct GemmLaunch {
   int64_t a0_rows;
   const uint8_t *a1;      // second activation tensor (may equal a0)
   int64_t a1_rows;
+  int64_t a1_ld;          // bytes between a1 rows (0: K); a multiple of 16
   int64_t K;
   const float *sw;        // weight scales [w_rows/128, K/128]
   const float *sa0;       // activation scales [a0_rows, K/128]
@@ -57,6 +58,7 @@ struct GemmLaunch {
   const int4 *chunks;
   const int32_t *n_chunks;
   int max_chunks;          // host-side upper bound (grid sizing)
+  int chunk_rows;          // most rows per chunk: 128 (one CTA per tile) or 256 (a CTA pair per tile)
   int64_t dense_M;
   int nb;                  // weight-block pairs per chunk
   int gate_up;             // pair block j with block j + half (SwiGLU) instead of 2j, 2j+1
@@ -99,15 +101,15 @@ cudaError_t launch_router_topk(const float *partial, int n_ks, int64_t T, int Nr
 cudaError_t launch_seq_balance(const float *partial, int n_ks, int64_t T, int Nr, const int32_t *idx, int Kr,
                                int64_t seq_len, float alpha, float *loss, int32_t *err, cudaStream_t st);
 
-cudaError_t launch_hist(const int32_t *idx, int64_t T, int Kr, int Nr, int32_t *blk_hist, int32_t *err,
-                        cudaStream_t st);
-cudaError_t launch_build_chunks(const int32_t *blk_hist, int64_t T, int Kr, int Nr, int Ns, int32_t *counts,
-                                int32_t *offsets, int32_t *blk_base, int4 *chunks, int32_t *meta,
+cudaError_t launch_hist(const int32_t *idx, int64_t T, int Kr, int Nr, int allow_empty, int32_t *blk_hist,
+                        int32_t *err, cudaStream_t st);
+cudaError_t launch_build_chunks(const int32_t *blk_hist, int64_t T, int Kr, int Nr, int Ns, int chunk_rows,
+                                int32_t *counts, int32_t *offsets, int32_t *blk_base, int4 *chunks, int32_t *meta,
                                 int32_t *counts_out, cudaStream_t st);
 cudaError_t launch_rank(const int32_t *idx, const float *gate, int64_t T, int Kr, int Nr, int Ns,
                         const int32_t *blk_base, float *row_gate, int32_t *row_src, int32_t *pos, cudaStream_t st);
-cudaError_t launch_copy_rows(const uint8_t *xq, const float *xs, const int32_t *row_src, int64_t R, int64_t T,
-                             int Ns, int H, uint8_t *ap, float *as_t, int64_t ld, cudaStream_t st);
+cudaError_t launch_copy_rows(const uint8_t *xq, int64_t xq_ld, const float *xs, const int32_t *row_src, int64_t R,
+                             int64_t T, int Ns, int H, uint8_t *ap, float *as_t, int64_t ld, cudaStream_t st);
 // Row pitch of the transposed scale tables [K/128][pitch]: R + T rounded up to
 // 4 floats (16-byte aligned rows for bulk copies); the tables carry
 // kScaleSlack floats after their last row so a 132-float copy stays in bounds.
@@ -115,13 +117,31 @@ inline int64_t scale_pitch(int64_t R, int64_t T) { return (R + T + 3) / 4 * 4; }
 constexpr int64_t kScaleSlack = 132;
 
 cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st);
+// The same GEMM on CTA pairs (clusters of two): chunk_rows = 256, one
+// tcgen05.mma.cta_group::2 per 32-long K step over both CTAs' tiles; the
+// weight-block count per expert must be even (always true for gate/up).
+cudaError_t launch_gemm_pair(const GemmLaunch &g, cudaStream_t st);
 // The same grouped GEMM with power-of-two scales applied by the tensor core
 // (block-scaled MMA); transposed activation scales, EPI_SWIGLU_Q (with
-// power-of-two requantization) or EPI_GATE_F32 only.
+// power-of-two requantization) or EPI_GATE_BF16 only.
 cudaError_t launch_gemm_mx(const GemmLaunch &g, cudaStream_t st);
 
-cudaError_t launch_combine(const void *x, const float *y, const int32_t *pos, int64_t T, int H, int Kr,
+// out[t] = x[t] (when x is not null) + y[R + t] (when Ns) + sum_k y[pos[t, k]]
+// (pos >= 0), FP32 in that order, written as FP32 or bf16 (RNE)
+cudaError_t launch_combine(const void *x, const void *y, const int32_t *pos, int64_t T, int H, int Kr,
                            int64_t R, int Ns, void *out, int out_f32, cudaStream_t st);
+// Expert parallelism (ep.cu): dispatch of one rank's routed tokens into a
+// send buffer ordered by destination, the receiving side's unpacking of the
+// packed rows, and the sending side's combine of the returned partial sums.
+cudaError_t launch_ep_dispatch(const uint8_t *xq, const float *xs, const int32_t *idx, const float *gate, int64_t T,
+                               int H, int Kr, int Nr, int W, int32_t *blk_cnt, int32_t *blk_base,
+                               int32_t *send_counts, int32_t *send_off, int32_t *row_of, uint8_t *send,
+                               int64_t row_bytes, uint8_t *self_rows, int32_t *err, cudaStream_t st);
+cudaError_t launch_ep_unpack(const uint8_t *rows, int64_t n, int64_t row_bytes, int H, int Kr, int n_local,
+                             int32_t *idx, float *gate, float *xs, int32_t *err, cudaStream_t st);
+cudaError_t launch_ep_combine(const void *x, const void *y_sh, const void *back, const int32_t *row_of, int64_t T,
+                              int W, int H, void *out, int out_f32, cudaStream_t st);
+
 cudaError_t launch_bias_update(float *bias, const int32_t *counts, int Nr, int64_t total, float gamma,
                                cudaStream_t st);
 cudaError_t launch_wait_selftest(int32_t *err, uint64_t limit_ns, cudaStream_t st);

@@ -10,10 +10,12 @@
 //
 //  hist_kernel         per 128-token block, per-expert counts
 //  build_chunks_kernel one CTA: totals, exclusive scans, per-block bases and
-//                      the chunk table (<= 128 rows of one expert per chunk)
-//                      from which both grouped GEMMs derive their tiles
-//  rank_kernel         per 128-token block: stable ranks (warp match) ->
-//                      row of every (token, slot), per-row gate and source
+//                      the chunk table (<= 128 or <= 256 rows of one expert
+//                      per chunk, for one CTA or a CTA pair per tile) from
+//                      which both grouped GEMMs derive their tiles
+//  rank_kernel         per 128-token block: stable ranks (warp matches over
+//                      8 ranges of the block) -> row of every (token, slot),
+//                      per-row gate and source
 //  copy_rows_kernel    one warp per row: FP8 row copy (16-byte vectors) and
 //                      the row's scales into the transposed scale table
 #include "common.cuh"
@@ -23,8 +25,12 @@ namespace moe {
 
 constexpr int kTokBlock = 128;
 
+// idx entries of -1 mean "no expert in this slot" when allow_empty is set
+// (rows received by an expert-parallel rank list only the slots whose expert
+// lives there); any other value outside [0, Nr) is reported.
 __global__ void __launch_bounds__(256) hist_kernel(const int32_t *__restrict__ idx, int64_t T, int Kr, int Nr,
-                                                    int32_t *__restrict__ blk_hist, int32_t *__restrict__ err) {
+                                                    int allow_empty, int32_t *__restrict__ blk_hist,
+                                                    int32_t *__restrict__ err) {
   __shared__ int h[256];
   for (int e = threadIdx.x; e < Nr; e += blockDim.x) h[e] = 0;
   __syncthreads();
@@ -36,7 +42,7 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t *__restrict__ i
     const int e = idx[t0 * Kr + a];
     if (e >= 0 && e < Nr)
       atomicAdd(&h[e], 1);
-    else
+    else if (!(allow_empty && e == -1))
       bad = true;
   }
   if (bad && err) atomicOr(err, MOE_DEVERR_BAD_INDEX);
@@ -68,9 +74,9 @@ __device__ int block_excl_scan(int v, int *total) {
 
 // Chunk table entry: {expert | from_input << 16, activation row, output row, rows}.
 __global__ void __launch_bounds__(256) build_chunks_kernel(const int32_t *__restrict__ blk_hist, int64_t T, int Kr,
-                                                            int Nr, int Ns, int32_t *counts, int32_t *offsets,
-                                                            int32_t *blk_base, int4 *chunks, int32_t *meta,
-                                                            int32_t *counts_out) {
+                                                            int Nr, int Ns, int chunk_rows, int32_t *counts,
+                                                            int32_t *offsets, int32_t *blk_base, int4 *chunks,
+                                                            int32_t *meta, int32_t *counts_out) {
   const int e = threadIdx.x;
   const int nblk = static_cast<int>((T + kTokBlock - 1) / kTokBlock);
   const int64_t R = T * Kr;
@@ -79,7 +85,7 @@ __global__ void __launch_bounds__(256) build_chunks_kernel(const int32_t *__rest
     for (int b = 0; b < nblk; ++b) cnt += blk_hist[static_cast<int64_t>(b) * Nr + e];
   int total_rows;
   const int off = block_excl_scan(cnt, &total_rows);
-  const int nch = (cnt + 127) / 128;
+  const int nch = (cnt + chunk_rows - 1) / chunk_rows;
   int total_chunks;
   const int cbase = block_excl_scan(nch, &total_chunks);
   if (e < Nr) {
@@ -93,14 +99,15 @@ __global__ void __launch_bounds__(256) build_chunks_kernel(const int32_t *__rest
       run += blk_hist[static_cast<int64_t>(b) * Nr + e];
     }
   }
-  // shared-expert chunks first (full 128-row chunks: largest work first)
-  const int sh_chunks = Ns ? static_cast<int>((T + 127) / 128) : 0;
+  // shared-expert chunks first (full chunks: largest work first)
+  const int sh_chunks = Ns ? static_cast<int>((T + chunk_rows - 1) / chunk_rows) : 0;
   for (int c = threadIdx.x; c < sh_chunks; c += blockDim.x) {
-    const int n = static_cast<int>((T - c * 128) < 128 ? (T - c * 128) : 128);
-    chunks[c] = make_int4(Nr | (1 << 16), c * 128, static_cast<int>(R) + c * 128, n);
+    const int64_t r0 = static_cast<int64_t>(c) * chunk_rows;
+    const int n = static_cast<int>((T - r0) < chunk_rows ? (T - r0) : chunk_rows);
+    chunks[c] = make_int4(Nr | (1 << 16), static_cast<int>(r0), static_cast<int>(R + r0), n);
   }
   if (e < Nr && nch > 0) {
-    const int sz = (cnt + nch - 1) / nch;  // <= 128: rows split evenly over the chunks
+    const int sz = (cnt + nch - 1) / nch;  // <= chunk_rows: rows split evenly over the chunks
     for (int c = 0; c < nch; ++c) {
       const int r0 = off + c * sz;
       const int n = (cnt - c * sz) < sz ? (cnt - c * sz) : sz;
@@ -113,12 +120,19 @@ __global__ void __launch_bounds__(256) build_chunks_kernel(const int32_t *__rest
   }
 }
 
+// Stable ranks of one 128-token block's assignments.  The block's A = nt*K_r
+// assignments (row-major (token, slot) order) are cut into 8 contiguous
+// ranges, one per warp: pass 1 counts each expert per range, the per-expert
+// counts of the earlier ranges give each range its starting rank, and pass 2
+// ranks within the range with warp matches -- the order is the same as one
+// sequential walk over the block, with an eighth of its dependent steps.
 __global__ void __launch_bounds__(256) rank_kernel(const int32_t *__restrict__ idx, const float *__restrict__ gate,
                                                     int64_t T, int Kr, int Nr, int Ns,
                                                     const int32_t *__restrict__ blk_base,
                                                     float *__restrict__ row_gate, int32_t *__restrict__ row_src,
                                                     int32_t *__restrict__ pos) {
-  __shared__ int s_cnt[256];
+  constexpr int W = 8;
+  __shared__ int s_cnt[W][256];   // pass 1: per range counts; then per range running ranks
   __shared__ int s_pos[kTokBlock * 16];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int b = blockIdx.x;
@@ -126,23 +140,44 @@ __global__ void __launch_bounds__(256) rank_kernel(const int32_t *__restrict__ i
   const int nt = static_cast<int>((T - t0) < kTokBlock ? (T - t0) : kTokBlock);
   const int na = nt * Kr;
   const int64_t R = T * Kr;
-  for (int e = threadIdx.x; e < Nr; e += blockDim.x) s_cnt[e] = 0;
+  const int per = (na + W - 1) / W;
+  const int a0 = warp * per, a1 = (a0 + per) < na ? (a0 + per) : na;
+  for (int i = threadIdx.x; i < W * 256; i += blockDim.x) (&s_cnt[0][0])[i] = 0;
   __syncthreads();
-  if (warp == 0) {
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    for (int base = 0; base < na; base += 32) {
-      const int a = base + lane;
-      const bool valid = a < na;
-      int e = valid ? idx[t0 * Kr + a] : -1;
-      if (e < 0 || e >= Nr) e = -1;
-      const uint32_t peers = __match_any_sync(0xffffffffu, e);
-      const int rank = __popc(peers & lt_mask);
-      const int prior = (e >= 0) ? s_cnt[e] : 0;
-      __syncwarp();
-      if (e >= 0 && rank == 0) s_cnt[e] = prior + __popc(peers);
-      __syncwarp();
-      if (valid) s_pos[a] = (e >= 0) ? blk_base[static_cast<int64_t>(b) * Nr + e] + prior + rank : -1;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  // pass 1: counts per expert in this warp's range
+  for (int base = a0; base < a1; base += 32) {
+    const int a = base + lane;
+    int e = a < a1 ? idx[t0 * Kr + a] : -1;
+    if (e < 0 || e >= Nr) e = -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && __popc(peers & lt_mask) == 0) s_cnt[warp][e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // exclusive prefix over the ranges, per expert, plus the block's base row
+  for (int e = threadIdx.x; e < Nr; e += blockDim.x) {
+    int run = blk_base[static_cast<int64_t>(b) * Nr + e];
+    for (int w = 0; w < W; ++w) {
+      const int c = s_cnt[w][e];
+      s_cnt[w][e] = run;
+      run += c;
     }
+  }
+  __syncthreads();
+  // pass 2: ranks inside the range
+  for (int base = a0; base < a1; base += 32) {
+    const int a = base + lane;
+    const bool valid = a < a1;
+    int e = valid ? idx[t0 * Kr + a] : -1;
+    if (e < 0 || e >= Nr) e = -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt_mask);
+    const int prior = (e >= 0) ? s_cnt[warp][e] : 0;
+    __syncwarp();
+    if (e >= 0 && rank == 0) s_cnt[warp][e] = prior + __popc(peers);
+    __syncwarp();
+    if (valid) s_pos[a] = (e >= 0) ? prior + rank : -1;
   }
   __syncthreads();
   for (int a = threadIdx.x; a < na; a += blockDim.x) {
@@ -157,11 +192,13 @@ __global__ void __launch_bounds__(256) rank_kernel(const int32_t *__restrict__ i
     for (int i = threadIdx.x; i < nt; i += blockDim.x) row_gate[R + t0 + i] = 1.0f;
 }
 
-// Rows [0, R): routed rows, copied from the quantized input row row_src[p];
+// Rows [0, R): routed rows, copied from the quantized input row row_src[p]
+// (xq rows xq_ld bytes apart, 16-byte aligned);
 // rows [R, R + T): the shared expert's rows (token p - R), scales only (the
 // gate/up GEMM reads their codes from the quantized input directly).
 // Scales go to the transposed table as_t[kb * ld + p].
-__global__ void __launch_bounds__(256) copy_rows_kernel(const uint8_t *__restrict__ xq, const float *__restrict__ xs,
+__global__ void __launch_bounds__(256) copy_rows_kernel(const uint8_t *__restrict__ xq, int64_t xq_ld,
+                                                         const float *__restrict__ xs,
                                                          const int32_t *__restrict__ row_src, int64_t R, int64_t T,
                                                          int Ns, int H, uint8_t *__restrict__ ap,
                                                          float *__restrict__ as_t, int64_t ld) {
@@ -174,7 +211,7 @@ __global__ void __launch_bounds__(256) copy_rows_kernel(const uint8_t *__restric
   if (p < R) {
     t = row_src[p];
     if (t < 0 || t >= T) return;
-    const uint4 *src = reinterpret_cast<const uint4 *>(xq + t * H);
+    const uint4 *src = reinterpret_cast<const uint4 *>(xq + t * xq_ld);
     uint4 *dst = reinterpret_cast<uint4 *>(ap + p * H);
     for (int i = lane; i < hv; i += 32) dst[i] = __ldg(src + i);
   } else {
@@ -183,19 +220,19 @@ __global__ void __launch_bounds__(256) copy_rows_kernel(const uint8_t *__restric
   for (int i = lane; i < kb; i += 32) as_t[i * ld + p] = __ldg(xs + t * kb + i);
 }
 
-cudaError_t launch_hist(const int32_t *idx, int64_t T, int Kr, int Nr, int32_t *blk_hist, int32_t *err,
-                        cudaStream_t st) {
+cudaError_t launch_hist(const int32_t *idx, int64_t T, int Kr, int Nr, int allow_empty, int32_t *blk_hist,
+                        int32_t *err, cudaStream_t st) {
   const int64_t nblk = (T + kTokBlock - 1) / kTokBlock;
   if (nblk == 0) return cudaSuccess;
-  hist_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(idx, T, Kr, Nr, blk_hist, err);
+  hist_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(idx, T, Kr, Nr, allow_empty, blk_hist, err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_build_chunks(const int32_t *blk_hist, int64_t T, int Kr, int Nr, int Ns, int32_t *counts,
-                                int32_t *offsets, int32_t *blk_base, int4 *chunks, int32_t *meta,
+cudaError_t launch_build_chunks(const int32_t *blk_hist, int64_t T, int Kr, int Nr, int Ns, int chunk_rows,
+                                int32_t *counts, int32_t *offsets, int32_t *blk_base, int4 *chunks, int32_t *meta,
                                 int32_t *counts_out, cudaStream_t st) {
-  build_chunks_kernel<<<1, 256, 0, st>>>(blk_hist, T, Kr, Nr, Ns, counts, offsets, blk_base, chunks, meta,
-                                         counts_out);
+  build_chunks_kernel<<<1, 256, 0, st>>>(blk_hist, T, Kr, Nr, Ns, chunk_rows, counts, offsets, blk_base, chunks,
+                                         meta, counts_out);
   return cudaGetLastError();
 }
 
@@ -208,12 +245,13 @@ cudaError_t launch_rank(const int32_t *idx, const float *gate, int64_t T, int Kr
   return cudaGetLastError();
 }
 
-cudaError_t launch_copy_rows(const uint8_t *xq, const float *xs, const int32_t *row_src, int64_t R, int64_t T,
-                             int Ns, int H, uint8_t *ap, float *as_t, int64_t ld, cudaStream_t st) {
+cudaError_t launch_copy_rows(const uint8_t *xq, int64_t xq_ld, const float *xs, const int32_t *row_src, int64_t R,
+                             int64_t T, int Ns, int H, uint8_t *ap, float *as_t, int64_t ld, cudaStream_t st) {
   const int64_t rows = R + (Ns ? T : 0);
   if (rows == 0) return cudaSuccess;
   const int64_t blocks = (rows + 7) / 8;
-  copy_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(xq, xs, row_src, R, T, Ns, H, ap, as_t, ld);
+  copy_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(xq, xq_ld, xs, row_src, R, T, Ns, H, ap, as_t,
+                                                                   ld);
   return cudaGetLastError();
 }
 

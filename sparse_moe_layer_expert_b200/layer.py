@@ -55,6 +55,20 @@ class MoeLayer:
         layer.set_router(wr, bias)
         return layer
 
+    def sibling(self, bias: torch.Tensor | None = None, **shape_overrides) -> "MoeLayer":
+        """A layer on the same device-resident weights with another routing
+        configuration (e.g. n_groups, topk_groups) and bias; nothing is
+        copied."""
+        other = object.__new__(MoeLayer)
+        other.shape = dict(self.shape, **shape_overrides)
+        other.cfg = B.config_from(other.shape)
+        other.E, other.device = self.E, self.device
+        other.w13, other.s13, other.w2, other.s2, other.wr = self.w13, self.s13, self.w2, self.s2, self.wr
+        other.bias = self.bias.clone() if bias is None else bias
+        other.err = B.new_err_flag(self.device)
+        other._ws = {}
+        return other
+
     def weights(self) -> dict:
         return dict(w13=self.w13, s13=self.s13, w2=self.w2, s2=self.s2, wr=self.wr)
 

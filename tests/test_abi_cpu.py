@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported(m):
 
 
 def test_status_strings_and_version(m):
-    assert m.lib.moe_abi_version() == 102
+    assert m.lib.moe_abi_version() == 103
     assert m.lib.moe_status_string(0) == b"ok"
     assert b"128" in m.lib.moe_status_string(m.MOE_ERR_UNSUPPORTED_SHAPE)
     assert m.lib.moe_status_string(12345) == b"unknown status"
@@ -63,6 +63,14 @@ def test_host_validation_without_device(m):
     assert m.moe_workspace_size(m.config(512, 256, 16, 4, 1, 8, 4), 8) > 0
     # a valid call with non-null pointers reaches the device check
     assert L.fp8_quant_1x128(16, 4, 128, 128, 16, 16, None) == m.MOE_ERR_NO_DEVICE
+
+
+def test_gemm_variant_switch(m):
+    L = m.lib
+    for v in (m.MOE_GEMM_SINGLE, m.MOE_GEMM_PAIR, m.MOE_GEMM_AUTO):
+        assert L.moe_set_gemm_variant(v) == m.MOE_OK
+    assert L.moe_set_gemm_variant(3) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_set_gemm_variant(-1) == m.MOE_ERR_INVALID_ARG
 
 
 def test_contraction_and_alignment_limits_without_device(m):
@@ -106,7 +114,7 @@ def test_workspace_layout_is_disjoint_and_aligned(m):
             assert o1 + n1 <= o2
         assert spans[-1][0] + spans[-1][1] <= L["total"] == m.moe_workspace_size(cfg, T)
         R = T * Kr
-        assert L["ap"][1] == R * H and L["y"][1] == (R + T) * H * 4 and L["hq"][1] == (R + T) * I
+        assert L["ap"][1] == R * H and L["y"][1] == (R + T) * H * 2 and L["hq"][1] == (R + T) * I
 
 
 def test_route_workspace_size(m):

@@ -1,8 +1,11 @@
 """Full-size parity: the DeepSeek-V3-shaped layer (hidden 7168, intermediate
 2048, 256 routed + 1 shared experts, top-8) in the launch configuration the
 benchmark times.  Quantization, routing, counts, grouping and weights are
-checked over the whole batch; the expert FFNs and the layer output on a seeded
-sample of tokens the double-precision oracle computes one by one."""
+checked over the whole batch; the expert FFNs and the layer output on tokens
+the double-precision oracle computes one by one: all 64 decode tokens, and at
+prefill and skewed sizes at least 64 tokens chosen so that their rows reach
+all four TMEM lane quarters (of both CTAs where tiles run on CTA pairs) and
+the most loaded expert (pick_tokens)."""
 import numpy as np
 import pytest
 import torch
@@ -38,6 +41,47 @@ def v3_layer(m):
     return layer, seed
 
 
+def pick_tokens(m, layer, prob, n: int, seed: int) -> np.ndarray:
+    """Tokens for the per-token FFN comparison, chosen so that their rows
+    reach every part of the grouped GEMMs' tiles.  From the chunk table the
+    forward leaves in its workspace (each chunk: one expert's rows, up to 128
+    per CTA; on CTA pairs up to 256, rows 128.. on the odd CTA): rows in each
+    of the four 32-row TMEM lane quarters of each CTA position, routed and
+    shared; rows of the most loaded expert; the first and the last token;
+    then seeded random tokens up to n."""
+    T, Kr, Nr = prob.T, prob.cfg["Kr"], prob.cfg["Nr"]
+    layer.forward(prob.x)
+    layer.check()
+    ws, L = layer.workspace(T), layer.layout(T)
+    idx = m.ws_view(ws, L, "idx", torch.int32, (T, Kr)).cpu().numpy()
+    pos = m.ws_view(ws, L, "pos", torch.int32, (T, Kr)).cpu().numpy()
+    off = m.ws_view(ws, L, "offsets", torch.int32, (Nr + 1,)).cpu().numpy()
+    nch = int(m.ws_view(ws, L, "meta", torch.int32, (4,)).cpu().numpy()[0])
+    chunks = m.ws_view(ws, L, "chunks", torch.int32, (nch, 4)).cpu().numpy()
+    R = T * Kr
+    token_of_row = np.empty(R + T, np.int64)
+    token_of_row[pos.reshape(-1)] = np.repeat(np.arange(T), Kr)
+    token_of_row[R:] = np.arange(T)
+    want = {}
+    for _, _, out_row, rows in chunks:
+        for r in range(rows):
+            row = out_row + r
+            key = ("shared" if row >= R else "routed", r >= 128, (r % 128) // 32)
+            want.setdefault(key, []).append(int(token_of_row[row]))
+    rng = np.random.default_rng(seed)
+    chosen = {0, T - 1}
+    for key in sorted(want):
+        cand = want[key]
+        chosen.update(int(c) for c in rng.choice(cand, min(2, len(cand)), replace=False))
+    hot = int(np.argmax(np.diff(off)))
+    hot_tokens = np.nonzero((idx == hot).any(axis=1))[0]
+    chosen.update(int(c) for c in rng.choice(hot_tokens, min(4, len(hot_tokens)), replace=False))
+    rest = np.setdiff1d(np.arange(T), np.array(sorted(chosen)))
+    extra = max(0, n - len(chosen))
+    chosen.update(int(c) for c in rng.choice(rest, min(extra, len(rest)), replace=False))
+    return np.array(sorted(chosen))
+
+
 def _problem(cfg, T, seed, layer, bias_kind):
     prob = Problem(cfg, T, seed=seed, device="cuda")
     # the layer's weights and router come from seed 0; only x differs per test
@@ -54,15 +98,16 @@ def _problem(cfg, T, seed, layer, bias_kind):
 def test_v3_decode_layer(m, oracle_lib, v3_layer):
     layer, _ = v3_layer
     prob = _problem(dict(S.DECODE), 64, 11, layer, "zero")
-    r = check_layer(m, oracle_lib, prob, layer, tokens=np.array([0, 9, 31, 63]), check_weights=True)
+    # every token of the batch
+    r = check_layer(m, oracle_lib, prob, layer, tokens=np.arange(64), check_weights=True)
     assert r["counts"].sum() == 64 * 8
 
 
 def test_v3_prefill_layer(m, oracle_lib, v3_layer):
     layer, _ = v3_layer
     prob = _problem(dict(S.PREFILL), 4096, 12, layer, "uniform")
-    rng = np.random.default_rng(12)
-    toks = np.sort(rng.choice(4096, 4, replace=False))
+    toks = pick_tokens(m, layer, prob, 64, 12)
+    assert len(toks) >= 64
     r = check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=False)
     c = r["counts"]
     print(f"prefill load: max {c.max()} mean {c.mean():.1f} min {c.min()} empty {(c == 0).sum()}")
@@ -88,8 +133,8 @@ def test_v3_skewed_layer(m, oracle_lib, v3_layer):
     prob.wr = base.wr
     prob.bias = torch.zeros(cfg["Nr"], dtype=torch.float32, device="cuda")
     layer.set_router(prob.wr, prob.bias)
-    rng = np.random.default_rng(13)
-    toks = np.sort(rng.choice(T, 4, replace=False))
+    toks = pick_tokens(m, layer, prob, 64, 13)
+    assert len(toks) >= 64
     r = check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=False)
     c = r["counts"]
     print(f"skewed load: max {c.max()} mean {c.mean():.1f} max/mean {c.max() / c.mean():.2f}")
@@ -120,7 +165,7 @@ def test_v3_prefill_layer_pow2(m, oracle_lib, v3_layer_pow2):
     layer, _ = v3_layer_pow2
     prob = _problem(dict(S.PREFILL, scale_mode=1), 4096, 12, layer, "uniform")
     rng = np.random.default_rng(14)
-    toks = np.sort(rng.choice(4096, 4, replace=False))
+    toks = np.sort(rng.choice(4096, 16, replace=False))
     check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=True)
 
 
@@ -146,7 +191,7 @@ def test_v3_skewed_layer_pow2(m, oracle_lib, v3_layer_pow2):
     prob.bias = torch.zeros(cfg["Nr"], dtype=torch.float32, device="cuda")
     layer.set_router(prob.wr, prob.bias)
     rng = np.random.default_rng(15)
-    toks = np.sort(rng.choice(T, 4, replace=False))
+    toks = np.sort(rng.choice(T, 16, replace=False))
     r = check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=False)
     c = r["counts"]
     assert c.max() >= 4 * c.mean()
