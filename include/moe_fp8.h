@@ -300,6 +300,47 @@ MOE_API int moe_workspace_layout(const moe_config *cfg, int64_t T, moe_ws_layout
 enum { MOE_PROFILE_EVENTS = 7 };
 MOE_API int moe_profile_events(void *const *events, int32_t n_events);
 
+/* ------------------------------------------------------------ backward */
+/* Backward of the layer's expert FFNs with the routing held fixed ([P4]
+ * Kernideen, FP8 bullet: "E4M3 for all tensors"; the tile orientation is a
+ * reading, the DeepSeek-V3 technical report's: each GEMM input quantized
+ * along that GEMM's contraction).  For out_t = u_t + FFN_s(u_t) +
+ * sum_k g_{t,k} FFN_{e_{t,k}}(u_t) and a gradient dout of out:
+ *   every expert row p (token t, gate g; g = 1 for the shared expert)
+ *   receives dY_p = g * dout_t (FP32);
+ *   G, U recomputed (the forward's gate/up GEMM, FP32 results);
+ *   dh = dY W2      (dY 1x128 along H, W2's blocks transposed)
+ *   dG = dh U silu'(G), dU = dh silu(G), h = silu(G) U       (FP32)
+ *   dx_p = dG W1 + dU W3  (dG, dU 1x128 along I, W1/W3's blocks transposed)
+ *   dx_t = dout_t + sum over the token's rows of dx_p         (FP32)
+ *   dW2_e = dY_e^T h_e, dW13_e = [dG | dU]_e^T x_e over expert e's tokens
+ *   (both operands 128x1 along tokens: one scale per channel per 128
+ *   tokens, a ragged last tile shorter; every GEMM promotes each 128-long
+ *   partial into FP32).
+ * The gates' own gradient (router backward) is not part of this.
+ *
+ * moe_transpose_weights (set-up): the dgrad GEMMs' weights, each expert's
+ * codes and 128x128 block scales transposed:
+ *   w13t_dev E4M3 [E, H, 2I], s13t_dev float [E, H/128, 2I/128]
+ *   w2t_dev  E4M3 [E, I, H],  s2t_dev  float [E, I/128, H/128]
+ * moe_backward: call after the moe_forward of the same batch, same cfg and T,
+ * passing that forward's workspace (fwd_ws_dev), whose routing and grouping
+ * it reuses.
+ *   x_dev     bf16 [T, H] the forward's input;  dout_dev bf16 [T, H]
+ *   dx_dev    float [T, H]
+ *   dW13_dev  float [E, 2I, H] (rows 0..I-1 gate W1, I..2I-1 up W3)
+ *   dW2_dev   float [E, H, I]  (an expert no token selected gets zeros)
+ *   ws_dev    moe_backward_workspace_size() bytes, 256-byte aligned
+ * T >= 1; only scale_mode MOE_SCALE_AMAX (else MOE_ERR_NOT_IMPLEMENTED). */
+MOE_API int moe_transpose_weights(const moe_config *cfg, const moe_weights *w, uint8_t *w13t_dev, float *s13t_dev,
+                                  uint8_t *w2t_dev, float *s2t_dev, void *stream);
+MOE_API size_t moe_backward_workspace_size(const moe_config *cfg, int64_t T);
+MOE_API int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13t_dev,
+                         const float *s13t_dev, const uint8_t *w2t_dev, const float *s2t_dev, const void *x_dev,
+                         const void *dout_dev, int64_t T, float *dx_dev, float *dW13_dev, float *dW2_dev,
+                         const void *fwd_ws_dev, size_t fwd_ws_bytes, void *ws_dev, size_t ws_bytes,
+                         int32_t *err_flag_dev, void *stream);
+
 /* ------------------------------------------------- expert parallelism */
 /* The layer with its routed experts spread over W ranks (one GPU each), as
  * the DeepSeek-V3 pages run it: tokens travel to the GPUs of their experts

@@ -44,7 +44,7 @@ EXPORTS = (
     "moe_bias_update", "moe_check_device_error", "moe_selftest_wait_timeout", "moe_profile_events",
     "moe_route_noalloc", "moe_seq_balance_loss", "moe_set_gemm_variant",
     "moe_ep_row_bytes", "moe_ep_dispatch_workspace_size", "moe_ep_dispatch", "moe_ep_experts_workspace_size",
-    "moe_ep_experts", "moe_ep_combine",
+    "moe_ep_experts", "moe_ep_combine", "moe_transpose_weights", "moe_backward_workspace_size", "moe_backward",
 )
 MOE_GEMM_AUTO = 0
 MOE_GEMM_SINGLE = 1
@@ -107,9 +107,15 @@ lib.moe_ep_experts_workspace_size.restype = _sz
 lib.moe_ep_experts_workspace_size.argtypes = [_cfgp, _i64]
 lib.moe_ep_experts.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _i64, _i64, _vp, _vp, _sz, _vp, _vp]
 lib.moe_ep_combine.argtypes = [_cfgp, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _i32, _vp]
+lib.moe_transpose_weights.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _vp, _vp, _vp, _vp]
+lib.moe_backward_workspace_size.restype = _sz
+lib.moe_backward_workspace_size.argtypes = [_cfgp, _i64]
+lib.moe_backward.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
+                             _sz, _vp, _sz, _vp, _vp]
 for _name in EXPORTS:
     if _name not in ("moe_status_string", "moe_route_workspace_size", "moe_workspace_size", "moe_ep_row_bytes",
-                     "moe_ep_dispatch_workspace_size", "moe_ep_experts_workspace_size"):
+                     "moe_ep_dispatch_workspace_size", "moe_ep_experts_workspace_size",
+                     "moe_backward_workspace_size"):
         getattr(lib, _name).restype = C.c_int
 
 
@@ -318,6 +324,45 @@ def moe_ep_combine(cfg: MoeConfig, world: int, x, row_of, back, y_shared, out, o
     _check(lib.moe_ep_combine(C.byref(cfg), world, _ptr(x), x.shape[0], _ptr(row_of), _ptr(back), _ptr(y_shared),
                               _ptr(out), out_dtype, _stream(stream)), "moe_ep_combine")
     return out
+
+
+# ------------------------------------------------------------ backward
+def moe_transpose_weights(cfg: MoeConfig, w: dict, stream=None) -> dict:
+    """The dgrad GEMMs' weights: each expert's codes and block scales
+    transposed (w13t [E, H, 2I], s13t, w2t [E, I, H], s2t)."""
+    E, I2, H = w["w13"].shape
+    I = I2 // 2
+    dev = w["w13"].device
+    t = dict(w13t=torch.empty((E, H, I2), dtype=torch.uint8, device=dev),
+             s13t=torch.empty((E, H // 128, I2 // 128), dtype=torch.float32, device=dev),
+             w2t=torch.empty((E, I, H), dtype=torch.uint8, device=dev),
+             s2t=torch.empty((E, I // 128, H // 128), dtype=torch.float32, device=dev))
+    ws = weights_struct(w)
+    _check(lib.moe_transpose_weights(C.byref(cfg), C.byref(ws), _ptr(t["w13t"]), _ptr(t["s13t"]), _ptr(t["w2t"]),
+                                     _ptr(t["s2t"]), _stream(stream)), "moe_transpose_weights")
+    return t
+
+
+def moe_backward(cfg: MoeConfig, w: dict, wt: dict, x, dout, fwd_ws, dx=None, dW13=None, dW2=None, ws=None,
+                 err=None, stream=None):
+    """Gradients of the layer's expert FFNs (routing held fixed) for the batch
+    whose forward left its state in fwd_ws: dx [T, H], dW13 [E, 2I, H],
+    dW2 [E, H, I], all float32."""
+    T, H = x.shape
+    dev = x.device
+    E, I2, _ = w["w13"].shape
+    dx = torch.empty((T, H), dtype=torch.float32, device=dev) if dx is None else dx
+    dW13 = torch.empty((E, I2, H), dtype=torch.float32, device=dev) if dW13 is None else dW13
+    dW2 = torch.empty((E, H, I2 // 2), dtype=torch.float32, device=dev) if dW2 is None else dW2
+    if ws is None:
+        ws = torch.empty(max(int(lib.moe_backward_workspace_size(C.byref(cfg), T)), 256), dtype=torch.uint8,
+                         device=dev)
+    err = new_err_flag(dev) if err is None else err
+    wst = weights_struct(w)
+    _check(lib.moe_backward(C.byref(cfg), C.byref(wst), _ptr(wt["w13t"]), _ptr(wt["s13t"]), _ptr(wt["w2t"]),
+                            _ptr(wt["s2t"]), _ptr(x), _ptr(dout), T, _ptr(dx), _ptr(dW13), _ptr(dW2), _ptr(fwd_ws),
+                            fwd_ws.numel(), _ptr(ws), ws.numel(), _ptr(err), _stream(stream)), "moe_backward")
+    return dx, dW13, dW2
 
 
 def ws_view(ws: torch.Tensor, layout: dict, name: str, dtype, shape) -> torch.Tensor:

@@ -686,6 +686,271 @@ int moe_ep_combine(const moe_config *cfg, int32_t world, const void *x, int64_t 
                                             out_dtype == MOE_DTYPE_F32, static_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------------------------ backward
+namespace {
+struct BwdLayout {
+  size_t gu[2], dyq[2], dys[2], dh[2], h[2], dgu[2], dguq[2], dgus[2], dxr[2];
+  size_t counts[2], offsets[2], blk_base[2], chunks[2], meta[2];
+  size_t seg[2], tiles[2], tmeta[2];
+  size_t dyt[2], sdy[2], ht[2], sh[2], dgut[2], sdgu[2], xt[2], sx[2];
+  int64_t P, max_tiles;
+  size_t total;
+};
+
+void make_bwd_layout(const moe_config *c, int64_t T, BwdLayout *B) {
+  const int64_t H = c->hidden, I = c->inter, Nr = c->n_routed, Kr = c->top_k, Ns = c->n_shared;
+  const int64_t R = T * Kr, RS = R + T * Ns, E = Nr + Ns;
+  const int64_t pitch = moe::scale_pitch(R, T);
+  const int64_t nblk = (T + 127) / 128;
+  B->P = (RS + 128 * E + 127) / 128 * 128;
+  B->max_tiles = RS / 128 + E;
+  Carve cv;
+  cv.take(B->gu, RS * 2 * I * 4);
+  cv.take(B->dyq, RS * H);
+  cv.take(B->dys, ((H / 128) * pitch + moe::kScaleSlack) * 4);
+  cv.take(B->dh, RS * I * 4);
+  cv.take(B->h, RS * I * 4);
+  cv.take(B->dgu, RS * 2 * I * 4);
+  cv.take(B->dguq, RS * 2 * I);
+  cv.take(B->dgus, ((2 * I / 128) * pitch + moe::kScaleSlack) * 4);
+  cv.take(B->dxr, RS * H * 4);
+  cv.take(B->counts, Nr * 4);
+  cv.take(B->offsets, (Nr + 1) * 4);
+  cv.take(B->blk_base, nblk * Nr * 4);
+  cv.take(B->chunks, moe::max_chunks(T, static_cast<int>(Kr), static_cast<int>(Nr), static_cast<int>(Ns)) * 16);
+  cv.take(B->meta, 4 * 4);
+  cv.take(B->seg, (E + 1) * 4);
+  cv.take(B->tiles, B->max_tiles * 16);
+  cv.take(B->tmeta, 4 * 4);
+  cv.take(B->dyt, H * B->P);
+  cv.take(B->sdy, (B->P / 128) * H * 4);
+  cv.take(B->ht, I * B->P);
+  cv.take(B->sh, (B->P / 128) * I * 4);
+  cv.take(B->dgut, 2 * I * B->P);
+  cv.take(B->sdgu, (B->P / 128) * 2 * I * 4);
+  cv.take(B->xt, H * B->P);
+  cv.take(B->sx, (B->P / 128) * H * 4);
+  B->total = (cv.off + 255) & ~size_t(255);
+}
+}  // namespace
+
+int moe_transpose_weights(const moe_config *cfg, const moe_weights *w, uint8_t *w13t, float *s13t, uint8_t *w2t,
+                          float *s2t, void *stream) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (!w || !w->w13_dev || !w->s13_dev || !w->w2_dev || !w->s2_dev || !w13t || !s13t || !w2t || !s2t)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned4(w->s13_dev) || !aligned4(w->s2_dev) || !aligned4(s13t) || !aligned4(s2t)) return MOE_ERR_INVALID_ARG;
+  if (const int d = check_device()) return d;
+  const int64_t E = static_cast<int64_t>(cfg->n_routed) + cfg->n_shared, H = cfg->hidden, I = cfg->inter;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = moe::launch_transpose_blocks(w->w13_dev, w->s13_dev, 2 * I, H, E, w13t, s13t, st);
+  if (e == cudaSuccess) e = moe::launch_transpose_blocks(w->w2_dev, w->s2_dev, H, I, E, w2t, s2t, st);
+  return cuda_status(e);
+}
+
+size_t moe_backward_workspace_size(const moe_config *cfg, int64_t T) {
+  if (check_cfg(cfg) != MOE_OK || T < 0 || T > kMaxTokens) return 0;
+  BwdLayout B;
+  make_bwd_layout(cfg, T, &B);
+  return B.total;
+}
+
+int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13t, const float *s13t,
+                 const uint8_t *w2t, const float *s2t, const void *x, const void *dout, int64_t T, float *dx,
+                 float *dW13, float *dW2, const void *fwd_ws, size_t fwd_ws_bytes, void *ws, size_t ws_bytes,
+                 int32_t *err_flag, void *stream) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (cfg->scale_mode != MOE_SCALE_AMAX) return MOE_ERR_NOT_IMPLEMENTED;
+  if (T < 1 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
+  if (!w || !w->w13_dev || !w->s13_dev || !w->w2_dev || !w->s2_dev || !w13t || !s13t || !w2t || !s2t || !x ||
+      !dout || !dx || !dW13 || !dW2 || !fwd_ws || !ws || !err_flag)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dout) || !aligned16(dx) || !aligned16(dW13) || !aligned16(dW2) ||
+      !aligned16(w13t) || !aligned16(w2t) || !aligned4(s13t) || !aligned4(s2t) || !aligned4(err_flag) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255) || (reinterpret_cast<uintptr_t>(fwd_ws) & 255))
+    return MOE_ERR_INVALID_ARG;
+  moe_ws_layout L;
+  make_layout(cfg, T, &L);
+  if (fwd_ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  BwdLayout B;
+  make_bwd_layout(cfg, T, &B);
+  if (ws_bytes < B.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (const int d = check_device()) return d;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void *fws = const_cast<void *>(fwd_ws);
+  const int H = cfg->hidden, I = cfg->inter, Nr = cfg->n_routed, Kr = cfg->top_k, Ns = cfg->n_shared;
+  const int64_t R = T * Kr, RS = R + T * Ns, E = static_cast<int64_t>(Nr) + Ns;
+  const int64_t pitch = moe::scale_pitch(R, T);
+  // the forward's intermediates this backward reads
+  const uint8_t *xq = at<uint8_t *>(fws, L.xq);
+  const uint8_t *ap = at<uint8_t *>(fws, L.ap);
+  const float *as_t = at<float *>(fws, L.as);
+  const int32_t *pos = at<int32_t *>(fws, L.pos);
+  const int32_t *row_src = at<int32_t *>(fws, L.row_src);
+  const float *row_gate = at<float *>(fws, L.row_gate);
+  const int32_t *blk_hist = at<int32_t *>(fws, L.blk_hist);
+  // this backward's own buffers
+  float *GU = at<float *>(ws, B.gu);
+  uint8_t *dyq = at<uint8_t *>(ws, B.dyq);
+  float *dys = at<float *>(ws, B.dys);
+  float *dh = at<float *>(ws, B.dh);
+  float *hbuf = at<float *>(ws, B.h);
+  float *dGU = at<float *>(ws, B.dgu);
+  uint8_t *dGUq = at<uint8_t *>(ws, B.dguq);
+  float *dGUs = at<float *>(ws, B.dgus);
+  float *dxr = at<float *>(ws, B.dxr);
+  int32_t *counts = at<int32_t *>(ws, B.counts);
+  int32_t *offsets = at<int32_t *>(ws, B.offsets);
+  int32_t *blk_base = at<int32_t *>(ws, B.blk_base);
+  int4 *chunks = at<int4 *>(ws, B.chunks);
+  int32_t *meta = at<int32_t *>(ws, B.meta);
+  int32_t *seg = at<int32_t *>(ws, B.seg);
+  int4 *tiles = at<int4 *>(ws, B.tiles);
+  int32_t *tmeta = at<int32_t *>(ws, B.tmeta);
+  const int64_t max_chunks = moe::max_chunks(T, Kr, Nr, Ns);
+
+  // 128-row chunks of the forward's expert grouping (the single-CTA GEMM)
+  cudaError_t e = moe::launch_build_chunks(blk_hist, T, Kr, Nr, Ns, 128, counts, offsets, blk_base, chunks, meta,
+                                           nullptr, st);
+  auto base_gemm = [&](moe::GemmLaunch &g) {
+    g.chunks = chunks;
+    g.n_chunks = meta;
+    g.max_chunks = static_cast<int>(max_chunks);
+    g.chunk_rows = 128;
+    g.sa_transposed = 1;
+    g.sa_ld = pitch;
+    g.err = err_flag;
+    g.wait_limit_ns = moe::kDefaultWaitLimitNs;
+  };
+  if (e == cudaSuccess) {
+    // G, U again: the forward's gate/up GEMM with FP32 outputs
+    moe::GemmLaunch g{};
+    base_gemm(g);
+    g.w = w->w13_dev;
+    g.w_rows = E * 2 * I;
+    g.a0 = ap;
+    g.a0_rows = R;
+    g.a1 = Ns ? xq : ap;
+    g.a1_rows = Ns ? T : R;
+    g.K = H;
+    g.sw = w->s13_dev;
+    g.sa0 = as_t;
+    g.sa1 = as_t;
+    g.nb = moe::gemm1_blocks(I);
+    g.gate_up = 1;
+    g.half = I;
+    g.rows_per_expert = 2 * static_cast<int64_t>(I);
+    g.epi = moe::EPI_F32;
+    g.out = GU;
+    g.ldo = 2 * I;
+    g.out_rows = RS;
+    g.out_cols = 2 * I;
+    e = moe::launch_gemm(g, st);
+  }
+  if (e == cudaSuccess) e = moe::launch_dy_quant(dout, row_src, row_gate, R, RS, H, dyq, dys, pitch, st);
+  if (e == cudaSuccess) {
+    // dh = dY W2: K = H against W2^T [E, I, H]
+    moe::GemmLaunch g{};
+    base_gemm(g);
+    g.w = w2t;
+    g.w_rows = E * I;
+    g.a0 = dyq;
+    g.a0_rows = RS;
+    g.a1 = dyq;
+    g.a1_rows = RS;
+    g.K = H;
+    g.sw = s2t;
+    g.sa0 = dys;
+    g.sa1 = dys;
+    g.nb = moe::gemm2_blocks(I);
+    g.gate_up = 0;
+    g.a_is_out_row = 1;
+    g.rows_per_expert = I;
+    g.epi = moe::EPI_F32;
+    g.out = dh;
+    g.ldo = I;
+    g.out_rows = RS;
+    g.out_cols = I;
+    e = moe::launch_gemm(g, st);
+  }
+  if (e == cudaSuccess) e = moe::launch_swiglu_bwd(GU, dh, RS, I, hbuf, dGU, dGUq, dGUs, pitch, st);
+  if (e == cudaSuccess) {
+    // dx rows = [dG|dU] [W1; W3] (FP32): K = 2I against W13^T [E, H, 2I]
+    moe::GemmLaunch g{};
+    base_gemm(g);
+    g.w = w13t;
+    g.w_rows = E * H;
+    g.a0 = dGUq;
+    g.a0_rows = RS;
+    g.a1 = dGUq;
+    g.a1_rows = RS;
+    g.K = 2 * I;
+    g.sw = s13t;
+    g.sa0 = dGUs;
+    g.sa1 = dGUs;
+    g.nb = moe::gemm2_blocks(H);
+    g.gate_up = 0;
+    g.a_is_out_row = 1;
+    g.rows_per_expert = H;
+    g.epi = moe::EPI_F32;
+    g.out = dxr;
+    g.ldo = H;
+    g.out_rows = RS;
+    g.out_cols = H;
+    e = moe::launch_gemm(g, st);
+  }
+  // dx_t = dout_t + the token's rows (shared, then its slots), FP32
+  if (e == cudaSuccess) e = moe::launch_combine(dout, dxr, pos, T, H, Kr, R, Ns, dx, 1, st, true);
+  // weight gradients: 128-token tiles of every expert, operands transposed
+  if (e == cudaSuccess) e = moe::launch_wgrad_tiles(offsets, Nr, Ns, R, T, seg, tiles, tmeta, st);
+  const int mt = static_cast<int>(B.max_tiles);
+  if (e == cudaSuccess)
+    e = moe::launch_colquant(1, tiles, tmeta, mt, nullptr, 0, dout, row_src, row_gate, R, H, at<uint8_t *>(ws, B.dyt),
+                             B.P, at<float *>(ws, B.sdy), st);
+  if (e == cudaSuccess)
+    e = moe::launch_colquant(0, tiles, tmeta, mt, hbuf, I, nullptr, row_src, row_gate, R, I, at<uint8_t *>(ws, B.ht),
+                             B.P, at<float *>(ws, B.sh), st);
+  if (e == cudaSuccess)
+    e = moe::launch_colquant(0, tiles, tmeta, mt, dGU, 2 * I, nullptr, row_src, row_gate, R, 2 * I,
+                             at<uint8_t *>(ws, B.dgut), B.P, at<float *>(ws, B.sdgu), st);
+  if (e == cudaSuccess)
+    e = moe::launch_colquant(2, tiles, tmeta, mt, nullptr, 0, x, row_src, row_gate, R, H, at<uint8_t *>(ws, B.xt),
+                             B.P, at<float *>(ws, B.sx), st);
+  if (e == cudaSuccess) {
+    moe::WgradLaunch g{};
+    g.a_t = at<uint8_t *>(ws, B.dyt);
+    g.b_t = at<uint8_t *>(ws, B.ht);
+    g.sa_t = at<float *>(ws, B.sdy);
+    g.sb_t = at<float *>(ws, B.sh);
+    g.seg = seg;
+    g.E = static_cast<int>(E);
+    g.C_out = H;
+    g.C_in = I;
+    g.P = B.P;
+    g.out = dW2;
+    g.err = err_flag;
+    g.wait_limit_ns = moe::kDefaultWaitLimitNs;
+    e = moe::launch_gemm_wgrad(g, st);
+  }
+  if (e == cudaSuccess) {
+    moe::WgradLaunch g{};
+    g.a_t = at<uint8_t *>(ws, B.dgut);
+    g.b_t = at<uint8_t *>(ws, B.xt);
+    g.sa_t = at<float *>(ws, B.sdgu);
+    g.sb_t = at<float *>(ws, B.sx);
+    g.seg = seg;
+    g.E = static_cast<int>(E);
+    g.C_out = 2 * I;
+    g.C_in = H;
+    g.P = B.P;
+    g.out = dW13;
+    g.err = err_flag;
+    g.wait_limit_ns = moe::kDefaultWaitLimitNs;
+    e = moe::launch_gemm_wgrad(g, st);
+  }
+  return cuda_status(e);
+}
+
 int moe_seq_balance_loss(const moe_config *cfg, int64_t T, int64_t seq_len, float alpha, const void *ws,
                          size_t ws_bytes, float *loss, int32_t *err_flag, void *stream) {
   if (const int c = check_cfg(cfg)) return c;

@@ -23,28 +23,47 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 &v) {
   }
 }
 
+// eight FP32 values (two 16-byte words) added to eight FP32 accumulators
+__device__ __forceinline__ void add_f32x8(float (&acc)[8], const float4 *p) {
+  const float4 a = __ldg(p), b = __ldg(p + 1);
+  acc[0] += a.x;
+  acc[1] += a.y;
+  acc[2] += a.z;
+  acc[3] += a.w;
+  acc[4] += b.x;
+  acc[5] += b.y;
+  acc[6] += b.z;
+  acc[7] += b.w;
+}
+
 // One CTA per token, 8 channels (16-byte loads of x and of every y row) per
-// thread and step.  y rows are bf16: the gate-scaled output of each routed
-// expert, the shared expert's at row R + t.
-template <bool OUT_F32>
-__global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16 *__restrict__ x,
-                                                       const __nv_bfloat16 *__restrict__ y,
+// thread and step.  y rows are bf16 (the gate-scaled output of each routed
+// expert, the shared expert's at row R + t), or FP32 when Y_F32.
+template <bool OUT_F32, bool Y_F32>
+__global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16 *__restrict__ x, const void *__restrict__ yv,
                                                        const int32_t *__restrict__ pos, int H, int Kr, int64_t R,
                                                        int Ns, void *__restrict__ out) {
+  const __nv_bfloat16 *y = static_cast<const __nv_bfloat16 *>(yv);
+  const float *yf = static_cast<const float *>(yv);
   const int64_t t = blockIdx.x;
   int p[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) p[k] = (k < Kr) ? pos[t * Kr + k] : -1;
   const int hv = H / 8;
-  const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * H);
-  const uint4 *ysh = reinterpret_cast<const uint4 *>(y + (R + t) * H);
+  const uint4 *xr = x ? reinterpret_cast<const uint4 *>(x + t * H) : nullptr;
   for (int v = threadIdx.x; v < hv; v += blockDim.x) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (x) add_bf16x8(acc, __ldg(xr + v));  // residual u_t
-    if (Ns) add_bf16x8(acc, __ldg(ysh + v));
+    if (xr) add_bf16x8(acc, __ldg(xr + v));  // residual u_t
+    auto add_row = [&](int64_t row) {
+      if (Y_F32)
+        add_f32x8(acc, reinterpret_cast<const float4 *>(yf + row * H) + 2 * v);
+      else
+        add_bf16x8(acc, __ldg(reinterpret_cast<const uint4 *>(y + row * H) + v));
+    };
+    if (Ns) add_row(R + t);
 #pragma unroll
     for (int k = 0; k < 16; ++k)
-      if (k < Kr && p[k] >= 0) add_bf16x8(acc, __ldg(reinterpret_cast<const uint4 *>(y + static_cast<int64_t>(p[k]) * H) + v));
+      if (k < Kr && p[k] >= 0) add_row(p[k]);
     if (OUT_F32) {
       float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + t * H) + 2 * v;
       o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -90,14 +109,21 @@ __global__ void wait_selftest_kernel(int32_t *err, uint64_t limit_ns) {
 }
 
 cudaError_t launch_combine(const void *x, const void *y, const int32_t *pos, int64_t T, int H, int Kr, int64_t R,
-                           int Ns, void *out, int out_f32, cudaStream_t st) {
+                           int Ns, void *out, int out_f32, cudaStream_t st, bool y_f32) {
   if (T == 0) return cudaSuccess;
   const auto *xb = static_cast<const __nv_bfloat16 *>(x);
-  const auto *yb = static_cast<const __nv_bfloat16 *>(y);
-  if (out_f32)
-    combine_kernel<true><<<static_cast<unsigned>(T), 128, 0, st>>>(xb, yb, pos, H, Kr, R, Ns, out);
-  else
-    combine_kernel<false><<<static_cast<unsigned>(T), 128, 0, st>>>(xb, yb, pos, H, Kr, R, Ns, out);
+  const dim3 grid(static_cast<unsigned>(T));
+  if (y_f32) {
+    if (out_f32)
+      combine_kernel<true, true><<<grid, 128, 0, st>>>(xb, y, pos, H, Kr, R, Ns, out);
+    else
+      combine_kernel<false, true><<<grid, 128, 0, st>>>(xb, y, pos, H, Kr, R, Ns, out);
+  } else {
+    if (out_f32)
+      combine_kernel<true, false><<<grid, 128, 0, st>>>(xb, y, pos, H, Kr, R, Ns, out);
+    else
+      combine_kernel<false, false><<<grid, 128, 0, st>>>(xb, y, pos, H, Kr, R, Ns, out);
+  }
   return cudaGetLastError();
 }
 

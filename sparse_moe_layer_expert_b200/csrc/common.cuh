@@ -420,6 +420,17 @@ __device__ __forceinline__ void ffma2_scalar(float &c_lo, float &c_hi, float p_l
   asm("mov.b64 {%0, %1}, %2;" : "=f"(c_lo), "=f"(c_hi) : "l"(c));
 }
 
+// (lo, hi) <- (p_lo * s_lo + c_lo, p_hi * s_hi + c_hi): two FMAs with their
+// own multipliers, one instruction.
+__device__ __forceinline__ void ffma2_vec(float &c_lo, float &c_hi, float p_lo, float p_hi, float s_lo, float s_hi) {
+  uint64_t c, p, ss;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(c_lo), "f"(c_hi));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(p) : "f"(p_lo), "f"(p_hi));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ss) : "f"(s_lo), "f"(s_hi));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(c) : "l"(p), "l"(ss));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(c_lo), "=f"(c_hi) : "l"(c));
+}
+
 // Power-of-two scale, the variant whose scale factors a tensor core applies
 // itself (block-scaled MMA with 8-bit exponent scale factors): S = 2^e with e
 // the smallest integer for which amax <= 448 * 2^e, held at 2^-127 or above;

@@ -32,6 +32,7 @@
 //                 thread stored as 16-byte vectors -> hq, scale -> hs
 //   EPI_GATE_BF16 y = bf16(acc * gate[row]) (down projection)
 //   EPI_BF16      C = bf16(acc) (plain GEMM)
+//   EPI_F32       C = acc in FP32 (the backward's recomputed G, U and dh)
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warp 2 scale producer, warp 3 idle, warps 4..11 promotion +
@@ -369,6 +370,7 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st) {
   switch (g.epi) {
     case EPI_SWIGLU_Q: return launch_epi<EPI_SWIGLU_Q>(mw, m0, m1, a, grid, st);
     case EPI_GATE_BF16: return launch_epi<EPI_GATE_BF16>(mw, m0, m1, a, grid, st);
+    case EPI_F32: return launch_epi<EPI_F32>(mw, m0, m1, a, grid, st);
     default: return launch_epi<EPI_BF16>(mw, m0, m1, a, grid, st);
   }
 }

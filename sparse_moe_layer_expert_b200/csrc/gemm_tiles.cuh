@@ -101,6 +101,8 @@ __device__ __forceinline__ bool tile_ok(const GemmArgs &a, const GemmTile &d) {
 //   EPI_GATE_BF16 y = bf16(acc * gate[row]) (down projection; the product in
 //                 FP32, rounded to nearest even)
 //   EPI_BF16      C = bf16(acc) (plain GEMM)
+//   EPI_F32       C = acc in FP32 (block B at +128 columns, or at +half for a
+//                 gate/up pair)
 // Both warpgroups take the named barrier 1 (256 threads) twice per tile in
 // EPI_SWIGLU_Q.
 constexpr int G_OPITCH = 20;  // floats per row of an output transpose buffer (16 + pad)
@@ -157,6 +159,37 @@ __device__ __forceinline__ void tile_epilogue(const GemmArgs &args, const GemmTi
       if (wg == 0) args.out_scale[static_cast<int64_t>(td.out_col / 128) * args.ld_os + orow] = S;
     }
     named_bar_sync(1, 256);  // amx is reused by the next tile
+  } else if constexpr (EPI == EPI_F32) {
+    // FP32 results of both blocks; block B's columns follow block A's (+128),
+    // or start at +half when the pair is gate block j / up block j
+    float *xb = outx + (warp - 4) * (32 * G_OPITCH);
+    const int rbase = q * 32;
+    const int64_t cB = args.gate_up ? args.half : 128;
+    auto emit = [&](const float(&acc)[64], int64_t cbase) {
+#pragma unroll
+      for (int piece = 0; piece < 4; ++piece) {
+        float4 *dst = reinterpret_cast<float4 *>(xb + lane * G_OPITCH);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int j = piece * 16 + 4 * v;
+          dst[v] = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int sgrp = 0; sgrp < 4; ++sgrp) {
+          const int rr = lane / 4 + 8 * sgrp;
+          if (rbase + rr < td.n) {
+            const float4 val = reinterpret_cast<const float4 *>(xb + rr * G_OPITCH)[lane & 3];
+            const int64_t grow = static_cast<int64_t>(td.out_row) + rbase + rr;
+            float *crow = static_cast<float *>(args.out) + grow * args.ldo + cbase + piece * 16;
+            reinterpret_cast<float4 *>(crow)[lane & 3] = val;
+          }
+        }
+        __syncwarp();
+      }
+    };
+    emit(acc0, c0);
+    if (two) emit(acc1, c0 + cB);
   } else {
     // Rows are written through a per-warp 32 x 16-float transpose buffer
     // so that each 16-byte store instruction covers 8 rows x 64

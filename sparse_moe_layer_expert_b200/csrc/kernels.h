@@ -38,7 +38,7 @@ struct GemmTile {
   int32_t pad;
 };
 
-enum EpiKind : int { EPI_SWIGLU_Q = 0, EPI_GATE_BF16 = 1, EPI_BF16 = 2 };
+enum EpiKind : int { EPI_SWIGLU_Q = 0, EPI_GATE_BF16 = 1, EPI_BF16 = 2, EPI_F32 = 3 };
 
 struct GemmLaunch {
   // tensor operands
@@ -128,8 +128,9 @@ cudaError_t launch_gemm_mx(const GemmLaunch &g, cudaStream_t st);
 
 // out[t] = x[t] (when x is not null) + y[R + t] (when Ns) + sum_k y[pos[t, k]]
 // (pos >= 0), FP32 in that order, written as FP32 or bf16 (RNE)
+// (y rows bf16, or FP32 when y_f32)
 cudaError_t launch_combine(const void *x, const void *y, const int32_t *pos, int64_t T, int H, int Kr,
-                           int64_t R, int Ns, void *out, int out_f32, cudaStream_t st);
+                           int64_t R, int Ns, void *out, int out_f32, cudaStream_t st, bool y_f32 = false);
 // Expert parallelism (ep.cu): dispatch of one rank's routed tokens into a
 // send buffer ordered by destination, the receiving side's unpacking of the
 // packed rows, and the sending side's combine of the returned partial sums.
@@ -141,6 +142,36 @@ cudaError_t launch_ep_unpack(const uint8_t *rows, int64_t n, int64_t row_bytes, 
                              int32_t *idx, float *gate, float *xs, int32_t *err, cudaStream_t st);
 cudaError_t launch_ep_combine(const void *x, const void *y_sh, const void *back, const int32_t *row_of, int64_t T,
                               int W, int H, void *out, int out_f32, cudaStream_t st);
+
+// Backward of the expert FFNs (backward.cu, gemm_wgrad.cu).
+cudaError_t launch_transpose_blocks(const uint8_t *q, const float *s, int64_t n, int64_t k, int64_t batch,
+                                    uint8_t *qt, float *st, cudaStream_t stream);
+cudaError_t launch_dy_quant(const void *dout, const int32_t *row_src, const float *row_gate, int64_t R, int64_t RS,
+                            int H, uint8_t *q, float *s_t, int64_t ld, cudaStream_t st);
+cudaError_t launch_swiglu_bwd(const float *GU, const float *dh, int64_t RS, int I, float *h, float *dGU, uint8_t *q,
+                              float *s_t, int64_t ld, cudaStream_t st);
+cudaError_t launch_wgrad_tiles(const int32_t *offsets, int Nr, int Ns, int64_t R, int64_t T, int32_t *seg,
+                               int4 *tiles, int32_t *meta, cudaStream_t st);
+// src: 0 = FP32 rows (f32rows, f32_ld floats apart), 1 = dY from bf16 dout
+// rows gathered by token times the row gate, 2 = bf16 rows gathered by token
+cudaError_t launch_colquant(int src, const int4 *tiles, const int32_t *meta, int max_tiles, const float *f32rows,
+                            int64_t f32_ld, const void *bf16rows, const int32_t *row_src, const float *row_gate,
+                            int64_t R, int C, uint8_t *out, int64_t out_ld, float *s_t, cudaStream_t st);
+
+// Weight-gradient GEMM: dW[e] = A_e^T B_e over each expert's token segment.
+struct WgradLaunch {
+  const uint8_t *a_t;    // E4M3 [C_out, P] (tokens contiguous)
+  const uint8_t *b_t;    // E4M3 [C_in, P]
+  const float *sa_t;     // [P/128][C_out]
+  const float *sb_t;     // [P/128][C_in]
+  const int32_t *seg;    // [E + 1] segment starts (multiples of 128), seg[E] <= P
+  int E;
+  int64_t C_out, C_in, P;
+  float *out;            // FP32 [E, C_out, C_in]
+  int32_t *err;
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_gemm_wgrad(const WgradLaunch &g, cudaStream_t st);
 
 cudaError_t launch_bias_update(float *bias, const int32_t *counts, int Nr, int64_t total, float gamma,
                                cudaStream_t st);

@@ -93,6 +93,17 @@ class MoeLayer:
         last forward of that size routed, one value per run of seq_len tokens."""
         return B.moe_seq_balance_loss(self.cfg, T, seq_len, self.workspace(T), self.err, alpha=alpha, stream=stream)
 
+    def backward(self, x: torch.Tensor, dout: torch.Tensor, stream=None):
+        """Gradients of the expert FFNs for the batch this layer's last forward
+        of that size routed (routing held fixed): (dx, dW13, dW2) in FP32.
+        The transposed weight copies the dgrad GEMMs read are made on first
+        use (set-up) and kept."""
+        if getattr(self, "_wt", None) is None:
+            self._wt = B.moe_transpose_weights(self.cfg, self.weights(), stream=stream)
+        T = x.shape[0]
+        return B.moe_backward(self.cfg, self.weights(), self._wt, x, dout, self.workspace(T), err=self.err,
+                              stream=stream)
+
     def check(self, stream=None) -> None:
         st, v = B.moe_check_device_error(self.err, stream)
         if st != B.MOE_OK:
