@@ -184,7 +184,7 @@ def profiled_traffic(workload: str, kernel: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle reasons sampled every 100 ms while running."""
+    """nvidia-smi clocks/throttle reasons sampled every 25 ms while running."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -200,10 +200,16 @@ class ClockSampler:
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "25"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        # the region to sample starts only once the sampler is producing
+        t0 = time.perf_counter()
+        while self.proc is not None and time.perf_counter() - t0 < 5.0:
+            if os.path.getsize(self.path) > 0 or self.proc.poll() is not None:
+                break
+            time.sleep(0.01)
         return self
 
     def __exit__(self, *a):

@@ -4,8 +4,9 @@
 // E4M3 for all tensors, 1x128 tiles for activations, 128x128 blocks for
 // weights.  "DeepSeek-V3 技術報告書" (singularity-lens.com), formula
 // paragraph: S = max|X| / 448 and X_FP8 = clip(round(X / S), -448, 448).
-// The quotient X / S is an IEEE FP32 division (this file is compiled without
-// fast-math) and the cast rounds to nearest even, saturating at +-448.
+// The quotient X / S is the IEEE FP32 correctly rounded one (this file is
+// compiled without fast-math) and the cast rounds to nearest even, saturating
+// at +-448.
 // POW2 = true: the power-of-two scale variant (pow2_scale in common.cuh),
 // for which X / S is an exact scaling.
 #include "common.cuh"
@@ -22,9 +23,20 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
   }
 }
 
+// Codes of 8 values sharing the scale S.  The quotients x / S are the IEEE
+// correctly rounded ones: for S well inside the normal range through the
+// reciprocal plus one residual correction (div_by_recip, common.cuh), which
+// gives the same correctly rounded result as the division; for tiny S by the
+// division itself.
 __device__ __forceinline__ uint2 codes8(const float (&f)[8], float S) {
   uint32_t lo = 0, hi = 0;
-  if (S != 0.0f) {
+  if (S >= 0x1p-100f) {
+    const float y = __frcp_rn(S);
+    lo = e4m3x2_rn_sat(div_by_recip(f[0], S, y), div_by_recip(f[1], S, y)) |
+         (e4m3x2_rn_sat(div_by_recip(f[2], S, y), div_by_recip(f[3], S, y)) << 16);
+    hi = e4m3x2_rn_sat(div_by_recip(f[4], S, y), div_by_recip(f[5], S, y)) |
+         (e4m3x2_rn_sat(div_by_recip(f[6], S, y), div_by_recip(f[7], S, y)) << 16);
+  } else if (S != 0.0f) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) lo |= static_cast<uint32_t>(e4m3_rn_sat(f[i] / S)) << (8 * i);
 #pragma unroll

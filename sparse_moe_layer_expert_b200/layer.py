@@ -73,12 +73,34 @@ class MoeLayer:
         return dict(w13=self.w13, s13=self.s13, w2=self.w2, s2=self.s2, wr=self.wr)
 
     # -------------------------------------------------------------- forward
+    # Guard bands (bytes, a multiple of 256) around every workspace, filled
+    # with GUARD_BYTE and checked by check_guards(): a kernel writing past
+    # either end of its workspace shows up there.  Off (0) unless set.
+    guard_bytes = 0
+    GUARD_BYTE = 0xA5
+
     def workspace(self, T: int) -> torch.Tensor:
         ws = self._ws.get(T)
         if ws is None:
-            ws = torch.empty(max(B.moe_workspace_size(self.cfg, T), 256), dtype=torch.uint8, device=self.device)
+            n = max(B.moe_workspace_size(self.cfg, T), 256)
+            g = self.guard_bytes
+            if g:
+                assert g % 256 == 0
+                buf = torch.full((n + 2 * g,), self.GUARD_BYTE, dtype=torch.uint8, device=self.device)
+                ws = buf[g:g + n]
+                self._guarded = getattr(self, "_guarded", [])
+                self._guarded.append((buf, g, n))
+            else:
+                ws = torch.empty(n, dtype=torch.uint8, device=self.device)
             self._ws[T] = ws
         return ws
+
+    def check_guards(self) -> None:
+        """Raise if any guard band around this layer's workspaces changed."""
+        for buf, g, n in getattr(self, "_guarded", []):
+            head, tail = buf[:g], buf[g + n:]
+            if not (bool((head == self.GUARD_BYTE).all()) and bool((tail == self.GUARD_BYTE).all())):
+                raise RuntimeError(f"workspace guard band overwritten (workspace of {n} bytes)")
 
     def forward(self, x: torch.Tensor, out=None, out_dtype=B.MOE_DTYPE_BF16, idx_out=None, counts_out=None,
                 stream=None) -> torch.Tensor:

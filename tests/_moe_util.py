@@ -110,3 +110,26 @@ class Problem:
         W13q, s13 = oracle.quant_128x128(w13, mode)
         W2q, s2 = oracle.quant_128x128(w2, mode)
         return W13q, s13, W2q, s2
+
+
+GUARD = 4096        # guard band (bytes) around buffers the GPU tests hand to the library
+GUARD_BYTE = 0xA5
+
+
+def guarded_empty(shape, dtype, device="cuda"):
+    """An uninitialised tensor inside a buffer with GUARD bytes of a fixed
+    pattern on both sides; returns (tensor, check) where check() raises if a
+    kernel wrote into either band."""
+    esz = torch.empty((), dtype=dtype).element_size()
+    n = 1
+    for s in shape:
+        n *= s
+    nbytes = n * esz
+    buf = torch.full((nbytes + 2 * GUARD,), GUARD_BYTE, dtype=torch.uint8, device=device)
+    t = buf[GUARD:GUARD + nbytes].view(dtype).view(shape)
+
+    def check():
+        ok = bool((buf[:GUARD] == GUARD_BYTE).all()) and bool((buf[GUARD + nbytes:] == GUARD_BYTE).all())
+        assert ok, f"guard band around a {tuple(shape)} {dtype} buffer overwritten"
+
+    return t, check

@@ -139,3 +139,31 @@ def test_seq_balance_loss_validation_without_device(m):
     assert L.moe_seq_balance_loss(C.byref(cfg), 96, 32, a, 256, 1024, 16, 16, None) == \
         m.MOE_ERR_WORKSPACE_TOO_SMALL
     assert L.moe_seq_balance_loss(C.byref(cfg), 96, 32, a, 256, big, 16, 16, None) == m.MOE_ERR_NO_DEVICE
+
+
+def test_workspace_guard_bands_catch_overruns(m):
+    """The guard bands the GPU tests put around every workspace and output
+    buffer: intact after a call that stays inside, reported when a byte past
+    either end changes (exercised here on host memory)."""
+    import sys
+
+    import torch
+    layer = m.MoeLayer(dict(H=512, I=256, Nr=16, Kr=4, Ns=1), "cpu")
+    layer.guard_bytes = 4096
+    ws = layer.workspace(64)
+    assert ws.numel() == m.moe_workspace_size(layer.cfg, 64)
+    ws.fill_(0)              # the call's own bytes may change freely
+    layer.check_guards()
+    buf, g, n = layer._guarded[0]
+    buf[g + n] = 0           # one byte past the end
+    with pytest.raises(RuntimeError):
+        layer.check_guards()
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from _moe_util import guarded_empty
+    t, check = guarded_empty((3, 5), torch.float32, "cpu")
+    t.fill_(1.0)
+    check()
+    raw = torch.tensor([], dtype=torch.uint8).set_(t.untyped_storage())
+    raw[0] = 0               # first byte of the leading band
+    with pytest.raises(AssertionError):
+        check()

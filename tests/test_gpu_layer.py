@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import moe_synth as S
-from _moe_util import NEAR_TIE, STATED_NEAR_TIE, Problem, assert_close, bf16_to_f64, oracle_cfg, route_sets_match, shape_of
+from _moe_util import GUARD, NEAR_TIE, STATED_NEAR_TIE, Problem, assert_close, guarded_empty, bf16_to_f64, oracle_cfg, route_sets_match, shape_of
 
 pytestmark = pytest.mark.gpu
 
@@ -28,6 +28,7 @@ def m():
 def build_gpu_layer(m, prob: Problem):
     shape = shape_of(prob.cfg)
     layer = m.MoeLayer(shape, "cuda")
+    layer.guard_bytes = GUARD  # guard bands around every workspace, checked by check_layer
     for e in range(prob.E):
         w13, w2 = prob.expert_bf16(e)
         layer.set_expert(e, w13.cuda(), w2.cuda())
@@ -42,10 +43,15 @@ def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts
     H, I, Nr, Kr, Ns = cfg["H"], cfg["I"], cfg["Nr"], cfg["Kr"], cfg.get("Ns", 1)
     R = T * Kr
     x_d = prob.x.to("cuda")
-    counts_out = torch.empty(Nr, dtype=torch.int32, device="cuda")
-    idx_out = torch.empty((T, Kr), dtype=torch.int32, device="cuda")
-    out32 = layer.forward(x_d, out_dtype=m.MOE_DTYPE_F32, idx_out=idx_out, counts_out=counts_out)
+    counts_out, chk_c = guarded_empty((Nr,), torch.int32)
+    idx_out, chk_i = guarded_empty((T, Kr), torch.int32)
+    out32, chk_o = guarded_empty((T, H), torch.float32)
+    layer.forward(x_d, out=out32, out_dtype=m.MOE_DTYPE_F32, idx_out=idx_out, counts_out=counts_out)
     layer.check()
+    for chk in (chk_c, chk_i, chk_o):
+        chk()
+    if getattr(layer, "guard_bytes", 0):
+        layer.check_guards()
     ws = layer.workspace(T)
     L = layer.layout(T)
     v = lambda name, dt, shp: m.ws_view(ws, L, name, dt, shp).cpu().numpy()  # noqa: E731

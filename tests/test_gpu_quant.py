@@ -36,6 +36,11 @@ def test_1x128_special_tiles(m, oracle_lib):
     x[7, 256:384] = 3.0e4                  # constant tile
     x[9, 0] = -x[9, 0].abs() * 1000        # negative outlier
     x[11, 5] = -0.0
+    # scales near and below the quantizer's switch from the reciprocal path to
+    # the plain division (S < 2^-100): amax around 2^-91 .. 2^-125, bf16
+    # subnormals included
+    for i, e in enumerate((-91, -92, -100, -110, -120, -125, -130)):
+        x[13 + i, 384:512] = (x[13 + i, 384:512].float() * 2.0 ** e).to(torch.bfloat16)
     _check_1x128(m, oracle_lib, x)
 
 
