@@ -586,7 +586,8 @@ static void ep_dispatch_layout(int32_t world, int64_t T, size_t *cnt_off, size_t
 }
 
 size_t moe_ep_dispatch_workspace_size(const moe_config *cfg, int32_t world, int64_t T) {
-  if (check_cfg(cfg) != MOE_OK || world < 1 || world > 64 || T < 0 || T > kMaxTokens) return 0;
+  if (check_cfg(cfg) != MOE_OK || world < 1 || world > 64 || cfg->n_routed % world || T < 0 || T > kMaxTokens)
+    return 0;
   size_t c, b, tot;
   ep_dispatch_layout(world, T, &c, &b, &tot);
   return tot < 256 ? 256 : tot;

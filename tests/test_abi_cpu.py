@@ -167,3 +167,50 @@ def test_workspace_guard_bands_catch_overruns(m):
     raw[0] = 0               # first byte of the leading band
     with pytest.raises(AssertionError):
         check()
+
+
+def test_expert_parallel_entry_points_validate_on_the_host(m):
+    import ctypes as C
+    L = m.lib
+    cfg = m.config(512, 256, 16, 4)
+    # packed row: H codes, H/128 scales, K_r slots and K_r gates, padded to 16 bytes
+    assert m.moe_ep_row_bytes(cfg) == (512 + 4 * 4 + 8 * 4 + 15) // 16 * 16
+    assert m.moe_ep_row_bytes(m.config(7168, 2048, 256, 8)) == 7168 + 224 + 64
+    assert m.moe_ep_row_bytes(m.config(7168, 2000, 256, 8)) == 0        # invalid shape
+    assert L.moe_ep_dispatch_workspace_size(C.byref(cfg), 3, 64) == 0    # 16 experts do not split over 3 ranks
+    assert L.moe_ep_dispatch_workspace_size(C.byref(cfg), 4, 64) >= 256
+    # world that does not divide the experts; too small a send capacity
+    assert L.moe_ep_dispatch(C.byref(cfg), 3, 16, 16, 16, 16, 8, 16, 64, 16, 16, 16, None, 256, 1 << 20, 16,
+                             None) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_dispatch(C.byref(cfg), 4, 16, 16, 16, 16, 8, 16, 31, 16, 16, 16, None, 256, 1 << 20, 16,
+                             None) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_dispatch(C.byref(cfg), 4, 16, 16, 16, 16, 8, 16, 32, 16, 16, 16, None, 256, 1 << 20, 16,
+                             None) == m.MOE_ERR_NO_DEVICE
+    # the experts' side takes no shared expert and the layer's packed row only
+    loc = m.config(512, 256, 4, 4, 0)
+    rb = m.moe_ep_row_bytes(loc)
+    w = m.MoeWeights(16, 16, 16, 16, None)
+    assert L.moe_ep_experts(C.byref(m.config(512, 256, 4, 4, 1)), C.byref(w), 16, 8, rb, 16, 256, 1 << 30, 16,
+                            None) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_experts(C.byref(loc), C.byref(w), 16, 8, rb + 16, 16, 256, 1 << 30, 16, None) == \
+        m.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_experts(C.byref(loc), C.byref(w), 16, 8, rb, 16, 256, 1 << 30, 16, None) == m.MOE_ERR_NO_DEVICE
+    assert L.moe_ep_combine(C.byref(cfg), 0, 16, 8, 16, 16, None, 16, 0, None) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_combine(C.byref(cfg), 2, 16, 8, 16, 16, None, 16, 0, None) == m.MOE_ERR_NO_DEVICE
+
+
+def test_backward_entry_points_validate_on_the_host(m):
+    import ctypes as C
+    L = m.lib
+    cfg = m.config(512, 256, 16, 4)
+    assert L.moe_backward_workspace_size(C.byref(cfg), 64) > 0
+    assert L.moe_backward_workspace_size(C.byref(m.config(512, 200, 16, 4)), 64) == 0
+    w = m.MoeWeights(16, 16, 16, 16, 16)
+    args = (16, 16, 16, 16, 16, 16, 64, 16, 16, 16, 256, 1 << 30, 256, 1 << 33, 16, None)
+    pow2 = m.config(512, 256, 16, 4, scale_mode=m.MOE_SCALE_POW2)
+    assert L.moe_backward(C.byref(pow2), C.byref(w), *args) == m.MOE_ERR_NOT_IMPLEMENTED
+    assert L.moe_backward(C.byref(cfg), C.byref(w), *args[:6], 0, *args[7:]) == m.MOE_ERR_INVALID_ARG  # T = 0
+    small = args[:11] + (1024,) + args[12:]   # forward workspace too small
+    assert L.moe_backward(C.byref(cfg), C.byref(w), *small) == m.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert L.moe_backward(C.byref(cfg), C.byref(w), *args) == m.MOE_ERR_NO_DEVICE
+    assert L.moe_transpose_weights(C.byref(cfg), C.byref(w), 16, 16, 16, 16, None) == m.MOE_ERR_NO_DEVICE
