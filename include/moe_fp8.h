@@ -237,9 +237,8 @@ MOE_API int moe_route_noalloc(const moe_config *cfg, const void *x_dev, const vo
  * GEMM: u quantized 1x128 (fp8_quant_1x128), routed as moe_route, rows
  * grouped per expert (stable: token order, then slot), h = silu(G) * U in FP32
  * re-quantized 1x128 along I before the down projection, the down-projection
- * output scaled by the gate (in FP32, then stored as bf16), then summed per
- * token in FP32 in a fixed order (residual, shared expert, slots 0..K_r-1)
- * and written as out_dtype.
+ * output scaled by the gate (FP32), then summed per token in FP32 in a fixed
+ * order (residual, shared expert, slots 0..K_r-1) and written as out_dtype.
  *   x_dev        bf16 [T, H]
  *   out_dev      [T, H] of MOE_DTYPE_BF16 (RNE) or MOE_DTYPE_F32
  *   idx_out_dev  nullable int32 [T, K_r]: routing decision
@@ -272,9 +271,7 @@ typedef struct {
     size_t row_src[2];  /* int32 [R]        token of each routed row           */
     size_t hq[2];       /* E4M3 [R + T*N_s, I] re-quantized SwiGLU output      */
     size_t hs[2];       /* float [I/128, P] its scales, transposed             */
-    size_t y[2];        /* bf16 [R + T*N_s, H] gate-scaled expert outputs
-                           (RNE of the FP32 product of the down projection
-                           and the gate)                                       */
+    size_t y[2];        /* float [R + T*N_s, H] gate-scaled expert outputs     */
     size_t meta[2];     /* int32 [4]: number of chunks, routed rows            */
     size_t logits[2];   /* float [S, T, N_r] router logit partials (S K-splits) */
     size_t blk_hist[2]; /* int32 [ceil(T/128), N_r] per-block expert counts    */
@@ -335,6 +332,17 @@ MOE_API int moe_profile_events(void *const *events, int32_t n_events);
 MOE_API int moe_transpose_weights(const moe_config *cfg, const moe_weights *w, uint8_t *w13t_dev, float *s13t_dev,
                                   uint8_t *w2t_dev, float *s2t_dev, void *stream);
 MOE_API size_t moe_backward_workspace_size(const moe_config *cfg, int64_t T);
+/* Byte offsets {offset, bytes} of the backward's intermediates inside its
+ * workspace (for tests and inspection), rows in the forward's row order
+ * (RS = T*K_r + T*N_s): gu float [RS, 2I] (G then U), dh and h float [RS, I],
+ * dgu float [RS, 2I] (dG then dU), dx_rows float [RS, H], seg int32 [E + 1]
+ * (each expert's token segment of the weight-gradient operands, P columns). */
+typedef struct {
+    size_t gu[2], dh[2], h[2], dgu[2], dx_rows[2], seg[2];
+    int64_t P;
+    size_t total;
+} moe_bwd_layout;
+MOE_API int moe_backward_workspace_layout(const moe_config *cfg, int64_t T, moe_bwd_layout *layout);
 MOE_API int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13t_dev,
                          const float *s13t_dev, const uint8_t *w2t_dev, const float *s2t_dev, const void *x_dev,
                          const void *dout_dev, int64_t T, float *dx_dev, float *dW13_dev, float *dW2_dev,
@@ -395,8 +403,9 @@ MOE_API int moe_ep_dispatch(const moe_config *cfg, int32_t world, const uint8_t 
 
 /* The experts of one rank over received packed rows (steps 4 and 6).
  *   cfg_local     n_routed = the rank's experts (N_r / W, or 1 for the
- *                 shared expert), top_k = the layer's K_r, n_shared = 0,
- *                 other fields as the layer's
+ *                 shared expert), top_k = the layer's K_r (the slots of a
+ *                 packed row; it may exceed n_routed), n_shared = 0,
+ *                 n_groups = 0, other fields as the layer's
  *   w_local       those experts' weights (layout of moe_weights; wr_dev unused)
  *   rows_dev      n_rows packed rows, row_bytes = moe_ep_row_bytes(cfg_local)
  *   partial_out_dev bf16 [n_rows, H]: per row, the sum over its slots of

@@ -45,6 +45,7 @@ EXPORTS = (
     "moe_route_noalloc", "moe_seq_balance_loss", "moe_set_gemm_variant",
     "moe_ep_row_bytes", "moe_ep_dispatch_workspace_size", "moe_ep_dispatch", "moe_ep_experts_workspace_size",
     "moe_ep_experts", "moe_ep_combine", "moe_transpose_weights", "moe_backward_workspace_size", "moe_backward",
+    "moe_backward_workspace_layout",
 )
 MOE_GEMM_AUTO = 0
 MOE_GEMM_SINGLE = 1
@@ -108,6 +109,12 @@ lib.moe_ep_experts_workspace_size.argtypes = [_cfgp, _i64]
 lib.moe_ep_experts.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _i64, _i64, _vp, _vp, _sz, _vp, _vp]
 lib.moe_ep_combine.argtypes = [_cfgp, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _i32, _vp]
 lib.moe_transpose_weights.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _vp, _vp, _vp, _vp]
+class MoeBwdLayout(C.Structure):
+    _fields_ = [(f, C.c_size_t * 2) for f in ("gu", "dh", "h", "dgu", "dx_rows", "seg")] + [("P", C.c_int64),
+                                                                                          ("total", C.c_size_t)]
+
+
+lib.moe_backward_workspace_layout.argtypes = [_cfgp, _i64, C.POINTER(MoeBwdLayout)]
 lib.moe_backward_workspace_size.restype = _sz
 lib.moe_backward_workspace_size.argtypes = [_cfgp, _i64]
 lib.moe_backward.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
@@ -341,6 +348,18 @@ def moe_transpose_weights(cfg: MoeConfig, w: dict, stream=None) -> dict:
     _check(lib.moe_transpose_weights(C.byref(cfg), C.byref(ws), _ptr(t["w13t"]), _ptr(t["s13t"]), _ptr(t["w2t"]),
                                      _ptr(t["s2t"]), _stream(stream)), "moe_transpose_weights")
     return t
+
+
+def ctypes_cfg(cfg: MoeConfig):
+    return C.byref(cfg)
+
+
+def moe_backward_workspace_layout(cfg: MoeConfig, T: int) -> dict:
+    L = MoeBwdLayout()
+    _check(lib.moe_backward_workspace_layout(C.byref(cfg), T, C.byref(L)), "moe_backward_workspace_layout")
+    d = {f: (int(getattr(L, f)[0]), int(getattr(L, f)[1])) for f in ("gu", "dh", "h", "dgu", "dx_rows", "seg")}
+    d["P"], d["total"] = int(L.P), int(L.total)
+    return d
 
 
 def moe_backward(cfg: MoeConfig, w: dict, wt: dict, x, dout, fwd_ws, dx=None, dW13=None, dW2=None, ws=None,

@@ -108,6 +108,18 @@ int check_cfg(const moe_config *c) {
   return MOE_OK;
 }
 
+// The expert side of expert parallelism: top_k counts the slots of a packed
+// row, which may exceed the rank's own experts (a slot whose expert lives
+// elsewhere is -1); no routing groups, no shared expert.
+int check_cfg_local(const moe_config *c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->top_k < 1 || c->top_k > 16 || c->n_routed < 1) return c->top_k > 16 ? MOE_ERR_UNSUPPORTED_SHAPE : MOE_ERR_INVALID_ARG;
+  if (c->n_shared != 0 || c->n_groups != 0) return MOE_ERR_INVALID_ARG;
+  moe_config t = *c;
+  t.top_k = 1;  // the rest of the checks as for a layer
+  return check_cfg(&t);
+}
+
 constexpr int64_t kMaxTokens = 1 << 20;
 
 // The grouped GEMMs of the default scale mode run on single CTAs; with
@@ -151,7 +163,7 @@ void make_layout(const moe_config *c, int64_t T, moe_ws_layout *L) {
   cv.take(L->row_src, R * 4);
   cv.take(L->hq, RS * I);
   cv.take(L->hs, ((I / 128) * pitch + moe::kScaleSlack) * 4);
-  cv.take(L->y, RS * H * 2);
+  cv.take(L->y, RS * H * 4);
   cv.take(L->meta, 4 * 4);
   cv.take(L->logits, ks * T * Nr * 4);
   cv.take(L->blk_hist, nblk * Nr * 4);
@@ -403,7 +415,7 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
   int32_t *row_src = at<int32_t *>(ws, L.row_src);
   uint8_t *hq = at<uint8_t *>(ws, L.hq);
   float *hs_t = at<float *>(ws, L.hs);
-  __nv_bfloat16 *y = at<__nv_bfloat16 *>(ws, L.y);
+  float *y = at<float *>(ws, L.y);
   int32_t *meta = at<int32_t *>(ws, L.meta);
   int32_t *blk_hist = at<int32_t *>(ws, L.blk_hist);
   int32_t *blk_base = at<int32_t *>(ws, L.blk_base);
@@ -480,7 +492,7 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
     g.gate_up = 0;
     g.a_is_out_row = 1;
     g.rows_per_expert = H;
-    g.epi = moe::EPI_GATE_BF16;
+    g.epi = moe::EPI_GATE_F32;
     g.out = y;
     g.ldo = H;
     g.out_rows = RS;
@@ -491,7 +503,7 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
     e = pow2 ? moe::launch_gemm_mx(g, st) : pair ? moe::launch_gemm_pair(g, st) : moe::launch_gemm(g, st);
   }
   if (e == cudaSuccess) e = prof_mark(5, st);
-  if (e == cudaSuccess) e = moe::launch_combine(P.x_resid, y, pos, T, H, Kr, R, Ns, P.out, P.out_f32, st);
+  if (e == cudaSuccess) e = moe::launch_combine(P.x_resid, y, pos, T, H, Kr, R, Ns, P.out, P.out_f32, st, true);
   if (e == cudaSuccess) e = prof_mark(6, st);
   return e;
 }
@@ -620,7 +632,7 @@ int moe_ep_dispatch(const moe_config *cfg, int32_t world, const uint8_t *xq, con
 }
 
 size_t moe_ep_experts_workspace_size(const moe_config *cfg_local, int64_t n_rows) {
-  if (check_cfg(cfg_local) != MOE_OK || cfg_local->n_shared != 0 || n_rows < 0 || n_rows > kMaxTokens) return 0;
+  if (check_cfg_local(cfg_local) != MOE_OK || n_rows < 0 || n_rows > kMaxTokens) return 0;
   moe_ws_layout L;
   make_layout(cfg_local, n_rows, &L);
   return L.total < 256 ? 256 : L.total;
@@ -628,10 +640,10 @@ size_t moe_ep_experts_workspace_size(const moe_config *cfg_local, int64_t n_rows
 
 int moe_ep_experts(const moe_config *cfg_local, const moe_weights *w_local, const uint8_t *rows, int64_t n_rows,
                    int64_t row_bytes, void *partial_out, void *ws, size_t ws_bytes, int32_t *err_flag, void *stream) {
-  if (const int c = check_cfg(cfg_local)) return c;
-  if (cfg_local->n_shared != 0) return MOE_ERR_INVALID_ARG;
+  if (const int c = check_cfg_local(cfg_local)) return c;
   if (n_rows < 0 || n_rows > kMaxTokens) return MOE_ERR_INVALID_ARG;
-  if (row_bytes != moe_ep_row_bytes(cfg_local)) return MOE_ERR_INVALID_ARG;
+  const int64_t H = cfg_local->hidden, Kr = cfg_local->top_k;
+  if (row_bytes != (H + 4 * (H / 128) + 8 * Kr + 15) / 16 * 16) return MOE_ERR_INVALID_ARG;
   if (n_rows == 0) return MOE_OK;
   if (!w_local || !rows || !partial_out || !ws || !err_flag) return MOE_ERR_INVALID_ARG;
   if (!w_local->w13_dev || !w_local->s13_dev || !w_local->w2_dev || !w_local->s2_dev) return MOE_ERR_INVALID_ARG;
@@ -747,6 +759,26 @@ int moe_transpose_weights(const moe_config *cfg, const moe_weights *w, uint8_t *
   cudaError_t e = moe::launch_transpose_blocks(w->w13_dev, w->s13_dev, 2 * I, H, E, w13t, s13t, st);
   if (e == cudaSuccess) e = moe::launch_transpose_blocks(w->w2_dev, w->s2_dev, H, I, E, w2t, s2t, st);
   return cuda_status(e);
+}
+
+int moe_backward_workspace_layout(const moe_config *cfg, int64_t T, moe_bwd_layout *out) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (T < 0 || T > kMaxTokens || !out) return MOE_ERR_INVALID_ARG;
+  BwdLayout B;
+  make_bwd_layout(cfg, T, &B);
+  auto cp = [](size_t (&d)[2], const size_t (&s_)[2]) {
+    d[0] = s_[0];
+    d[1] = s_[1];
+  };
+  cp(out->gu, B.gu);
+  cp(out->dh, B.dh);
+  cp(out->h, B.h);
+  cp(out->dgu, B.dgu);
+  cp(out->dx_rows, B.dxr);
+  cp(out->seg, B.seg);
+  out->P = B.P;
+  out->total = B.total;
+  return MOE_OK;
 }
 
 size_t moe_backward_workspace_size(const moe_config *cfg, int64_t T) {

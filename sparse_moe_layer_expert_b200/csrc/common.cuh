@@ -304,14 +304,16 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 }
 
 // Arrive on an mbarrier given by its shared::cluster address (this CTA's or
-// another CTA's of the cluster), releasing this thread's prior writes at
-// cluster scope.
+// another CTA's of the cluster) with the default release semantics at CTA
+// scope.  These arrivals carry no generic-memory data between the CTAs: they
+// order TMEM reads (with the tcgen05 fences around them) and count TMA bytes,
+// so no cluster-wide fence is needed -- and one costs about a microsecond on
+// the critical path of the pair GEMM.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t caddr, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(caddr), "r"(bytes)
-               : "memory");
+  asm volatile("mbarrier.arrive.expect_tx.shared::cluster.b64 _, [%0], %1;" ::"r"(caddr), "r"(bytes) : "memory");
 }
 
 // Barrier over every thread of the cluster (all threads of both CTAs of a

@@ -30,7 +30,7 @@
 //                 (amax of the row's two 64-channel halves exchanged between
 //                 the warpgroups, S = amax / 448, E4M3 RNE), 64 codes per
 //                 thread stored as 16-byte vectors -> hq, scale -> hs
-//   EPI_GATE_BF16 y = bf16(acc * gate[row]) (down projection)
+//   EPI_GATE_F32  y = acc * gate[row] in FP32 (down projection)
 //   EPI_BF16      C = bf16(acc) (plain GEMM)
 //   EPI_F32       C = acc in FP32 (the backward's recomputed G, U and dh)
 //
@@ -369,7 +369,7 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st) {
   const int grid = static_cast<int>(max_tiles < sms ? max_tiles : sms);
   switch (g.epi) {
     case EPI_SWIGLU_Q: return launch_epi<EPI_SWIGLU_Q>(mw, m0, m1, a, grid, st);
-    case EPI_GATE_BF16: return launch_epi<EPI_GATE_BF16>(mw, m0, m1, a, grid, st);
+    case EPI_GATE_F32: return launch_epi<EPI_GATE_F32>(mw, m0, m1, a, grid, st);
     case EPI_F32: return launch_epi<EPI_F32>(mw, m0, m1, a, grid, st);
     default: return launch_epi<EPI_BF16>(mw, m0, m1, a, grid, st);
   }

@@ -377,7 +377,7 @@ static cudaError_t launch_mx(const CUtensorMap &mw, const CUtensorMap &m0, const
 // the activation scales stored transposed (the layer's tables).
 cudaError_t launch_gemm_mx(const GemmLaunch &g, cudaStream_t st) {
   if (g.max_chunks <= 0 || g.nb <= 0) return cudaSuccess;
-  if (!g.sa_transposed || !g.chunks || (g.epi != EPI_SWIGLU_Q && g.epi != EPI_GATE_BF16))
+  if (!g.sa_transposed || !g.chunks || (g.epi != EPI_SWIGLU_Q && g.epi != EPI_GATE_F32))
     return cudaErrorInvalidValue;
   CUtensorMap mw, m0, m1;
   const uint64_t K = static_cast<uint64_t>(g.K);
@@ -393,7 +393,7 @@ cudaError_t launch_gemm_mx(const GemmLaunch &g, cudaStream_t st) {
   const int64_t max_tiles = static_cast<int64_t>(g.max_chunks) * g.nb;
   const int grid = static_cast<int>(max_tiles < sms ? max_tiles : sms);
   return g.epi == EPI_SWIGLU_Q ? launch_mx<EPI_SWIGLU_Q>(mw, m0, m1, a, grid, st)
-                               : launch_mx<EPI_GATE_BF16>(mw, m0, m1, a, grid, st);
+                               : launch_mx<EPI_GATE_F32>(mw, m0, m1, a, grid, st);
 }
 
 }  // namespace moe

@@ -419,7 +419,7 @@ cudaError_t launch_gemm_pair(const GemmLaunch &g, cudaStream_t st) {
   const int64_t max_tiles = static_cast<int64_t>(g.max_chunks) * g.nb;
   switch (g.epi) {
     case EPI_SWIGLU_Q: return launch_pair_epi<EPI_SWIGLU_Q>(mw, m0, m1, a, max_tiles, st);
-    case EPI_GATE_BF16: return launch_pair_epi<EPI_GATE_BF16>(mw, m0, m1, a, max_tiles, st);
+    case EPI_GATE_F32: return launch_pair_epi<EPI_GATE_F32>(mw, m0, m1, a, max_tiles, st);
     default: return launch_pair_epi<EPI_BF16>(mw, m0, m1, a, max_tiles, st);
   }
 }

@@ -98,8 +98,7 @@ __device__ __forceinline__ bool tile_ok(const GemmArgs &a, const GemmTile &d) {
 //                 the warpgroups through amx; S = amax / 448, or the power-of-
 //                 two scale when POW2; E4M3 RNE), 64 codes per thread stored
 //                 as 16-byte vectors -> hq, scale -> hs
-//   EPI_GATE_BF16 y = bf16(acc * gate[row]) (down projection; the product in
-//                 FP32, rounded to nearest even)
+//   EPI_GATE_F32  y = acc * gate[row] in FP32 (down projection)
 //   EPI_BF16      C = bf16(acc) (plain GEMM)
 //   EPI_F32       C = acc in FP32 (block B at +128 columns, or at +half for a
 //                 gate/up pair)
@@ -159,12 +158,14 @@ __device__ __forceinline__ void tile_epilogue(const GemmArgs &args, const GemmTi
       if (wg == 0) args.out_scale[static_cast<int64_t>(td.out_col / 128) * args.ld_os + orow] = S;
     }
     named_bar_sync(1, 256);  // amx is reused by the next tile
-  } else if constexpr (EPI == EPI_F32) {
-    // FP32 results of both blocks; block B's columns follow block A's (+128),
-    // or start at +half when the pair is gate block j / up block j
+  } else if constexpr (EPI == EPI_F32 || EPI == EPI_GATE_F32) {
+    // FP32 results of both blocks (times the row's gate for EPI_GATE_F32);
+    // block B's columns follow block A's (+128), or start at +half when the
+    // pair is gate block j / up block j
     float *xb = outx + (warp - 4) * (32 * G_OPITCH);
     const int rbase = q * 32;
     const int64_t cB = args.gate_up ? args.half : 128;
+    const float g = (EPI == EPI_GATE_F32 && valid) ? __ldg(args.row_gate + orow) : 1.0f;
     auto emit = [&](const float(&acc)[64], int64_t cbase) {
 #pragma unroll
       for (int piece = 0; piece < 4; ++piece) {
@@ -172,7 +173,7 @@ __device__ __forceinline__ void tile_epilogue(const GemmArgs &args, const GemmTi
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const int j = piece * 16 + 4 * v;
-          dst[v] = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+          dst[v] = make_float4(acc[j] * g, acc[j + 1] * g, acc[j + 2] * g, acc[j + 3] * g);
         }
         __syncwarp();
 #pragma unroll
@@ -196,7 +197,6 @@ __device__ __forceinline__ void tile_epilogue(const GemmArgs &args, const GemmTi
     // contiguous bytes instead of 32 scattered rows.
     float *xb = outx + (warp - 4) * (32 * G_OPITCH);
     const int rbase = q * 32;  // this warp's first row in the tile
-    const float g = (EPI == EPI_GATE_BF16 && valid) ? __ldg(args.row_gate + orow) : 1.0f;
     auto emit = [&](const float(&acc)[64], int b) {
 #pragma unroll
       for (int piece = 0; piece < 2; ++piece) {
@@ -208,8 +208,7 @@ __device__ __forceinline__ void tile_epilogue(const GemmArgs &args, const GemmTi
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int j = piece * 32 + 8 * v + 2 * k;
-            const __nv_bfloat162 b2 = EPI == EPI_GATE_BF16 ? __floats2bfloat162_rn(acc[j] * g, acc[j + 1] * g)
-                                                           : __floats2bfloat162_rn(acc[j], acc[j + 1]);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[j], acc[j + 1]);
             f[k] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&b2));
           }
           dst[v] = make_float4(f[0], f[1], f[2], f[3]);

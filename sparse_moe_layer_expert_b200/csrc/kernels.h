@@ -38,7 +38,7 @@ struct GemmTile {
   int32_t pad;
 };
 
-enum EpiKind : int { EPI_SWIGLU_Q = 0, EPI_GATE_BF16 = 1, EPI_BF16 = 2, EPI_F32 = 3 };
+enum EpiKind : int { EPI_SWIGLU_Q = 0, EPI_GATE_F32 = 1, EPI_BF16 = 2, EPI_F32 = 3 };
 
 struct GemmLaunch {
   // tensor operands
@@ -123,7 +123,7 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st);
 cudaError_t launch_gemm_pair(const GemmLaunch &g, cudaStream_t st);
 // The same grouped GEMM with power-of-two scales applied by the tensor core
 // (block-scaled MMA); transposed activation scales, EPI_SWIGLU_Q (with
-// power-of-two requantization) or EPI_GATE_BF16 only.
+// power-of-two requantization) or EPI_GATE_F32 only.
 cudaError_t launch_gemm_mx(const GemmLaunch &g, cudaStream_t st);
 
 // out[t] = x[t] (when x is not null) + y[R + t] (when Ns) + sum_k y[pos[t, k]]

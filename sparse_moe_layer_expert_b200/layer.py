@@ -123,8 +123,19 @@ class MoeLayer:
         if getattr(self, "_wt", None) is None:
             self._wt = B.moe_transpose_weights(self.cfg, self.weights(), stream=stream)
         T = x.shape[0]
-        return B.moe_backward(self.cfg, self.weights(), self._wt, x, dout, self.workspace(T), err=self.err,
-                              stream=stream)
+        return B.moe_backward(self.cfg, self.weights(), self._wt, x, dout, self.workspace(T),
+                              ws=self.backward_workspace(T), err=self.err, stream=stream)
+
+    def backward_workspace(self, T: int) -> torch.Tensor:
+        bws = getattr(self, "_bws", None)
+        if bws is None:
+            bws = self._bws = {}
+        ws = bws.get(T)
+        if ws is None:
+            ws = torch.empty(max(int(B.lib.moe_backward_workspace_size(B.ctypes_cfg(self.cfg), T)), 256),
+                             dtype=torch.uint8, device=self.device)
+            bws[T] = ws
+        return ws
 
     def check(self, stream=None) -> None:
         st, v = B.moe_check_device_error(self.err, stream)

@@ -114,7 +114,7 @@ def test_workspace_layout_is_disjoint_and_aligned(m):
             assert o1 + n1 <= o2
         assert spans[-1][0] + spans[-1][1] <= L["total"] == m.moe_workspace_size(cfg, T)
         R = T * Kr
-        assert L["ap"][1] == R * H and L["y"][1] == (R + T) * H * 2 and L["hq"][1] == (R + T) * I
+        assert L["ap"][1] == R * H and L["y"][1] == (R + T) * H * 4 and L["hq"][1] == (R + T) * I
 
 
 def test_route_workspace_size(m):

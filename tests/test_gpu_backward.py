@@ -45,11 +45,66 @@ def run_backward_case(m, oracle_lib, cfg, T, seed, bias_shift=None, tokens_check
     got_idx = idx_out.cpu().numpy()
     for t in range(T):
         assert set(got_idx[t].tolist()) == set(ref["idx"][t].tolist()), t
+    H, I, Kr, Ns = cfg["H"], cfg["I"], cfg["Kr"], cfg.get("Ns", 1)
+    R, E = T * Kr, prob.E
+    RS = R + T * Ns
+    # the backward's own intermediates, step by step against the oracle's
+    # expert backward on the same tokens
+    bws, BL = layer.backward_workspace(T), m.moe_backward_workspace_layout(layer.cfg, T)
+
+    def view(name, shape):
+        off, nb = BL[name]
+        n = int(np.prod(shape))
+        assert n * 4 <= nb
+        return bws[off:off + 4 * n].view(torch.float32).view(shape).cpu().numpy().astype(np.float64)
+
+    GU, dh, hh, dGU = view("gu", (RS, 2 * I)), view("dh", (RS, I)), view("h", (RS, I)), view("dgu", (RS, 2 * I))
+    ws, L = layer.workspace(T), layer.layout(T)
+    offsets = m.ws_view(ws, L, "offsets", torch.int32, (cfg["Nr"] + 1,)).cpu().numpy()
+    xu = prob.x
+    d32 = dout.float().numpy()
+    msgs, fails = [], []
+    for e in sorted(ref["dW13"].keys()):
+        if e < cfg["Nr"]:
+            toks, slots = np.nonzero(ref["idx"] == e)
+            order = np.argsort(toks, kind="stable")
+            toks, slots = toks[order], slots[order]
+            rows = np.arange(offsets[e], offsets[e + 1])
+            dy = (ref["gate"][toks, slots].astype(np.float32)[:, None] * d32[toks]).astype(np.float32)
+        else:
+            toks = np.arange(T)
+            rows = R + toks
+            dy = d32
+        r = OB.expert_backward(xu[torch.as_tensor(toks)], dy, *experts[e])
+        for nm, got, want in (("G", GU[rows, :I], r["G"]), ("U", GU[rows, I:], r["U"]), ("dh", dh[rows], r["dh"]),
+                              ("h", hh[rows], r["h"]), ("dG", dGU[rows, :I], r["dG"]),
+                              ("dU", dGU[rows, I:], r["dU"])):
+            rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+            msgs.append(f"expert {e} {nm}: rel-Frobenius {rel:.2e}")
+            if not rel < 1e-4:
+                fails.append(msgs[-1])
+        # the weight-gradient GEMM on the GPU's own operands (its dY, h, dG|dU
+        # and x), quantized 128x1 by the oracle: only the GEMM's FP32 rounding
+        # separates the two
+        dyq, dys = OB.quant_128x1_f32(dy)
+        hq, hs = OB.quant_128x1_f32(hh[rows].astype(np.float32))
+        w2_own = OB.rows_scaled_gemm(dyq.T, dys.T, hq.T, hs.T)
+        gq, gs = OB.quant_128x1_f32(dGU[rows].astype(np.float32))
+        xq, xs = OB.quant_128x1_bf16(xu[torch.as_tensor(toks)])
+        w13_own = OB.rows_scaled_gemm(gq.T, gs.T, xq.T, xs.T)
+        got13, got2 = dW13[e].cpu().numpy().astype(np.float64), dW2[e].cpu().numpy().astype(np.float64)
+        for nm, got, want in (("dW13 (own operands)", got13, w13_own), ("dW2 (own operands)", got2, w2_own)):
+            rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+            msgs.append(f"expert {e} {nm}: rel-Frobenius {rel:.2e}")
+            if not rel < 1e-5:
+                fails.append(msgs[-1])
+    print("\n".join(msgs[:60]))
+    assert not fails, fails[:10]
     dx_h = dx.cpu().numpy().astype(np.float64)
     assert_close(dx_h, ref["dx"], what="dx")
     dW13_h, dW2_h = dW13.cpu().numpy(), dW2.cpu().numpy()
     used = set(ref["dW13"].keys())
-    for e in range(prob.E):
+    for e in range(E):
         if e in used:
             assert_close(dW13_h[e].astype(np.float64), ref["dW13"][e], what=f"dW13 of expert {e}")
             assert_close(dW2_h[e].astype(np.float64), ref["dW2"][e], what=f"dW2 of expert {e}")

@@ -21,7 +21,14 @@ def _check_1x128(m, oracle_lib, x_cpu):
     q, s = m.fp8_quant_1x128(x_cpu.cuda())
     torch.cuda.synchronize()
     qo, so = oracle_lib.quant_1x128(x_cpu)
-    assert np.array_equal(q.cpu().numpy(), qo)
+    qg = q.cpu().numpy()
+    if not np.array_equal(qg, qo):
+        r, c = np.nonzero(qg != qo)
+        sg = s.cpu().numpy()
+        xs = x_cpu.float().numpy()
+        print("codes differ at", [(int(i), int(j), float(xs[i, j]), int(qg[i, j]), int(qo[i, j]),
+                                   float(sg[i, j // 128]), float(so[i, j // 128])) for i, j in zip(r[:12], c[:12])])
+    assert np.array_equal(qg, qo)
     assert np.array_equal(s.cpu().numpy(), so)
 
 
