@@ -23,13 +23,20 @@ orientation is a reading (the DeepSeek-V3 technical report's recipe):
   rounded to FP32.
 
 For one expert with input x [rows, H] (bf16), weights W1, W3 [I, H] and
-W2 [H, I] (E4M3 codes with 128x128 block scales) and the gradient dY of its
-output [rows, H] (bf16; for a routed expert the caller folds in the gate):
+W2 [H, I] (E4M3 codes with 128x128 block scales), the layer-output gradient
+D of its rows [rows, H] (bf16) and the rows' gates g (1 for the shared
+expert), the expert's output gradient is dY = g D:
     G = x W1^T, U = x W3^T, h = silu(G) * U, Y = h W2^T       (forward)
-    dh  = dY W2                    dW2 = dY^T h
+    dh  = g (D W2)                 dW2 = D^T (g h)
     dG  = dh * U * silu'(G)        dU  = dh * silu(G)
     dx  = dG W1 + dU W3            dW1 = dG^T x,   dW3 = dU^T x
 with silu(G) = G sigma(G) and silu'(G) = sigma(G) (1 + G (1 - sigma(G))).
+Where the gate sits is a reading.  For the dgrad, 1x128 tiles of g D along H
+have the codes of D's tiles (g cancels in x / (amax / 448)), so D is
+quantized and g scales the FP32 product: the exact-arithmetic result of
+quantizing g D, without the rounding of g D deciding codes.  For the wgrad
+(128x1 tiles along tokens, different gates in one tile) g rides on h, an
+FP32 intermediate already: D^T (g h) = (g D)^T h.
 The gate's own gradient (router backward) is not part of this.
 """
 from __future__ import annotations
@@ -99,22 +106,26 @@ def _as_f32_values(a) -> np.ndarray:
     return np.ascontiguousarray(u.view(np.float32))
 
 
-def expert_backward(x, dy, W13q, s13, W2q, s2, mode: int = SCALE_AMAX) -> dict:
+def expert_backward(x, dy, W13q, s13, W2q, s2, gate=None, mode: int = SCALE_AMAX) -> dict:
     """Backward of one expert FFN under the FP8 recipe above.
 
     x: bf16 [rows, H] (torch bf16 tensor or uint16 bit patterns); dy: the
-    gradient of the expert's output [rows, H], bf16 as x or float32 values;
+    layer-output gradient D of the rows [rows, H], bf16 as x or float32
+    values; gate: the rows' gates (double, [rows]) or None for 1;
     W13q u8 [2I, H] (gate rows 0..I-1, up rows I..2I-1), s13 f32 [2I/128, H/128];
     W2q u8 [H, I], s2 f32 [H/128, I/128].
     Returns FP32-rounded values (as float64 arrays): dx [rows, H],
-    dW13 [2I, H], dW2 [H, I], and the intermediates dh, dG, dU [rows, I] and
-    the forward's G, U, h [rows, I]."""
+    dW13 [2I, H], dW2 [H, I], the intermediates dh, dG, dU [rows, I], the
+    forward's G, U, h [rows, I] and the wgrad operand gh = g h."""
     W13q = np.asarray(W13q, np.uint8)
     W2q = np.asarray(W2q, np.uint8)
     s13 = np.asarray(s13, np.float32)
     s2 = np.asarray(s2, np.float32)
     I2, H = W13q.shape
     I = I2 // 2
+    dy = _as_f32_values(dy)
+    g = np.ones(dy.shape[0]) if gate is None else np.asarray(gate, np.float64).reshape(-1)
+    assert g.shape[0] == dy.shape[0]
     # forward recomputation (as the forward oracle: 1x128 x, FP32 G and U)
     xq, xs = quant_1x128(x, mode)
     G = _f32(blockscaled_gemm(xq, xs, W13q[:I], s13[:I // 128]))
@@ -122,13 +133,14 @@ def expert_backward(x, dy, W13q, s13, W2q, s2, mode: int = SCALE_AMAX) -> dict:
     sig = 1.0 / (1.0 + np.exp(-G))
     silu = G * sig
     h = _f32(silu * U)
-    # dgrad of the down projection: dY 1x128 along H, W2^T as [I, H] blocks
-    dy = _as_f32_values(dy)
+    # dgrad of the down projection: D 1x128 along H, W2^T as [I, H] blocks,
+    # the gate on the FP32 result
     dyq, dys = quant_1x128_f32(dy, mode)
-    dh = _f32(blockscaled_gemm(dyq, dys, np.ascontiguousarray(W2q.T), np.ascontiguousarray(s2.T)))
-    # wgrad of the down projection: dY and h as 128x1 tiles along tokens
+    dh = _f32(g[:, None] * blockscaled_gemm(dyq, dys, np.ascontiguousarray(W2q.T), np.ascontiguousarray(s2.T)))
+    # wgrad of the down projection: D and g h as 128x1 tiles along tokens
+    gh = _f32(g[:, None] * h)
     dyq_c, dys_c = quant_128x1_f32(dy, mode)
-    hq_c, hs_c = quant_128x1_f32(h, mode)
+    hq_c, hs_c = quant_128x1_f32(gh, mode)
     dW2 = _f32(rows_scaled_gemm(dyq_c.T, dys_c.T, hq_c.T, hs_c.T))
     # SwiGLU backward (double, rounded to FP32)
     dG = _f32(dh * U * sig * (1.0 + G * (1.0 - sig)))
@@ -147,44 +159,51 @@ def expert_backward(x, dy, W13q, s13, W2q, s2, mode: int = SCALE_AMAX) -> dict:
     dW1 = rows_scaled_gemm(dGq_c.T, dGs_c.T, xq_c.T, xs_c.T)
     dW3 = rows_scaled_gemm(dUq_c.T, dUs_c.T, xq_c.T, xs_c.T)
     dW13 = _f32(np.concatenate([dW1, dW3], axis=0))
-    return dict(dx=dx, dW13=dW13, dW2=dW2, dh=dh, dG=dG, dU=dU, G=G, U=U, h=h)
+    return dict(dx=dx, dW13=dW13, dW2=dW2, dh=dh, dG=dG, dU=dU, G=G, U=U, h=h, gh=gh)
 
 
-def layer_backward(cf, x, Wr, bias, experts, dout, mode: int = SCALE_AMAX) -> dict:
+def layer_backward(cf, x, Wr, bias, experts, dout, mode: int = SCALE_AMAX, details: bool = False) -> dict:
     """Backward of the layer's FFN part with the routing held fixed:
         out_t = u_t + FFN_shared(u_t) + sum_k g_{t,k} FFN_{e_{t,k}}(u_t)
     ("DeepSeek-V3 Technischer Bericht", Methode section 2, layer output
     equation).  Given dout [T, H] (bf16), each routed expert e receives, for
-    every token t that selected it (slot k), dY = g_{t,k} * dout_t in FP32
-    (the gate rounded to FP32, one FP32 product), the shared expert dY = dout;
-    each runs expert_backward on its tokens in token order.
+    every token t that selected it (slot k), dY = g_{t,k} * dout_t, handed to
+    expert_backward as dout_t and the gate (the placement of g is described
+    at the top of this module), the shared expert dY = dout; each runs
+    expert_backward on its tokens in token order.
         dx_t = dout_t + dx_shared,t + sum_k dx_{e_{t,k}},t    (double, then FP32)
     The routing (and with it every gate) is the oracle's own; the gradient of
     the gates themselves (router backward) is not part of this.
     experts: list indexed by expert id (routed 0..N_r-1, shared N_r) of
     (W13q, s13, W2q, s2) tuples, None for experts no token uses.
     Returns dx [T, H], dW13 and dW2 dicts keyed by expert id (FP32 values as
-    double arrays), and the routing (idx, gate, gap)."""
+    double arrays), and the routing (idx, gate, gap); with details, also
+    per_expert: expert id -> (its tokens in order, expert_backward's dict)."""
     idx, gate, gap, _ = route(cf, x, Wr, bias)
     xu = _u16(x)
     d = _as_f32_values(dout)
     T = xu.shape[0]
     Nr = cf.Nr
     acc = d.astype(np.float64)
-    dW13, dW2 = {}, {}
+    dW13, dW2, per_expert = {}, {}, {}
     for e in range(Nr):
         toks, slots = np.nonzero(idx == e)
         if toks.size == 0:
             continue
         order = np.argsort(toks, kind="stable")
         toks, slots = toks[order], slots[order]
-        g32 = gate[toks, slots].astype(np.float32)
-        dy = (g32[:, None] * d[toks]).astype(np.float32)
-        r = expert_backward(xu[toks], dy, *experts[e], mode=mode)
+        r = expert_backward(xu[toks], d[toks], *experts[e], gate=gate[toks, slots], mode=mode)
         acc[toks] += r["dx"]
         dW13[e], dW2[e] = r["dW13"], r["dW2"]
+        if details:
+            per_expert[e] = (toks, r)
     if cf.Ns:
         r = expert_backward(xu, d, *experts[Nr], mode=mode)
         acc += r["dx"]
         dW13[Nr], dW2[Nr] = r["dW13"], r["dW2"]
-    return dict(dx=_f32(acc), dW13=dW13, dW2=dW2, idx=idx, gate=gate, gap=gap)
+        if details:
+            per_expert[Nr] = (np.arange(T), r)
+    out = dict(dx=_f32(acc), dW13=dW13, dW2=dW2, idx=idx, gate=gate, gap=gap)
+    if details:
+        out["per_expert"] = per_expert
+    return out

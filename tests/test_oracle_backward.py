@@ -247,3 +247,31 @@ def test_layer_backward_tracks_the_dense_layer_gradient(oracle_lib, bw):
     rel = _rel(r["dx"] - dd, dx - dd)
     print(f"layer dx rel-Frobenius {rel:.3f}; weight gradients max {max(rel_w):.3f}")
     assert rel < 0.12 and max(rel_w) < 0.15
+
+
+def test_gate_placement(oracle_lib, bw):
+    # dY = g D.  A power-of-two gate is exact in every step, so handing the
+    # gate to expert_backward must give bitwise the gradients of the scaled
+    # D (a dropped gate, or one applied twice, differs by 2x).  A general
+    # gate moves only the rounding of g D out of the dgrad's codes.
+    x, dy, W13q, s13, W2q, s2 = _problem(oracle_lib, 200, seed=8)
+    rows = dy.shape[0]
+    g = 2.0 ** np.random.default_rng(8).integers(-3, 1, size=rows)
+    a = bw.expert_backward(x, dy, W13q, s13, W2q, s2, gate=g)
+    b = bw.expert_backward(x, (dy.float() * torch.from_numpy(g).float()[:, None]).numpy(), W13q, s13, W2q, s2)
+    for k in ("dx", "dW13", "dh", "dG", "dU"):
+        assert np.array_equal(a[k], b[k]), k
+    assert np.array_equal(a["gh"], g[:, None] * a["h"])
+    # in dW2 the gate moves between the operands of 128x1 tiles with mixed
+    # gates, which changes their codes; with one gate for every row it does not
+    assert _rel(a["dW2"], b["dW2"]) < 0.1
+    a = bw.expert_backward(x, dy, W13q, s13, W2q, s2, gate=np.full(rows, 0.25))
+    b = bw.expert_backward(x, (dy.float() * 0.25).numpy(), W13q, s13, W2q, s2)
+    assert np.array_equal(a["dW2"], b["dW2"])
+    g = np.random.default_rng(9).uniform(0.05, 0.6, size=rows)
+    a = bw.expert_backward(x, dy, W13q, s13, W2q, s2, gate=g)
+    b = bw.expert_backward(x, (dy.float() * torch.from_numpy(g).float()[:, None]).numpy(), W13q, s13, W2q, s2)
+    for k in ("dx", "dW13", "dh"):
+        assert _rel(a[k], b[k]) < 2e-2, k
+    assert _rel(a["dW2"], b["dW2"]) < 0.1
+    assert np.array_equal(a["G"], b["G"])
