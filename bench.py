@@ -154,6 +154,30 @@ def algorithmic_counts(cfg: dict, T: int, touched_routed: int) -> dict:
                 layer_weight_bytes=E_t * (w13 + w2))
 
 
+def gemm_work(M, torch, layer, T: int, stage_ms: dict, sm_mhz, pair: bool) -> dict:
+    """Work of the two grouped GEMM launches of the last forward, from the
+    chunk table it left in the workspace: chunks, tiles, K blocks per
+    processing unit (an SM, or a pair of SMs on the CTA-pair kernel), and the
+    cycles one K block took on average at the sampled SM clock."""
+    import math as _m
+    c = layer.cfg
+    ws, L = layer.workspace(T), layer.layout(T)
+    nch = int(M.ws_view(ws, L, "meta", torch.int32, (4,)).cpu()[0])
+    sms = torch.cuda.get_device_properties(ws.device).multi_processor_count
+    units = sms // 2 if pair else sms
+    out = {}
+    for name, nb, kb in (("gemm_gate_up", c.inter // 128, c.hidden // 128),
+                         ("gemm_down", (c.hidden // 128 + 1) // 2, c.inter // 128)):
+        tiles = nch * nb
+        kpu = tiles * kb / units
+        d = dict(chunks=nch, tiles=tiles, k_blocks=tiles * kb, k_blocks_per_unit=round(kpu, 1),
+                 unit="SM pair" if pair else "SM")
+        if sm_mhz:
+            d["cycles_per_k_block"] = round(stage_ms[name] * 1e-3 * sm_mhz * 1e6 / _m.ceil(kpu), 1)
+        out[name] = d
+    return out
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -640,6 +664,9 @@ def main(argv=None):
 
     counts_h = counts.cpu()
     touched = int((counts_h > 0).sum())
+    gemm_kernel = M.moe_gemm_kernel_for(layer.cfg, T)
+    pair_kernel = gemm_kernel == M.MOE_GEMM_PAIR
+    work = gemm_work(M, torch, layer, T, stage_ms, clocks.get("sm_mhz"), pair_kernel)
     # sequence-wise balance loss (alpha = 1e-4) of the batch the timed steps
     # routed, read from the last forward's workspace before anything reroutes
     seq_len = math.gcd(T, 4096)
@@ -671,8 +698,8 @@ def main(argv=None):
     fp8_src = peaks["src"] + (" bf16 sustained x 2" if sustained else " bf16 burst x 2")
     t_mem = dom_bytes / (peaks["hbm"] * 1e9)
     t_tc = dom_flops / (fp8_peak * 1e12)
-    pair = args.scale_mode != "pow2" and args.gemm == "pair" and (cfg["H"] // 128) % 2 == 0
-    kname = "gemm_mx_kernel" if args.scale_mode == "pow2" else ("gemm_pair_kernel" if pair else "gemm_fp8_kernel")
+    kname = {M.MOE_GEMM_BLOCK_SCALED: "gemm_mx_kernel", M.MOE_GEMM_PAIR: "gemm_pair_kernel"}.get(gemm_kernel,
+                                                                                              "gemm_fp8_kernel")
     kernel_name = f"{kname}<0>" if dom == "gemm_gate_up" else f"{kname}<1>"
     if t_mem >= t_tc:
         achieved = dom_bytes / (dom_ms / 1e3) / 1e9
@@ -780,6 +807,7 @@ def main(argv=None):
         load=load,
         **({"balance": balance} if balance else {}),
         stage_ms={k: round(v, 4) for k, v in stage_ms.items()},
+        gemm_work=work,
         step_ms_min=round(min(step_ms), 4),
         cpu_baseline=cpu,
         e2e=e2e,

@@ -304,16 +304,19 @@ MOE_API int moe_profile_events(void *const *events, int32_t n_events);
  * along that GEMM's contraction).  For out_t = u_t + FFN_s(u_t) +
  * sum_k g_{t,k} FFN_{e_{t,k}}(u_t) and a gradient dout of out:
  *   every expert row p (token t, gate g; g = 1 for the shared expert)
- *   receives dY_p = g * dout_t (FP32);
+ *   receives dY_p = g * dout_t, and the gate is kept out of every
+ *   quantized tile of dY: a 1x128 tile of g * dout has the codes of dout's
+ *   tile (g cancels in the quotient), so
  *   G, U recomputed (the forward's gate/up GEMM, FP32 results);
- *   dh = dY W2      (dY 1x128 along H, W2's blocks transposed)
+ *   dh = g (dout_t W2)  (dout 1x128 along H, W2's blocks transposed; g
+ *                        times the FP32 result)
  *   dG = dh U silu'(G), dU = dh silu(G), h = silu(G) U       (FP32)
  *   dx_p = dG W1 + dU W3  (dG, dU 1x128 along I, W1/W3's blocks transposed)
  *   dx_t = dout_t + sum over the token's rows of dx_p         (FP32)
- *   dW2_e = dY_e^T h_e, dW13_e = [dG | dU]_e^T x_e over expert e's tokens
- *   (both operands 128x1 along tokens: one scale per channel per 128
- *   tokens, a ragged last tile shorter; every GEMM promotes each 128-long
- *   partial into FP32).
+ *   dW2_e = dout_e^T (g h)_e (= dY_e^T h_e), dW13_e = [dG | dU]_e^T x_e
+ *   over expert e's tokens (both operands 128x1 along tokens: one scale per
+ *   channel per 128 tokens, a ragged last tile shorter; every GEMM promotes
+ *   each 128-long partial into FP32).
  * The gates' own gradient (router backward) is not part of this.
  *
  * moe_transpose_weights (set-up): the dgrad GEMMs' weights, each expert's
@@ -334,11 +337,12 @@ MOE_API int moe_transpose_weights(const moe_config *cfg, const moe_weights *w, u
 MOE_API size_t moe_backward_workspace_size(const moe_config *cfg, int64_t T);
 /* Byte offsets {offset, bytes} of the backward's intermediates inside its
  * workspace (for tests and inspection), rows in the forward's row order
- * (RS = T*K_r + T*N_s): gu float [RS, 2I] (G then U), dh and h float [RS, I],
+ * (RS = T*K_r + T*N_s): gu float [RS, 2I] (G then U), dh float [RS, I] (with
+ * the gate), gh float [RS, I] (the row's gate times h),
  * dgu float [RS, 2I] (dG then dU), dx_rows float [RS, H], seg int32 [E + 1]
  * (each expert's token segment of the weight-gradient operands, P columns). */
 typedef struct {
-    size_t gu[2], dh[2], h[2], dgu[2], dx_rows[2], seg[2];
+    size_t gu[2], dh[2], gh[2], dgu[2], dx_rows[2], seg[2];
     int64_t P;
     size_t total;
 } moe_bwd_layout;
@@ -430,7 +434,10 @@ MOE_API int moe_ep_combine(const moe_config *cfg, int32_t world, const void *x_d
 
 /* Kernel choice of the grouped expert GEMMs in the default scale mode
  * (process-wide; a tuning and testing switch, the arithmetic is the same):
- *   MOE_GEMM_AUTO   (default) the measured-fastest choice: single CTAs
+ *   MOE_GEMM_AUTO   (default) the measured-faster choice: CTA pairs when
+ *                   the routed experts average >= 256 rows (T * top_k >=
+ *                   256 * n_routed) and hidden is a multiple of 256, else
+ *                   single CTAs
  *   MOE_GEMM_SINGLE one CTA per tile: <= 128 rows of one expert per pass over
  *                   a weight-block pair
  *   MOE_GEMM_PAIR   a pair of CTAs on two SMs per tile (<= 256 rows per
@@ -439,8 +446,14 @@ MOE_API int moe_ep_combine(const moe_config *cfg, int32_t world, const void *x_d
  *                   (hidden a multiple of 256), else single CTAs
  * Returns MOE_ERR_INVALID_ARG for any other value.  Takes effect for the
  * next moe_forward on any thread; not synchronised with calls in flight. */
-enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SINGLE = 1, MOE_GEMM_PAIR = 2 };
+enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SINGLE = 1, MOE_GEMM_PAIR = 2, MOE_GEMM_BLOCK_SCALED = 3 };
 MOE_API int moe_set_gemm_variant(int32_t variant);
+/* The grouped-GEMM kernel the next moe_forward of T tokens under cfg runs
+ * with the current variant setting: MOE_GEMM_SINGLE, MOE_GEMM_PAIR, or
+ * MOE_GEMM_BLOCK_SCALED (scale_mode MOE_SCALE_POW2: the tensor core applies
+ * the power-of-two scales), or a (negative) error status for an invalid
+ * cfg or T.  Host-only; no device work. */
+MOE_API int moe_gemm_kernel_for(const moe_config *cfg, int64_t T);
 
 /* --------------------------------------------------------- bias update */
 /* Auxiliary-loss-free balancing step ([P4] Methode 2; [P1]): with

@@ -42,7 +42,7 @@ EXPORTS = (
     "fp8_quant_128x128_pow2", "fp8_blockscaled_gemm",
     "moe_route_workspace_size", "moe_route", "moe_workspace_size", "moe_forward", "moe_workspace_layout",
     "moe_bias_update", "moe_check_device_error", "moe_selftest_wait_timeout", "moe_profile_events",
-    "moe_route_noalloc", "moe_seq_balance_loss", "moe_set_gemm_variant",
+    "moe_route_noalloc", "moe_seq_balance_loss", "moe_set_gemm_variant", "moe_gemm_kernel_for",
     "moe_ep_row_bytes", "moe_ep_dispatch_workspace_size", "moe_ep_dispatch", "moe_ep_experts_workspace_size",
     "moe_ep_experts", "moe_ep_combine", "moe_transpose_weights", "moe_backward_workspace_size", "moe_backward",
     "moe_backward_workspace_layout",
@@ -50,6 +50,7 @@ EXPORTS = (
 MOE_GEMM_AUTO = 0
 MOE_GEMM_SINGLE = 1
 MOE_GEMM_PAIR = 2
+MOE_GEMM_BLOCK_SCALED = 3
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 16 << 20
 MOE_PROFILE_EVENTS = 7
 PROFILE_STAGES = ("quantize", "route", "group", "gemm_gate_up", "gemm_down", "combine")
@@ -98,6 +99,7 @@ lib.moe_check_device_error.argtypes = [_vp, C.POINTER(C.c_int32), _vp]
 lib.moe_selftest_wait_timeout.argtypes = [_vp, _i64, _vp]
 lib.moe_profile_events.argtypes = [C.POINTER(_vp), _i32]
 lib.moe_set_gemm_variant.argtypes = [_i32]
+lib.moe_gemm_kernel_for.argtypes = [_cfgp, _i64]
 lib.moe_ep_row_bytes.restype = _i64
 lib.moe_ep_row_bytes.argtypes = [_cfgp]
 lib.moe_ep_dispatch_workspace_size.restype = _sz
@@ -110,7 +112,7 @@ lib.moe_ep_experts.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _i64, _i64, _v
 lib.moe_ep_combine.argtypes = [_cfgp, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _i32, _vp]
 lib.moe_transpose_weights.argtypes = [_cfgp, C.POINTER(MoeWeights), _vp, _vp, _vp, _vp, _vp]
 class MoeBwdLayout(C.Structure):
-    _fields_ = [(f, C.c_size_t * 2) for f in ("gu", "dh", "h", "dgu", "dx_rows", "seg")] + [("P", C.c_int64),
+    _fields_ = [(f, C.c_size_t * 2) for f in ("gu", "dh", "gh", "dgu", "dx_rows", "seg")] + [("P", C.c_int64),
                                                                                           ("total", C.c_size_t)]
 
 
@@ -295,6 +297,15 @@ def moe_set_gemm_variant(variant: int) -> None:
     _check(lib.moe_set_gemm_variant(variant), "moe_set_gemm_variant")
 
 
+def moe_gemm_kernel_for(cfg, T: int) -> int:
+    """The grouped-GEMM kernel (MOE_GEMM_SINGLE, _PAIR or _BLOCK_SCALED) the
+    next moe_forward of T tokens runs under the current variant setting."""
+    r = lib.moe_gemm_kernel_for(C.byref(cfg), int(T))
+    if r < 0:
+        _check(r, "moe_gemm_kernel_for")
+    return r
+
+
 # ---------------------------------------------------- expert parallelism
 def moe_ep_row_bytes(cfg: MoeConfig) -> int:
     return int(lib.moe_ep_row_bytes(C.byref(cfg)))
@@ -357,7 +368,7 @@ def ctypes_cfg(cfg: MoeConfig):
 def moe_backward_workspace_layout(cfg: MoeConfig, T: int) -> dict:
     L = MoeBwdLayout()
     _check(lib.moe_backward_workspace_layout(C.byref(cfg), T, C.byref(L)), "moe_backward_workspace_layout")
-    d = {f: (int(getattr(L, f)[0]), int(getattr(L, f)[1])) for f in ("gu", "dh", "h", "dgu", "dx_rows", "seg")}
+    d = {f: (int(getattr(L, f)[0]), int(getattr(L, f)[1])) for f in ("gu", "dh", "gh", "dgu", "dx_rows", "seg")}
     d["P"], d["total"] = int(L.P), int(L.total)
     return d
 

@@ -122,14 +122,22 @@ int check_cfg_local(const moe_config *c) {
 
 constexpr int64_t kMaxTokens = 1 << 20;
 
-// The grouped GEMMs of the default scale mode run on single CTAs; with
-// moe_set_gemm_variant(MOE_GEMM_PAIR) on CTA pairs (256 rows per weight pass)
+// The grouped GEMMs of the default scale mode run on single CTAs (<= 128 rows
+// of an expert per weight pass) or on CTA pairs (<= 256 rows), the latter only
 // when the down projection's weight blocks pair up (H a multiple of 256).
+// MOE_GEMM_AUTO takes pairs when the routed experts average at least 256 rows
+// (T * K_r >= 256 * N_r): then most experts fill pair tiles and each weight
+// block is read half as often; below that, half-empty pair tiles cost more
+// than the saved weight reads (measured at V3 sizes: 128 rows per expert is
+// faster on single CTAs, 512 on pairs).
 std::atomic<int> g_gemm_variant{MOE_GEMM_AUTO};
 
-bool use_pair_gemm(int64_t H) {
-  if ((H / 128) % 2 != 0) return false;
-  return g_gemm_variant.load(std::memory_order_relaxed) == MOE_GEMM_PAIR;
+bool use_pair_gemm(const moe_config *c, int64_t T) {
+  if ((c->hidden / 128) % 2 != 0) return false;
+  const int v = g_gemm_variant.load(std::memory_order_relaxed);
+  if (v == MOE_GEMM_PAIR) return true;
+  if (v == MOE_GEMM_SINGLE) return false;
+  return T * static_cast<int64_t>(c->top_k) >= 256 * static_cast<int64_t>(c->n_routed);
 }
 
 struct Carve {
@@ -203,12 +211,19 @@ const char *moe_status_string(int s) {
   }
 }
 
-int moe_abi_version(void) { return 103; }
+int moe_abi_version(void) { return 104; }
 
 int moe_set_gemm_variant(int32_t variant) {
   if (variant != MOE_GEMM_AUTO && variant != MOE_GEMM_SINGLE && variant != MOE_GEMM_PAIR) return MOE_ERR_INVALID_ARG;
   g_gemm_variant.store(variant, std::memory_order_relaxed);
   return MOE_OK;
+}
+
+int moe_gemm_kernel_for(const moe_config *cfg, int64_t T) {
+  if (const int c = check_cfg(cfg)) return c;
+  if (T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
+  if (cfg->scale_mode == MOE_SCALE_POW2) return MOE_GEMM_BLOCK_SCALED;
+  return use_pair_gemm(cfg, T) ? MOE_GEMM_PAIR : MOE_GEMM_SINGLE;
 }
 
 static int quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q, float *scales,
@@ -422,7 +437,7 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
   int4 *chunks = at<int4 *>(ws, L.chunks);
   const int64_t max_chunks = moe::max_chunks(T, Kr, Nr, Ns);
   const bool pow2 = cfg->scale_mode == MOE_SCALE_POW2;
-  const bool pair = !pow2 && use_pair_gemm(H);
+  const bool pair = !pow2 && use_pair_gemm(cfg, T);
   const int chunk_rows = pair ? 256 : 128;
 
   cudaError_t e = moe::launch_hist(P.idx, T, Kr, Nr, P.allow_empty, blk_hist, err_flag, st);
@@ -702,7 +717,7 @@ int moe_ep_combine(const moe_config *cfg, int32_t world, const void *x, int64_t 
 // ------------------------------------------------------------ backward
 namespace {
 struct BwdLayout {
-  size_t gu[2], dyq[2], dys[2], dh[2], h[2], dgu[2], dguq[2], dgus[2], dxr[2];
+  size_t gu[2], dyq[2], dys[2], dh[2], gh[2], dgu[2], dguq[2], dgus[2], dxr[2];
   size_t counts[2], offsets[2], blk_base[2], chunks[2], meta[2];
   size_t seg[2], tiles[2], tmeta[2];
   size_t dyt[2], sdy[2], ht[2], sh[2], dgut[2], sdgu[2], xt[2], sx[2];
@@ -722,7 +737,7 @@ void make_bwd_layout(const moe_config *c, int64_t T, BwdLayout *B) {
   cv.take(B->dyq, RS * H);
   cv.take(B->dys, ((H / 128) * pitch + moe::kScaleSlack) * 4);
   cv.take(B->dh, RS * I * 4);
-  cv.take(B->h, RS * I * 4);
+  cv.take(B->gh, RS * I * 4);
   cv.take(B->dgu, RS * 2 * I * 4);
   cv.take(B->dguq, RS * 2 * I);
   cv.take(B->dgus, ((2 * I / 128) * pitch + moe::kScaleSlack) * 4);
@@ -772,7 +787,7 @@ int moe_backward_workspace_layout(const moe_config *cfg, int64_t T, moe_bwd_layo
   };
   cp(out->gu, B.gu);
   cp(out->dh, B.dh);
-  cp(out->h, B.h);
+  cp(out->gh, B.gh);
   cp(out->dgu, B.dgu);
   cp(out->dx_rows, B.dxr);
   cp(out->seg, B.seg);
@@ -827,7 +842,7 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
   uint8_t *dyq = at<uint8_t *>(ws, B.dyq);
   float *dys = at<float *>(ws, B.dys);
   float *dh = at<float *>(ws, B.dh);
-  float *hbuf = at<float *>(ws, B.h);
+  float *ghbuf = at<float *>(ws, B.gh);
   float *dGU = at<float *>(ws, B.dgu);
   uint8_t *dGUq = at<uint8_t *>(ws, B.dguq);
   float *dGUs = at<float *>(ws, B.dgus);
@@ -880,9 +895,10 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
     g.out_cols = 2 * I;
     e = moe::launch_gemm(g, st);
   }
-  if (e == cudaSuccess) e = moe::launch_dy_quant(dout, row_src, row_gate, R, RS, H, dyq, dys, pitch, st);
+  if (e == cudaSuccess) e = moe::launch_dout_quant(dout, row_src, R, RS, H, dyq, dys, pitch, st);
   if (e == cudaSuccess) {
-    // dh = dY W2: K = H against W2^T [E, I, H]
+    // dh = g (dout W2): K = H against W2^T [E, I, H], the row's gate in the
+    // FP32 epilogue
     moe::GemmLaunch g{};
     base_gemm(g);
     g.w = w2t;
@@ -899,14 +915,15 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
     g.gate_up = 0;
     g.a_is_out_row = 1;
     g.rows_per_expert = I;
-    g.epi = moe::EPI_F32;
+    g.epi = moe::EPI_GATE_F32;
+    g.row_gate = row_gate;
     g.out = dh;
     g.ldo = I;
     g.out_rows = RS;
     g.out_cols = I;
     e = moe::launch_gemm(g, st);
   }
-  if (e == cudaSuccess) e = moe::launch_swiglu_bwd(GU, dh, RS, I, hbuf, dGU, dGUq, dGUs, pitch, st);
+  if (e == cudaSuccess) e = moe::launch_swiglu_bwd(GU, dh, row_gate, RS, I, ghbuf, dGU, dGUq, dGUs, pitch, st);
   if (e == cudaSuccess) {
     // dx rows = [dG|dU] [W1; W3] (FP32): K = 2I against W13^T [E, H, 2I]
     moe::GemmLaunch g{};
@@ -938,17 +955,17 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
   if (e == cudaSuccess) e = moe::launch_wgrad_tiles(offsets, Nr, Ns, R, T, seg, tiles, tmeta, st);
   const int mt = static_cast<int>(B.max_tiles);
   if (e == cudaSuccess)
-    e = moe::launch_colquant(1, tiles, tmeta, mt, nullptr, 0, dout, row_src, row_gate, R, H, at<uint8_t *>(ws, B.dyt),
-                             B.P, at<float *>(ws, B.sdy), st);
+    e = moe::launch_colquant(1, tiles, tmeta, mt, nullptr, 0, dout, row_src, R, H, at<uint8_t *>(ws, B.dyt), B.P,
+                             at<float *>(ws, B.sdy), st);
   if (e == cudaSuccess)
-    e = moe::launch_colquant(0, tiles, tmeta, mt, hbuf, I, nullptr, row_src, row_gate, R, I, at<uint8_t *>(ws, B.ht),
-                             B.P, at<float *>(ws, B.sh), st);
+    e = moe::launch_colquant(0, tiles, tmeta, mt, ghbuf, I, nullptr, row_src, R, I, at<uint8_t *>(ws, B.ht), B.P,
+                             at<float *>(ws, B.sh), st);
   if (e == cudaSuccess)
-    e = moe::launch_colquant(0, tiles, tmeta, mt, dGU, 2 * I, nullptr, row_src, row_gate, R, 2 * I,
+    e = moe::launch_colquant(0, tiles, tmeta, mt, dGU, 2 * I, nullptr, row_src, R, 2 * I,
                              at<uint8_t *>(ws, B.dgut), B.P, at<float *>(ws, B.sdgu), st);
   if (e == cudaSuccess)
-    e = moe::launch_colquant(2, tiles, tmeta, mt, nullptr, 0, x, row_src, row_gate, R, H, at<uint8_t *>(ws, B.xt),
-                             B.P, at<float *>(ws, B.sx), st);
+    e = moe::launch_colquant(1, tiles, tmeta, mt, nullptr, 0, x, row_src, R, H, at<uint8_t *>(ws, B.xt), B.P,
+                             at<float *>(ws, B.sx), st);
   if (e == cudaSuccess) {
     moe::WgradLaunch g{};
     g.a_t = at<uint8_t *>(ws, B.dyt);

@@ -11,23 +11,28 @@
 // as 128x1 tiles along tokens (a ragged last tile holds fewer).
 //
 // With the forward's row order (routed rows per expert in token order, then
-// the shared expert's rows) and for one layer-output gradient dout [T, H]:
-//   dY[p]  = g_p * dout[token(p)]                    (FP32; g = 1 for shared)
+// the shared expert's rows), one layer-output gradient dout [T, H] and the
+// row gates g_p (1 for the shared expert), row p's output gradient is
+// dY[p] = g_p dout[token(p)].  The gate is kept out of every quantized tile
+// of dY: a 1x128 tile of g D has the codes of D's tile (g cancels in the
+// quotient), so the dgrad quantizes dout and scales its FP32 result by g;
+// the wgrad carries g on h (dY^T h = dout^T (g h)).
 //   G, U   = the forward's gate/up GEMM, FP32          (grouped GEMM, EPI_F32)
-//   dh     = dY W2        (dY 1x128 along H)          (grouped GEMM, EPI_F32)
+//   dh     = g (dout W2)  (dout 1x128 along H)   (grouped GEMM, EPI_GATE_F32)
 //   h      = silu(G) U,   dG = dh U silu'(G),   dU = dh silu(G)   (FP32)
-//   dx_p   = dG W1 + dU W3  (dG|dU 1x128 along I)     (grouped GEMM, bf16)
+//   dx_p   = dG W1 + dU W3  (dG|dU 1x128 along I)     (grouped GEMM, FP32)
 //   dx_t   = dout_t + sum over the token's rows of dx_p   (the combine)
-//   dW2_e  = dY_e^T h_e,  dW13_e = [dG|dU]_e^T x_e    (128x1 along tokens;
-//                                                      gemm_wgrad.cu)
+//   dW2_e  = dout_e^T (g h)_e,  dW13_e = [dG|dU]_e^T x_e  (128x1 along
+//                                                   tokens; gemm_wgrad.cu)
 //
 // Kernels here:
 //   transpose_blocks_kernel  E4M3 [n, k] with [n/128, k/128] block scales ->
 //                            the transpose [k, n] and [k/128, n/128] (set-up
 //                            of the dgrad weights)
-//   dy_quant_kernel          dY rows, 1x128 along H -> codes + transposed
-//                            scale table (the dgrad GEMM's A operand)
-//   swiglu_bwd_kernel        h, dG, dU from G, U, dh; dG|dU 1x128 along I
+//   dout_quant_kernel        dout rows in the forward's row order, 1x128
+//                            along H -> codes + transposed scale table (the
+//                            dgrad GEMM's A operand)
+//   swiglu_bwd_kernel        g h, dG, dU from G, U, dh; dG|dU 1x128 along I
 //   wgrad_tiles_kernel       per expert: its padded token segment and its
 //                            128-token tiles
 //   colquant_kernel          128x1 tiles along an expert's tokens, stored
@@ -84,15 +89,14 @@ __device__ __forceinline__ uint2 codes8_div(const float (&f)[8], float S) {
   return make_uint2(lo, hi);
 }
 
-// -------------------------------------------------------------- dY rows
+// ------------------------------------------------------------ dout rows
 // Row p of the forward's row order: token t = row_src[p] (routed, p < R) or
-// p - R (shared); dY = gate_p * dout[t] (one FP32 product), quantized 1x128
-// along H: codes [RS, H], scales into the transposed table [H/128][ld].
-__global__ void __launch_bounds__(256) dy_quant_kernel(const uint16_t *__restrict__ dout,
-                                                        const int32_t *__restrict__ row_src,
-                                                        const float *__restrict__ row_gate, int64_t R, int64_t RS,
-                                                        int H, uint8_t *__restrict__ q, float *__restrict__ s_t,
-                                                        int64_t ld) {
+// p - R (shared); dout[t] quantized 1x128 along H: codes [RS, H], scales
+// into the transposed table [H/128][ld].
+__global__ void __launch_bounds__(256) dout_quant_kernel(const uint16_t *__restrict__ dout,
+                                                          const int32_t *__restrict__ row_src, int64_t R,
+                                                          int64_t RS, int H, uint8_t *__restrict__ q,
+                                                          float *__restrict__ s_t, int64_t ld) {
   const int64_t groups = H / 128;
   const int64_t gid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
   const int sub = threadIdx.x & 15;
@@ -102,13 +106,12 @@ __global__ void __launch_bounds__(256) dy_quant_kernel(const uint16_t *__restric
   float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (valid) {
     const int64_t t = p < R ? row_src[p] : p - R;
-    const float gt = row_gate[p];
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(dout + t * H + g * 128 + sub * 8));
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      f[2 * i] = gt * __uint_as_float(w[i] << 16);
-      f[2 * i + 1] = gt * __uint_as_float(w[i] & 0xFFFF0000u);
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
   }
   const float S = group_scale16(f);
@@ -119,14 +122,16 @@ __global__ void __launch_bounds__(256) dy_quant_kernel(const uint16_t *__restric
 }
 
 // --------------------------------------------------------- SwiGLU backward
-// Per row p and 128-channel group j of I (one warp: 4 channels per lane):
+// Per row p and 128-channel group j of I (one warp: 4 channels per lane),
+// with dh already carrying the row's gate g:
 //   sig = 1/(1+exp(-G)), silu = G sig, h = silu U,
 //   dG = dh U sig (1 + G (1 - sig)), dU = dh silu          (FP32)
-// Writes h [RS, I] and dGU [RS, 2I] (dG at column c, dU at I + c) in FP32,
-// and dG | dU quantized 1x128 along I: codes [RS, 2I], scales into the
-// transposed table [2I/128][ld].
+// Writes gh = g h [RS, I] (the dW2 operand) and dGU [RS, 2I] (dG at column
+// c, dU at I + c) in FP32, and dG | dU quantized 1x128 along I: codes
+// [RS, 2I], scales into the transposed table [2I/128][ld].
 __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const float *__restrict__ GU, const float *__restrict__ dh,
-                                                          int64_t RS, int I, float *__restrict__ h,
+                                                          const float *__restrict__ row_gate, int64_t RS, int I,
+                                                          float *__restrict__ h,
                                                           float *__restrict__ dGU, uint8_t *__restrict__ q,
                                                           float *__restrict__ s_t, int64_t ld) {
   const int lane = threadIdx.x & 31;
@@ -139,13 +144,14 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const float *__restrict
   const float4 U4 = *reinterpret_cast<const float4 *>(GU + p * 2 * I + I + c);
   const float4 D4 = *reinterpret_cast<const float4 *>(dh + p * I + c);
   const float G[4] = {G4.x, G4.y, G4.z, G4.w}, U[4] = {U4.x, U4.y, U4.z, U4.w}, D[4] = {D4.x, D4.y, D4.z, D4.w};
+  const float gt = __ldg(row_gate + p);
   float hv[4], dg[4], du[4];
   float ag = 0.0f, au = 0.0f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float sig = 1.0f / (1.0f + expf(-G[i]));
     const float silu = G[i] * sig;
-    hv[i] = silu * U[i];
+    hv[i] = gt * (silu * U[i]);
     dg[i] = D[i] * U[i] * sig * (1.0f + G[i] * (1.0f - sig));
     du[i] = D[i] * silu;
     ag = fmaxf(ag, fabsf(dg[i]));
@@ -225,20 +231,19 @@ __global__ void __launch_bounds__(512) wgrad_tiles_kernel(const int32_t *__restr
 
 // ------------------------------------------------ 128x1 tiles, transposed
 // Grid: (tile, 64-channel block).  The tile's rows (tokens) of 64 channels
-// are read in FP32 (from an FP32 row matrix, or dY rebuilt from dout and the
-// row gate, or the layer input gathered by token), each channel's amax over
+// are read in FP32 (from an FP32 row matrix, or a bf16 [T, C] matrix gathered
+// by the row's token: dout, the layer input), each channel's amax over
 // the tile's rows gives its scale, and the codes are written channel-major:
 // out[c][col0 + r] (K-major along tokens for the wgrad GEMM); scales to
 // s_t[(col0 / 128)][c].  Padding rows (beyond the tile's rows) are zero.
-enum ColSrc : int { COL_F32 = 0, COL_DY = 1, COL_X = 2 };
+enum ColSrc : int { COL_F32 = 0, COL_TOKEN = 1 };
 constexpr int kColCh = 64;
 
 template <int SRC>
 __global__ void __launch_bounds__(256) colquant_kernel(const int4 *__restrict__ tiles, const int32_t *__restrict__ meta,
                                                         int max_tiles, const float *__restrict__ f32rows,
                                                         int64_t f32_ld, const uint16_t *__restrict__ bf16rows,
-                                                        const int32_t *__restrict__ row_src,
-                                                        const float *__restrict__ row_gate, int64_t R, int C,
+                                                        const int32_t *__restrict__ row_src, int64_t R, int C,
                                                         uint8_t *__restrict__ out, int64_t out_ld,
                                                         float *__restrict__ s_t) {
   __shared__ float vals[128][kColCh + 1];
@@ -266,11 +271,10 @@ __global__ void __launch_bounds__(256) colquant_kernel(const int4 *__restrict__ 
       } else {
         const int64_t t = p < R ? row_src[p] : p - R;
         const uint2 b = *reinterpret_cast<const uint2 *>(bf16rows + t * C + c0 + c4);
-        const float g = SRC == COL_DY ? row_gate[p] : 1.0f;
-        const float x[4] = {__uint_as_float(b.x << 16), __uint_as_float(b.x & 0xFFFF0000u),
-                            __uint_as_float(b.y << 16), __uint_as_float(b.y & 0xFFFF0000u)};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = SRC == COL_DY ? g * x[k] : x[k];
+        v[0] = __uint_as_float(b.x << 16);
+        v[1] = __uint_as_float(b.x & 0xFFFF0000u);
+        v[2] = __uint_as_float(b.y << 16);
+        v[3] = __uint_as_float(b.y & 0xFFFF0000u);
       }
     }
 #pragma unroll
@@ -310,22 +314,22 @@ cudaError_t launch_transpose_blocks(const uint8_t *q, const float *s, int64_t n,
   return cudaGetLastError();
 }
 
-cudaError_t launch_dy_quant(const void *dout, const int32_t *row_src, const float *row_gate, int64_t R, int64_t RS,
-                            int H, uint8_t *q, float *s_t, int64_t ld, cudaStream_t st) {
+cudaError_t launch_dout_quant(const void *dout, const int32_t *row_src, int64_t R, int64_t RS, int H, uint8_t *q,
+                              float *s_t, int64_t ld, cudaStream_t st) {
   const int64_t groups = RS * (H / 128);
   if (groups == 0) return cudaSuccess;
   const int64_t blocks = (groups * 16 + 255) / 256;
-  dy_quant_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(static_cast<const uint16_t *>(dout), row_src,
-                                                                  row_gate, R, RS, H, q, s_t, ld);
+  dout_quant_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(static_cast<const uint16_t *>(dout), row_src, R,
+                                                                    RS, H, q, s_t, ld);
   return cudaGetLastError();
 }
 
-cudaError_t launch_swiglu_bwd(const float *GU, const float *dh, int64_t RS, int I, float *h, float *dGU, uint8_t *q,
-                              float *s_t, int64_t ld, cudaStream_t st) {
+cudaError_t launch_swiglu_bwd(const float *GU, const float *dh, const float *row_gate, int64_t RS, int I, float *h,
+                              float *dGU, uint8_t *q, float *s_t, int64_t ld, cudaStream_t st) {
   const int64_t warps = RS * (I / 128);
   if (warps == 0) return cudaSuccess;
   const int64_t blocks = (warps + 7) / 8;
-  swiglu_bwd_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(GU, dh, RS, I, h, dGU, q, s_t, ld);
+  swiglu_bwd_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(GU, dh, row_gate, RS, I, h, dGU, q, s_t, ld);
   return cudaGetLastError();
 }
 
@@ -336,24 +340,17 @@ cudaError_t launch_wgrad_tiles(const int32_t *offsets, int Nr, int Ns, int64_t R
 }
 
 cudaError_t launch_colquant(int src, const int4 *tiles, const int32_t *meta, int max_tiles, const float *f32rows,
-                            int64_t f32_ld, const void *bf16rows, const int32_t *row_src, const float *row_gate,
-                            int64_t R, int C, uint8_t *out, int64_t out_ld, float *s_t, cudaStream_t st) {
+                            int64_t f32_ld, const void *bf16rows, const int32_t *row_src, int64_t R, int C,
+                            uint8_t *out, int64_t out_ld, float *s_t, cudaStream_t st) {
   if (max_tiles <= 0) return cudaSuccess;
   const dim3 grid(static_cast<unsigned>(max_tiles), static_cast<unsigned>(C / kColCh));
   const auto *b = static_cast<const uint16_t *>(bf16rows);
-  switch (src) {
-    case COL_F32:
-      colquant_kernel<COL_F32><<<grid, 256, 0, st>>>(tiles, meta, max_tiles, f32rows, f32_ld, b, row_src, row_gate,
-                                                      R, C, out, out_ld, s_t);
-      break;
-    case COL_DY:
-      colquant_kernel<COL_DY><<<grid, 256, 0, st>>>(tiles, meta, max_tiles, f32rows, f32_ld, b, row_src, row_gate,
-                                                     R, C, out, out_ld, s_t);
-      break;
-    default:
-      colquant_kernel<COL_X><<<grid, 256, 0, st>>>(tiles, meta, max_tiles, f32rows, f32_ld, b, row_src, row_gate,
-                                                    R, C, out, out_ld, s_t);
-  }
+  if (src == COL_F32)
+    colquant_kernel<COL_F32><<<grid, 256, 0, st>>>(tiles, meta, max_tiles, f32rows, f32_ld, b, row_src, R, C, out,
+                                                    out_ld, s_t);
+  else
+    colquant_kernel<COL_TOKEN><<<grid, 256, 0, st>>>(tiles, meta, max_tiles, f32rows, f32_ld, b, row_src, R, C, out,
+                                                      out_ld, s_t);
   return cudaGetLastError();
 }
 

@@ -404,10 +404,12 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 // quotient (Markstein's division by reciprocal, as presented in Muller et al.,
 // "Handbook of Floating-Point Arithmetic", chapter on division) -- used where
 // many values share one divisor; b > 0 normal, a/b far from over/underflow.
+// With b > 0 the quotient carries a's sign; copysignf keeps it for a = -0,
+// where the residual step would otherwise return +0 (-0 + +0 = +0).
 __device__ __forceinline__ float div_by_recip(float a, float b, float y) {
   const float q0 = a * y;
   const float r = fmaf(-b, q0, a);
-  return fmaf(r, y, q0);
+  return copysignf(fmaf(r, y, q0), a);
 }
 
 // Two independent FP32 fused multiply-adds in one instruction:

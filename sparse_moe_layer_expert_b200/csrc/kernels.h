@@ -146,17 +146,17 @@ cudaError_t launch_ep_combine(const void *x, const void *y_sh, const void *back,
 // Backward of the expert FFNs (backward.cu, gemm_wgrad.cu).
 cudaError_t launch_transpose_blocks(const uint8_t *q, const float *s, int64_t n, int64_t k, int64_t batch,
                                     uint8_t *qt, float *st, cudaStream_t stream);
-cudaError_t launch_dy_quant(const void *dout, const int32_t *row_src, const float *row_gate, int64_t R, int64_t RS,
-                            int H, uint8_t *q, float *s_t, int64_t ld, cudaStream_t st);
-cudaError_t launch_swiglu_bwd(const float *GU, const float *dh, int64_t RS, int I, float *h, float *dGU, uint8_t *q,
+cudaError_t launch_dout_quant(const void *dout, const int32_t *row_src, int64_t R, int64_t RS, int H, uint8_t *q,
                               float *s_t, int64_t ld, cudaStream_t st);
+cudaError_t launch_swiglu_bwd(const float *GU, const float *dh, const float *row_gate, int64_t RS, int I, float *h,
+                              float *dGU, uint8_t *q, float *s_t, int64_t ld, cudaStream_t st);
 cudaError_t launch_wgrad_tiles(const int32_t *offsets, int Nr, int Ns, int64_t R, int64_t T, int32_t *seg,
                                int4 *tiles, int32_t *meta, cudaStream_t st);
-// src: 0 = FP32 rows (f32rows, f32_ld floats apart), 1 = dY from bf16 dout
-// rows gathered by token times the row gate, 2 = bf16 rows gathered by token
+// src: 0 = FP32 rows (f32rows, f32_ld floats apart), 1 = bf16 [T, C] rows
+// gathered by the row's token (row_src for p < R, p - R after)
 cudaError_t launch_colquant(int src, const int4 *tiles, const int32_t *meta, int max_tiles, const float *f32rows,
-                            int64_t f32_ld, const void *bf16rows, const int32_t *row_src, const float *row_gate,
-                            int64_t R, int C, uint8_t *out, int64_t out_ld, float *s_t, cudaStream_t st);
+                            int64_t f32_ld, const void *bf16rows, const int32_t *row_src, int64_t R, int C,
+                            uint8_t *out, int64_t out_ld, float *s_t, cudaStream_t st);
 
 // Weight-gradient GEMM: dW[e] = A_e^T B_e over each expert's token segment.
 struct WgradLaunch {

@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported(m):
 
 
 def test_status_strings_and_version(m):
-    assert m.lib.moe_abi_version() == 103
+    assert m.lib.moe_abi_version() == 104
     assert m.lib.moe_status_string(0) == b"ok"
     assert b"128" in m.lib.moe_status_string(m.MOE_ERR_UNSUPPORTED_SHAPE)
     assert m.lib.moe_status_string(12345) == b"unknown status"
@@ -71,6 +71,31 @@ def test_gemm_variant_switch(m):
         assert L.moe_set_gemm_variant(v) == m.MOE_OK
     assert L.moe_set_gemm_variant(3) == m.MOE_ERR_INVALID_ARG
     assert L.moe_set_gemm_variant(-1) == m.MOE_ERR_INVALID_ARG
+
+
+def test_gemm_kernel_choice(m):
+    v3 = m.config(7168, 2048, 256, 8, 1, 8, 4)
+    try:
+        # AUTO: CTA pairs once the routed experts average 256 rows (T * 8 >= 256 * 256)
+        assert m.moe_gemm_kernel_for(v3, 64) == m.MOE_GEMM_SINGLE
+        assert m.moe_gemm_kernel_for(v3, 4096) == m.MOE_GEMM_SINGLE
+        assert m.moe_gemm_kernel_for(v3, 8191) == m.MOE_GEMM_SINGLE
+        assert m.moe_gemm_kernel_for(v3, 8192) == m.MOE_GEMM_PAIR
+        assert m.moe_gemm_kernel_for(v3, 16384) == m.MOE_GEMM_PAIR
+        # hidden 7168 = 56 blocks pairs up; 640 = 5 blocks does not
+        odd = m.config(640, 256, 16, 4, 1, 0, 0)
+        assert m.moe_gemm_kernel_for(odd, 4096) == m.MOE_GEMM_SINGLE
+        m.moe_set_gemm_variant(m.MOE_GEMM_PAIR)
+        assert m.moe_gemm_kernel_for(v3, 64) == m.MOE_GEMM_PAIR
+        assert m.moe_gemm_kernel_for(odd, 64) == m.MOE_GEMM_SINGLE
+        m.moe_set_gemm_variant(m.MOE_GEMM_SINGLE)
+        assert m.moe_gemm_kernel_for(v3, 16384) == m.MOE_GEMM_SINGLE
+        pow2 = m.config(7168, 2048, 256, 8, 1, 8, 4, scale_mode=m.MOE_SCALE_POW2)
+        assert m.moe_gemm_kernel_for(pow2, 16384) == m.MOE_GEMM_BLOCK_SCALED
+        with pytest.raises(m.MoeError):
+            m.moe_gemm_kernel_for(v3, -1)
+    finally:
+        m.moe_set_gemm_variant(m.MOE_GEMM_AUTO)
 
 
 def test_contraction_and_alignment_limits_without_device(m):

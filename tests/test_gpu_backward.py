@@ -6,13 +6,16 @@ tails) and on one expert at full DeepSeek-V3 size ("DeepSeek-V3 Technischer
 Bericht", Kernideen, FP8 bullet: E4M3 for all tensors; the backward tile
 orientation is the reading the oracle documents).  Tolerance: the layer's
 stated bound (relative Frobenius error 2e-3, max |diff| 1e-2 rms) on every
-FP32 output."""
+FP32 output, the max bound widened by what codes of the FP32 intermediates
+dG, dU and g*h at a rounding near-tie can change (either code is a correct
+result there; near_tie_steps); the intermediates themselves agree to FP32
+rounding."""
 import numpy as np
 import pytest
 import torch
 
 import moe_synth as S
-from _moe_util import NEAR_TIE, Problem, assert_close, oracle_cfg
+from _moe_util import NEAR_TIE, Problem, assert_close, near_tie_steps, oracle_cfg, tiles_128x1, tiles_1x128
 from test_gpu_layer import build_gpu_layer
 
 pytestmark = pytest.mark.gpu
@@ -24,7 +27,46 @@ def m():
     return pkg
 
 
-def run_backward_case(m, oracle_lib, cfg, T, seed, bias_shift=None, tokens_checked=None):
+def expert_tie_allowance(oracle_lib, OB, dec, r, x_rows, d_rows, W13q, s13):
+    """What codes at a rounding near-tie of the FP32 intermediates dG, dU
+    (1x128 along I for dx, 128x1 along tokens for dW13) and g*h (128x1 for
+    dW2) can change: per dx row [rows, H], dW13 [2I, H] and dW2 [H, I]
+    (near_tie_steps).  The other operand of each GEMM is the oracle's:
+    the dequantized weights, the 128x1-quantized x and dout rows."""
+    I = r["dG"].shape[1]
+    rows = r["dG"].shape[0]
+    H = W13q.shape[1]
+    W = np.asarray(W13q)
+    s13 = np.asarray(s13, np.float64)
+    dx_a = np.zeros((rows, H))
+    for half, name in ((0, "dG"), (1, "dU")):
+        v = r[name].astype(np.float32)
+        _, s1 = oracle_lib.quant_1x128_f32(v)
+        st = near_tie_steps(v, tiles_1x128(s1), dec)
+        for p, i in zip(*np.nonzero(st)):
+            row = half * I + i
+            dx_a[p] += st[p, i] * np.abs(dec[W[row]] * np.repeat(s13[row // 128], 128))
+    xq, xs = OB.quant_128x1_bf16(x_rows)
+    xd = np.abs(dec[xq] * tiles_128x1(xs, rows))
+    dW13_a = np.zeros((2 * I, H))
+    for half, name in ((0, "dG"), (1, "dU")):
+        v = r[name].astype(np.float32)
+        _, sc = OB.quant_128x1_f32(v)
+        st = near_tie_steps(v, tiles_128x1(sc, rows), dec)
+        for t, i in zip(*np.nonzero(st)):
+            dW13_a[half * I + i] += st[t, i] * xd[t]
+    dq, ds = OB.quant_128x1_f32(np.ascontiguousarray(d_rows, np.float32))
+    dd = np.abs(dec[dq] * tiles_128x1(ds, rows))
+    v = r["gh"].astype(np.float32)
+    _, sc = OB.quant_128x1_f32(v)
+    st = near_tie_steps(v, tiles_128x1(sc, rows), dec)
+    dW2_a = np.zeros((H, I))
+    for t, i in zip(*np.nonzero(st)):
+        dW2_a[:, i] += st[t, i] * dd[t]
+    return dx_a, dW13_a, dW2_a
+
+
+def run_backward_case(m, oracle_lib, cfg, T, seed, bias_shift=None):
     import oracle.backward as OB
     prob = Problem(cfg, T, seed=seed)
     if bias_shift is not None:
@@ -39,7 +81,7 @@ def run_backward_case(m, oracle_lib, cfg, T, seed, bias_shift=None, tokens_check
     layer.check()
     experts = [prob.oracle_expert(oracle_lib, e) for e in range(prob.E)]
     ocf = oracle_cfg(oracle_lib, cfg)
-    ref = OB.layer_backward(ocf, prob.x, prob.wr, prob.bias, experts, dout)
+    ref = OB.layer_backward(ocf, prob.x, prob.wr, prob.bias, experts, dout, details=True)
     # the same routing on both sides (the configurations are chosen without near-ties)
     assert (ref["gap"] >= NEAR_TIE).all()
     got_idx = idx_out.cpu().numpy()
@@ -49,7 +91,6 @@ def run_backward_case(m, oracle_lib, cfg, T, seed, bias_shift=None, tokens_check
     R, E = T * Kr, prob.E
     RS = R + T * Ns
     # the backward's own intermediates, step by step against the oracle's
-    # expert backward on the same tokens
     bws, BL = layer.backward_workspace(T), m.moe_backward_workspace_layout(layer.cfg, T)
 
     def view(name, shape):
@@ -58,56 +99,42 @@ def run_backward_case(m, oracle_lib, cfg, T, seed, bias_shift=None, tokens_check
         assert n * 4 <= nb
         return bws[off:off + 4 * n].view(torch.float32).view(shape).cpu().numpy().astype(np.float64)
 
-    GU, dh, hh, dGU = view("gu", (RS, 2 * I)), view("dh", (RS, I)), view("h", (RS, I)), view("dgu", (RS, 2 * I))
+    GU, dh, gh, dGU = view("gu", (RS, 2 * I)), view("dh", (RS, I)), view("gh", (RS, I)), view("dgu", (RS, 2 * I))
     ws, L = layer.workspace(T), layer.layout(T)
     offsets = m.ws_view(ws, L, "offsets", torch.int32, (cfg["Nr"] + 1,)).cpu().numpy()
-    xu = prob.x
     d32 = dout.float().numpy()
+    dec = oracle_lib.e4m3_decode_table()
+    dx_allow = np.zeros((T, H))
+    w_allow = {}
     msgs, fails = [], []
-    for e in sorted(ref["dW13"].keys()):
-        if e < cfg["Nr"]:
-            toks, slots = np.nonzero(ref["idx"] == e)
-            order = np.argsort(toks, kind="stable")
-            toks, slots = toks[order], slots[order]
-            rows = np.arange(offsets[e], offsets[e + 1])
-            dy = (ref["gate"][toks, slots].astype(np.float32)[:, None] * d32[toks]).astype(np.float32)
-        else:
-            toks = np.arange(T)
-            rows = R + toks
-            dy = d32
-        r = OB.expert_backward(xu[torch.as_tensor(toks)], dy, *experts[e])
+    for e in sorted(ref["per_expert"].keys()):
+        toks, r = ref["per_expert"][e]
+        rows = np.arange(offsets[e], offsets[e + 1]) if e < cfg["Nr"] else R + toks
+        assert rows.size == toks.size
+        # G, U from the same x codes; dh from the same dout codes (the gate on
+        # the FP32 result); the rest FP32 elementwise: rounding apart only
         for nm, got, want in (("G", GU[rows, :I], r["G"]), ("U", GU[rows, I:], r["U"]), ("dh", dh[rows], r["dh"]),
-                              ("h", hh[rows], r["h"]), ("dG", dGU[rows, :I], r["dG"]),
+                              ("g*h", gh[rows], r["gh"]), ("dG", dGU[rows, :I], r["dG"]),
                               ("dU", dGU[rows, I:], r["dU"])):
-            rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
-            msgs.append(f"expert {e} {nm}: rel-Frobenius {rel:.2e}")
-            if not rel < 1e-4:
-                fails.append(msgs[-1])
-        # the weight-gradient GEMM on the GPU's own operands (its dY, h, dG|dU
-        # and x), quantized 128x1 by the oracle: only the GEMM's FP32 rounding
-        # separates the two
-        dyq, dys = OB.quant_128x1_f32(dy)
-        hq, hs = OB.quant_128x1_f32(hh[rows].astype(np.float32))
-        w2_own = OB.rows_scaled_gemm(dyq.T, dys.T, hq.T, hs.T)
-        gq, gs = OB.quant_128x1_f32(dGU[rows].astype(np.float32))
-        xq, xs = OB.quant_128x1_bf16(xu[torch.as_tensor(toks)])
-        w13_own = OB.rows_scaled_gemm(gq.T, gs.T, xq.T, xs.T)
-        got13, got2 = dW13[e].cpu().numpy().astype(np.float64), dW2[e].cpu().numpy().astype(np.float64)
-        for nm, got, want in (("dW13 (own operands)", got13, w13_own), ("dW2 (own operands)", got2, w2_own)):
             rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
             msgs.append(f"expert {e} {nm}: rel-Frobenius {rel:.2e}")
             if not rel < 1e-5:
                 fails.append(msgs[-1])
+        dxa, w13a, w2a = expert_tie_allowance(oracle_lib, OB, dec, r, prob.x[torch.as_tensor(toks)], d32[toks],
+                                              experts[e][0], experts[e][1])
+        dx_allow[toks] += dxa
+        w_allow[e] = (w13a, w2a)
     print("\n".join(msgs[:60]))
     assert not fails, fails[:10]
-    dx_h = dx.cpu().numpy().astype(np.float64)
-    assert_close(dx_h, ref["dx"], what="dx")
+    assert_close(dx.cpu().numpy().astype(np.float64), ref["dx"], what="dx", tie_allow=dx_allow)
     dW13_h, dW2_h = dW13.cpu().numpy(), dW2.cpu().numpy()
     used = set(ref["dW13"].keys())
     for e in range(E):
         if e in used:
-            assert_close(dW13_h[e].astype(np.float64), ref["dW13"][e], what=f"dW13 of expert {e}")
-            assert_close(dW2_h[e].astype(np.float64), ref["dW2"][e], what=f"dW2 of expert {e}")
+            assert_close(dW13_h[e].astype(np.float64), ref["dW13"][e], what=f"dW13 of expert {e}",
+                         tie_allow=w_allow[e][0])
+            assert_close(dW2_h[e].astype(np.float64), ref["dW2"][e], what=f"dW2 of expert {e}",
+                         tie_allow=w_allow[e][1])
         else:
             assert not dW13_h[e].any() and not dW2_h[e].any(), f"expert {e} has no token but a gradient"
     return ref

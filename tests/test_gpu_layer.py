@@ -13,7 +13,8 @@ import pytest
 import torch
 
 import moe_synth as S
-from _moe_util import GUARD, NEAR_TIE, STATED_NEAR_TIE, Problem, assert_close, guarded_empty, bf16_to_f64, oracle_cfg, route_sets_match, shape_of
+from _moe_util import (GUARD, NEAR_TIE, STATED_NEAR_TIE, TIE_BAND, TIE_BAND_POW2, Problem, assert_close, bf16_to_f64,
+                       guarded_empty, near_tie_steps, oracle_cfg, route_sets_match, shape_of, tiles_1x128)
 
 pytestmark = pytest.mark.gpu
 
@@ -111,7 +112,9 @@ def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts
             assert np.array_equal(layer.w2[e].cpu().numpy(), W2q)
             assert np.array_equal(layer.s2[e].cpu().numpy(), s2)
     # S4-S6: per (token, expert) FFN pieces
-    hq_got, hs_got, hq_ref, hs_ref, h_ref, y_got, y_ref = [], [], [], [], [], [], []
+    hq_got, hs_got, hq_ref, hs_ref, h_ref, y_got, y_ref, y_tie = [], [], [], [], [], [], [], []
+    tok_tie = {}
+    dec = oracle_lib.e4m3_decode_table()
     for t in tok:
         rows = [(int(pos[t, k]), int(idx[t, k]), float(gate[t, k])) for k in range(Kr)]
         if Ns:
@@ -125,22 +128,53 @@ def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts
             h_ref.append(ho[0])
             y_got.append(y[p].astype(np.float64))
             y_ref.append(g * yo[0])
+            # what codes of h at a rounding near-tie can move y by
+            y_tie.append(g * h_tie_allowance(dec, ho[0], hso[0], experts[e][2], experts[e][3], mode))
+            tok_tie[int(t)] = tok_tie.get(int(t), 0.0) + y_tie[-1]
     check_requantized(oracle_lib, np.stack(hq_got), np.stack(hs_got), np.stack(hq_ref), np.stack(hs_ref),
                       np.stack(h_ref), mode)
-    assert_close(np.stack(y_got), np.stack(y_ref), what="gate-scaled expert outputs y")
+    assert_close(np.stack(y_got), np.stack(y_ref), what="gate-scaled expert outputs y", tie_allow=np.stack(y_tie))
     # S7: layer output (near-tie tokens may legitimately pick another expert)
     tok = tok[gap[tok] >= NEAR_TIE]
     res = oracle_lib.forward(ocf, prob.x, prob.wr, prob.bias,
                              [experts.get(e) for e in range(Nr + Ns)], tokens=tok)
     assert np.array_equal(res["idx"], oi[tok])
     o32 = out32.cpu().numpy()[tok].astype(np.float64)
-    assert_close(o32, res["out"], what="layer output (fp32)")
+    out_tie = np.stack([tok_tie[int(t)] for t in tok]) if len(tok) else None
+    assert_close(o32, res["out"], what="layer output (fp32)", tie_allow=out_tie)
     out16 = layer.forward(x_d, out_dtype=m.MOE_DTYPE_BF16)
     layer.check()
     o16 = out16.cpu()[torch.as_tensor(tok)]
-    assert_close(bf16_to_f64(o16), res["out"], bf16_out=True, what="layer output (bf16)")
+    assert_close(bf16_to_f64(o16), res["out"], bf16_out=True, what="layer output (bf16)", tie_allow=out_tie)
     assert torch.equal(o16, out32.cpu()[torch.as_tensor(tok)].to(torch.bfloat16))
     return dict(counts=counts, idx=idx, n_exempt=n_exempt, n_stated_near_tie=n_stated, idx_ref=oi, s_ref=s_o)
+
+
+def h_tie_allowance(dec, h_o, hs_o, W2q, s2, mode=0):
+    """Per output channel of one row's down projection: the largest change
+    that the codes of h sitting at a rounding near-tie (near_tie_steps) can
+    make, sum_i step_i S_i |W2[:, i]|.  In the power-of-two mode a tile whose
+    amax lies within 1e-5 of a scale threshold 448 * 2^e may take the next
+    scale on the other side: every element of it may then differ by up to two
+    code steps."""
+    h_o = np.asarray(h_o, np.float64).reshape(-1)
+    S = tiles_1x128(np.asarray(hs_o).reshape(1, -1))[0]
+    steps = near_tie_steps(h_o, S, dec, TIE_BAND_POW2 if mode == 1 else TIE_BAND)
+    if mode == 1:
+        amax = np.abs(h_o).reshape(-1, 128).max(axis=1)
+        t = np.log2(np.where(amax > 0, amax, 448.0) / 448.0)
+        near_tile = np.abs(t - np.round(t)) * np.log(2) < 1e-5
+        if near_tile.any():
+            grid = np.unique(np.abs(dec[np.isfinite(dec)]))
+            q = np.abs(h_o) / np.where(S > 0, S, 1.0)
+            i = np.clip(np.searchsorted(grid, q, side="right"), 1, grid.size - 1)
+            wide = 2.0 * (grid[i] - grid[i - 1]) * S
+            steps = np.where(np.repeat(near_tile, 128), np.maximum(steps, wide), steps)
+    cols = np.nonzero(steps)[0]
+    if cols.size == 0:
+        return np.zeros(W2q.shape[0])
+    W = dec[np.asarray(W2q)[:, cols]] * np.repeat(np.asarray(s2, np.float64)[:, cols // 128], 128, axis=0)
+    return np.abs(W) @ steps[cols]
 
 
 def check_balance_loss(oracle_lib, prob: Problem, layer, r: dict, seq_len: int, alpha: float = 1e-4):
