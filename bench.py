@@ -55,6 +55,7 @@ GEMM_SOURCES = {
     "gemm_fp8_kernel": [os.path.join(_CSRC, f) for f in ("gemm.cu", "gemm_tiles.cuh", "common.cuh")],
     "gemm_mx_kernel": [os.path.join(_CSRC, f) for f in ("gemm_mx.cu", "gemm_tiles.cuh", "common.cuh")],
     "gemm_pair_kernel": [os.path.join(_CSRC, f) for f in ("gemm_pair.cu", "gemm_tiles.cuh", "common.cuh")],
+    "gemm_tall_kernel": [os.path.join(_CSRC, f) for f in ("gemm_tall.cu", "gemm_tiles.cuh", "common.cuh")],
 }
 
 
@@ -77,9 +78,9 @@ def parse(argv=None):
     p.add_argument("--scale-mode", choices=("amax", "pow2"), default="amax",
                    help="amax: S = amax/448 (the pages, default); pow2: power-of-two scales applied by the "
                         "tensor core (block-scaled MMA)")
-    p.add_argument("--gemm", choices=("auto", "single", "pair"), default="auto",
-                   help="grouped GEMM kernel of the default scale mode: the library's default (auto: single "
-                        "CTAs), single CTAs, or CTA pairs (tcgen05 cta_group::2)")
+    p.add_argument("--gemm", choices=("auto", "single", "pair", "tall"), default="auto",
+                   help="grouped GEMM kernel of the default scale mode: the library's choice (auto), single "
+                        "CTAs, CTA pairs (tcgen05 cta_group::2) or tall tiles (256 rows x 128 weight rows)")
     p.add_argument("--no-extras", action="store_true",
                    help="skip the other workloads (decode, skewed, standalone GEMM, FP8 ceiling) measured after "
                         "the headline at N = 1")
@@ -154,11 +155,15 @@ def algorithmic_counts(cfg: dict, T: int, touched_routed: int) -> dict:
                 layer_weight_bytes=E_t * (w13 + w2))
 
 
-def gemm_work(M, torch, layer, T: int, stage_ms: dict, sm_mhz, pair: bool) -> dict:
+def gemm_work(M, torch, layer, T: int, stage_ms: dict, sm_mhz, kernel: int) -> dict:
     """Work of the two grouped GEMM launches of the last forward, from the
     chunk table it left in the workspace: chunks, tiles, K blocks per
     processing unit (an SM, or a pair of SMs on the CTA-pair kernel), and the
-    cycles one K block took on average at the sampled SM clock."""
+    cycles one K block took on average at the sampled SM clock.  A tile is
+    128 rows x 256 weight rows (single CTA, CTA pair: 256 rows over two SMs)
+    or up to 256 rows x 128 weight rows (tall tiles)."""
+    pair = kernel == M.MOE_GEMM_PAIR
+    tall = kernel == M.MOE_GEMM_TALL
     import math as _m
     c = layer.cfg
     ws, L = layer.workspace(T), layer.layout(T)
@@ -166,8 +171,9 @@ def gemm_work(M, torch, layer, T: int, stage_ms: dict, sm_mhz, pair: bool) -> di
     sms = torch.cuda.get_device_properties(ws.device).multi_processor_count
     units = sms // 2 if pair else sms
     out = {}
-    for name, nb, kb in (("gemm_gate_up", c.inter // 128, c.hidden // 128),
-                         ("gemm_down", (c.hidden // 128 + 1) // 2, c.inter // 128)):
+    nb1 = 2 * (c.inter // 128) if tall else c.inter // 128
+    nb2 = 2 * (c.hidden // 256) if tall else (c.hidden // 128 + 1) // 2
+    for name, nb, kb in (("gemm_gate_up", nb1, c.hidden // 128), ("gemm_down", nb2, c.inter // 128)):
         tiles = nch * nb
         kpu = tiles * kb / units
         d = dict(chunks=nch, tiles=tiles, k_blocks=tiles * kb, k_blocks_per_unit=round(kpu, 1),
@@ -582,7 +588,8 @@ def main(argv=None):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    M.moe_set_gemm_variant({"auto": M.MOE_GEMM_AUTO, "single": M.MOE_GEMM_SINGLE, "pair": M.MOE_GEMM_PAIR}[args.gemm])
+    M.moe_set_gemm_variant({"auto": M.MOE_GEMM_AUTO, "single": M.MOE_GEMM_SINGLE, "pair": M.MOE_GEMM_PAIR,
+                            "tall": M.MOE_GEMM_TALL}[args.gemm])
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
@@ -665,8 +672,7 @@ def main(argv=None):
     counts_h = counts.cpu()
     touched = int((counts_h > 0).sum())
     gemm_kernel = M.moe_gemm_kernel_for(layer.cfg, T)
-    pair_kernel = gemm_kernel == M.MOE_GEMM_PAIR
-    work = gemm_work(M, torch, layer, T, stage_ms, clocks.get("sm_mhz"), pair_kernel)
+    work = gemm_work(M, torch, layer, T, stage_ms, clocks.get("sm_mhz"), gemm_kernel)
     # sequence-wise balance loss (alpha = 1e-4) of the batch the timed steps
     # routed, read from the last forward's workspace before anything reroutes
     seq_len = math.gcd(T, 4096)
@@ -698,8 +704,8 @@ def main(argv=None):
     fp8_src = peaks["src"] + (" bf16 sustained x 2" if sustained else " bf16 burst x 2")
     t_mem = dom_bytes / (peaks["hbm"] * 1e9)
     t_tc = dom_flops / (fp8_peak * 1e12)
-    kname = {M.MOE_GEMM_BLOCK_SCALED: "gemm_mx_kernel", M.MOE_GEMM_PAIR: "gemm_pair_kernel"}.get(gemm_kernel,
-                                                                                              "gemm_fp8_kernel")
+    kname = {M.MOE_GEMM_BLOCK_SCALED: "gemm_mx_kernel", M.MOE_GEMM_PAIR: "gemm_pair_kernel",
+             M.MOE_GEMM_TALL: "gemm_tall_kernel"}.get(gemm_kernel, "gemm_fp8_kernel")
     kernel_name = f"{kname}<0>" if dom == "gemm_gate_up" else f"{kname}<1>"
     if t_mem >= t_tc:
         achieved = dom_bytes / (dom_ms / 1e3) / 1e9

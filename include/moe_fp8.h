@@ -434,19 +434,21 @@ MOE_API int moe_ep_combine(const moe_config *cfg, int32_t world, const void *x_d
 
 /* Kernel choice of the grouped expert GEMMs in the default scale mode
  * (process-wide; a tuning and testing switch, the arithmetic is the same):
- *   MOE_GEMM_AUTO   (default) the measured-faster choice: CTA pairs when
- *                   the routed experts average >= 256 rows (T * top_k >=
- *                   256 * n_routed) and hidden is a multiple of 256, else
- *                   single CTAs
+ *   MOE_GEMM_AUTO   (default) the measured-fastest choice: single CTAs
  *   MOE_GEMM_SINGLE one CTA per tile: <= 128 rows of one expert per pass over
  *                   a weight-block pair
  *   MOE_GEMM_PAIR   a pair of CTAs on two SMs per tile (<= 256 rows per
  *                   weight pass, one tcgen05.mma.cta_group::2 per K step)
  *                   when the down projection's 128-row weight blocks pair up
  *                   (hidden a multiple of 256), else single CTAs
+ *   MOE_GEMM_TALL   tall tiles: up to 256 rows of an expert x 64 gate + 64 up
+ *                   channels (or 128 output channels) per CTA, so an expert
+ *                   of up to 256 rows streams each weight tile once; clusters
+ *                   of two exchange the requantization amax (hidden a
+ *                   multiple of 256, else single CTAs)
  * Returns MOE_ERR_INVALID_ARG for any other value.  Takes effect for the
  * next moe_forward on any thread; not synchronised with calls in flight. */
-enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SINGLE = 1, MOE_GEMM_PAIR = 2, MOE_GEMM_BLOCK_SCALED = 3 };
+enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SINGLE = 1, MOE_GEMM_PAIR = 2, MOE_GEMM_BLOCK_SCALED = 3, MOE_GEMM_TALL = 4 };
 MOE_API int moe_set_gemm_variant(int32_t variant);
 /* The grouped-GEMM kernel the next moe_forward of T tokens under cfg runs
  * with the current variant setting: MOE_GEMM_SINGLE, MOE_GEMM_PAIR, or

@@ -14,7 +14,7 @@ from ._binding import (  # noqa: F401
     fp8_blockscaled_gemm, fp8_quant_128x128, fp8_quant_1x128, lib, moe_bias_update, moe_check_device_error,
     moe_forward, moe_profile_events, moe_route, moe_route_noalloc, moe_route_workspace_size, moe_selftest_wait_timeout,
     moe_seq_balance_loss, moe_set_gemm_variant, moe_gemm_kernel_for, moe_workspace_layout, MOE_GEMM_AUTO, MOE_GEMM_PAIR,
-    MOE_GEMM_SINGLE, MOE_GEMM_BLOCK_SCALED,
+    MOE_GEMM_SINGLE, MOE_GEMM_BLOCK_SCALED, MOE_GEMM_TALL,
     moe_workspace_size, new_err_flag, weights_struct, ws_view, moe_ep_row_bytes, moe_ep_dispatch, moe_ep_experts,
     moe_ep_combine, moe_transpose_weights, moe_backward, moe_backward_workspace_layout,
 )

@@ -51,6 +51,7 @@ MOE_GEMM_AUTO = 0
 MOE_GEMM_SINGLE = 1
 MOE_GEMM_PAIR = 2
 MOE_GEMM_BLOCK_SCALED = 3
+MOE_GEMM_TALL = 4
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 16 << 20
 MOE_PROFILE_EVENTS = 7
 PROFILE_STAGES = ("quantize", "route", "group", "gemm_gate_up", "gemm_down", "combine")
@@ -293,12 +294,12 @@ def moe_profile_events(events) -> None:
 
 def moe_set_gemm_variant(variant: int) -> None:
     """Kernel choice of the grouped expert GEMMs (MOE_GEMM_AUTO, _SINGLE,
-    _PAIR), process-wide."""
+    _PAIR, _TALL), process-wide."""
     _check(lib.moe_set_gemm_variant(variant), "moe_set_gemm_variant")
 
 
 def moe_gemm_kernel_for(cfg, T: int) -> int:
-    """The grouped-GEMM kernel (MOE_GEMM_SINGLE, _PAIR or _BLOCK_SCALED) the
+    """The grouped-GEMM kernel (MOE_GEMM_SINGLE, _PAIR, _TALL or _BLOCK_SCALED) the
     next moe_forward of T tokens runs under the current variant setting."""
     r = lib.moe_gemm_kernel_for(C.byref(cfg), int(T))
     if r < 0:

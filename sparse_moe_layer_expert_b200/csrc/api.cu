@@ -132,12 +132,19 @@ constexpr int64_t kMaxTokens = 1 << 20;
 // faster on single CTAs, 512 on pairs).
 std::atomic<int> g_gemm_variant{MOE_GEMM_AUTO};
 
-bool use_pair_gemm(const moe_config *c, int64_t T) {
-  if ((c->hidden / 128) % 2 != 0) return false;
+// The grouped-GEMM kernel of a forward of T tokens (MOE_GEMM_SINGLE, _PAIR,
+// _TALL or _BLOCK_SCALED).  Pairs and tall tiles need the down projection's
+// 128-row weight blocks to pair up (H a multiple of 256).  MOE_GEMM_AUTO takes
+// single CTAs: with the tiles of an expert's chunks run side by side (one HBM
+// read of each weight tile), they were the fastest at every V3 size measured
+// (decode 64, prefill 4096 and skewed 16384 tokens).
+int gemm_kernel_for(const moe_config *c, int64_t T) {
+  (void)T;
+  if (c->scale_mode == MOE_SCALE_POW2) return MOE_GEMM_BLOCK_SCALED;
+  if ((c->hidden / 128) % 2 != 0) return MOE_GEMM_SINGLE;
   const int v = g_gemm_variant.load(std::memory_order_relaxed);
-  if (v == MOE_GEMM_PAIR) return true;
-  if (v == MOE_GEMM_SINGLE) return false;
-  return T * static_cast<int64_t>(c->top_k) >= 256 * static_cast<int64_t>(c->n_routed);
+  if (v == MOE_GEMM_PAIR || v == MOE_GEMM_TALL) return v;
+  return MOE_GEMM_SINGLE;
 }
 
 struct Carve {
@@ -214,7 +221,8 @@ const char *moe_status_string(int s) {
 int moe_abi_version(void) { return 104; }
 
 int moe_set_gemm_variant(int32_t variant) {
-  if (variant != MOE_GEMM_AUTO && variant != MOE_GEMM_SINGLE && variant != MOE_GEMM_PAIR) return MOE_ERR_INVALID_ARG;
+  if (variant != MOE_GEMM_AUTO && variant != MOE_GEMM_SINGLE && variant != MOE_GEMM_PAIR && variant != MOE_GEMM_TALL)
+    return MOE_ERR_INVALID_ARG;
   g_gemm_variant.store(variant, std::memory_order_relaxed);
   return MOE_OK;
 }
@@ -222,8 +230,7 @@ int moe_set_gemm_variant(int32_t variant) {
 int moe_gemm_kernel_for(const moe_config *cfg, int64_t T) {
   if (const int c = check_cfg(cfg)) return c;
   if (T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
-  if (cfg->scale_mode == MOE_SCALE_POW2) return MOE_GEMM_BLOCK_SCALED;
-  return use_pair_gemm(cfg, T) ? MOE_GEMM_PAIR : MOE_GEMM_SINGLE;
+  return gemm_kernel_for(cfg, T);
 }
 
 static int quant_1x128(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *q, float *scales,
@@ -436,9 +443,11 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
   int32_t *blk_base = at<int32_t *>(ws, L.blk_base);
   int4 *chunks = at<int4 *>(ws, L.chunks);
   const int64_t max_chunks = moe::max_chunks(T, Kr, Nr, Ns);
-  const bool pow2 = cfg->scale_mode == MOE_SCALE_POW2;
-  const bool pair = !pow2 && use_pair_gemm(cfg, T);
-  const int chunk_rows = pair ? 256 : 128;
+  const int kern = gemm_kernel_for(cfg, T);
+  const bool pow2 = kern == MOE_GEMM_BLOCK_SCALED;
+  const bool pair = kern == MOE_GEMM_PAIR;
+  const bool tall = kern == MOE_GEMM_TALL;
+  const int chunk_rows = pair || tall ? 256 : 128;
 
   cudaError_t e = moe::launch_hist(P.idx, T, Kr, Nr, P.allow_empty, blk_hist, err_flag, st);
   if (e == cudaSuccess)
@@ -481,7 +490,10 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
     g.ld_os = pitch;
     g.err = err_flag;
     g.wait_limit_ns = moe::kDefaultWaitLimitNs;
-    e = pow2 ? moe::launch_gemm_mx(g, st) : pair ? moe::launch_gemm_pair(g, st) : moe::launch_gemm(g, st);
+    e = pow2   ? moe::launch_gemm_mx(g, st)
+        : pair ? moe::launch_gemm_pair(g, st)
+        : tall ? moe::launch_gemm_tall(g, st)
+               : moe::launch_gemm(g, st);
   }
   if (e == cudaSuccess) e = prof_mark(4, st);
   if (e == cudaSuccess) {
@@ -503,7 +515,7 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
     g.n_chunks = meta;
     g.max_chunks = static_cast<int>(max_chunks);
     g.chunk_rows = chunk_rows;
-    g.nb = moe::gemm2_blocks(H);
+    g.nb = tall ? H / 256 : moe::gemm2_blocks(H);
     g.gate_up = 0;
     g.a_is_out_row = 1;
     g.rows_per_expert = H;
@@ -515,7 +527,10 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
     g.row_gate = row_gate;
     g.err = err_flag;
     g.wait_limit_ns = moe::kDefaultWaitLimitNs;
-    e = pow2 ? moe::launch_gemm_mx(g, st) : pair ? moe::launch_gemm_pair(g, st) : moe::launch_gemm(g, st);
+    e = pow2   ? moe::launch_gemm_mx(g, st)
+        : pair ? moe::launch_gemm_pair(g, st)
+        : tall ? moe::launch_gemm_tall(g, st)
+               : moe::launch_gemm(g, st);
   }
   if (e == cudaSuccess) e = prof_mark(5, st);
   if (e == cudaSuccess) e = moe::launch_combine(P.x_resid, y, pos, T, H, Kr, R, Ns, P.out, P.out_f32, st, true);

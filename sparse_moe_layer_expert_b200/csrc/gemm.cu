@@ -140,7 +140,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     if (warp == 0) {
       // ---------------------------------------------------------- TMA producer
       if (lane == 0) {
-        const uint64_t pol_w = policy_evict_first();
+        // weights: evict-first when one pass reads them, normal when the
+        // other chunks of the expert read the same tiles right after
+        const uint64_t pol_w1 = policy_evict_first();
+        const uint64_t pol_wk = policy_evict_normal();
         const uint64_t pol_a = policy_evict_last();
         uint32_t it = 0;
         bool stop = false;
@@ -153,6 +156,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           const CUtensorMap *amap = td.from1 ? &map_a1 : &map_a0;
           const bool two = td.w_row1 >= 0;
           const uint32_t bytes = G_AB + (two ? 2 : 1) * G_WB;
+          const uint64_t pol_w = td.group > 1 ? pol_wk : pol_w1;
           for (int kb = 0; kb < KB; ++kb, ++it) {
             const int s = it % G_STAGES;
             if (!mbar_wait(&bars->empty[s], ((it / G_STAGES) & 1) ^ 1, ctl)) {

@@ -162,7 +162,8 @@ __global__ void __launch_bounds__(X_THREADS, 1)
     if (warp == 0) {
       // ---------------------------------------------------------- TMA producer
       if (lane == 0) {
-        const uint64_t pol_w = policy_evict_first();
+        const uint64_t pol_w1 = policy_evict_first();  // one pass reads the weight tile
+        const uint64_t pol_wk = policy_evict_normal(); // the expert's other chunks read it next
         const uint64_t pol_a = policy_evict_last();
         uint32_t it = 0;
         bool stop = false;
@@ -173,6 +174,7 @@ __global__ void __launch_bounds__(X_THREADS, 1)
           const CUtensorMap *amap = td.from1 ? &map_a1 : &map_a0;
           const bool two = td.w_row1 >= 0;
           const uint32_t bytes = X_AB + (two ? 2 : 1) * X_WB;
+          const uint64_t pol_w = td.group > 1 ? pol_wk : pol_w1;
           for (int kb = 0; kb < KB; ++kb, ++it) {
             const int s = it % X_STAGES;
             if (!mbar_wait(&bars->empty[s], ((it / X_STAGES) & 1) ^ 1, ctl)) {

@@ -154,7 +154,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     if (warp == 0) {
       // ---------------------------------------------------------- TMA producer
       if (lane == 0) {
-        const uint64_t pol_w = policy_evict_first();
+        const uint64_t pol_w1 = policy_evict_first();  // one pass reads the weight tile
+        const uint64_t pol_wk = policy_evict_normal(); // the expert's other chunks read it next
         const uint64_t pol_a = policy_evict_last();
         uint32_t it = 0;
         bool stop = false;
@@ -166,6 +167,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
           const CUtensorMap *amap = td.from1 ? &map_a1 : &map_a0;
           const int32_t w_row = pair_rank() == 0 ? td.w_row0 : td.w_row1;
           const uint32_t bytes = P_WB + (sd.n > 0 ? P_AB : 0);
+          const uint64_t pol_w = td.group > 1 ? pol_wk : pol_w1;
           for (int kb = 0; kb < KB; ++kb, ++it) {
             const int s = it % P_STAGES;
             if (!mbar_wait(&bars->empty[s], ((it / P_STAGES) & 1) ^ 1, ctl)) {

@@ -40,18 +40,44 @@ struct GemmArgs {
   int64_t w_rows, a_rows0, a_rows1, out_rows, out_cols;
 };
 
-// Tile t = (chunk t / nb, weight-block pair t % nb).
+// Tile order.  Tiles t in [c0 nb, (c0 + k) nb) belong to the k chunks
+// c0 .. c0 + k - 1 of one expert; inside that range they run weight block by
+// weight block (t = c0 nb + rb k + i: chunk c0 + i, block rb), so the k tiles
+// that read the same weight tile are neighbours in the persistent walk and
+// run side by side: the weight tile comes from HBM once and from L2 for the
+// other k - 1.  An expert of one chunk keeps (chunk, block) = (t / nb, t % nb).
+__device__ __forceinline__ void tile_coords(const GemmArgs &a, int t, int &c, int &rb, int4 &ch) {
+  c = t / a.nb;
+  rb = t - c * a.nb;
+  if (!a.chunks) return;
+  ch = a.chunks[c];
+  const int k = chunk_group(ch);
+  if (k > 1) {
+    // (a table that does not describe a group keeps the plain order; every
+    // entry read stays inside the table's max_chunks entries)
+    const int c0 = c - chunk_pos(ch);
+    const int local = t - c0 * a.nb;
+    if (c0 >= 0 && c0 + k <= a.max_chunks && local >= 0 && local < k * a.nb) {
+      rb = local / k;
+      c = c0 + (local - rb * k);
+      ch = a.chunks[c];
+    }
+  }
+}
+
 __device__ __forceinline__ GemmTile get_tile(const GemmArgs &a, int t) {
-  const int c = t / a.nb, rb = t - (t / a.nb) * a.nb;
+  int c, rb;
+  int4 ch = make_int4(0, 0, 0, 0);
+  tile_coords(a, t, c, rb, ch);
   GemmTile d;
   int e;
   if (a.chunks) {
-    const int4 ch = a.chunks[c];
-    e = ch.x & 0xFFFF;
-    d.from1 = (ch.x >> 16) & 1;
+    e = chunk_expert(ch);
+    d.from1 = chunk_from1(ch);
     d.a_row = ch.y;
     d.out_row = ch.z;
-    d.n = ch.w;
+    d.n = chunk_rows_of(ch);
+    d.group = chunk_group(ch);
   } else {
     e = 0;
     d.from1 = 0;
@@ -59,6 +85,7 @@ __device__ __forceinline__ GemmTile get_tile(const GemmArgs &a, int t) {
     const int64_t rem = a.dense_M - static_cast<int64_t>(c) * a.chunk_rows;
     d.n = rem < a.chunk_rows ? static_cast<int32_t>(rem) : a.chunk_rows;
     d.out_row = d.a_row;
+    d.group = 1;
   }
   if (a.a_is_out_row) {
     d.a_row = d.out_row;
@@ -74,7 +101,6 @@ __device__ __forceinline__ GemmTile get_tile(const GemmArgs &a, int t) {
     d.w_row1 = (static_cast<int64_t>(2 * rb + 1) * 128 < a.rows_per_expert) ? d.w_row0 + 128 : -1;
     d.out_col = 2 * rb * 128;
   }
-  d.pad = 0;
   return d;
 }
 

@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(W_THREADS, 1)
       ot.out_row = td.e * args.C_out + td.mb * 128;
       ot.out_col = td.nb * 256;
       ot.from1 = 0;
-      ot.pad = 0;
+      ot.group = 1;
       tile_epilogue<EPI_F32, false>(args.epi, ot, acc0, acc1, td.two, warp, lane, nullptr, outx);
     }
   }

@@ -35,8 +35,19 @@ struct GemmTile {
   int32_t out_row;  // first output row (also the column of the transposed scales)
   int32_t out_col;  // first output column of block A's outputs
   int32_t from1;    // activations come from the second tensor map
-  int32_t pad;
+  int32_t group;    // chunks of this tile's expert (their tiles of one weight block run side by side)
 };
+
+// Chunk table entry (int4), written by build_chunks_kernel:
+//   x = expert | from1 << 16 | (index of the chunk among its expert's) << 17
+//   y = first activation row, z = first output row,
+//   w = rows | (chunks of the expert) << 16
+// Field accessors shared by every kernel that reads the table.
+__host__ __device__ inline int chunk_expert(const int4 &c) { return c.x & 0xFFFF; }
+__host__ __device__ inline int chunk_from1(const int4 &c) { return (c.x >> 16) & 1; }
+__host__ __device__ inline int chunk_pos(const int4 &c) { return (c.x >> 17) & 0x7FFF; }
+__host__ __device__ inline int chunk_rows_of(const int4 &c) { return c.w & 0xFFFF; }
+__host__ __device__ inline int chunk_group(const int4 &c) { return (c.w >> 16) & 0x7FFF; }
 
 enum EpiKind : int { EPI_SWIGLU_Q = 0, EPI_GATE_F32 = 1, EPI_BF16 = 2, EPI_F32 = 3 };
 
@@ -112,15 +123,20 @@ cudaError_t launch_copy_rows(const uint8_t *xq, int64_t xq_ld, const float *xs, 
                              int64_t T, int Ns, int H, uint8_t *ap, float *as_t, int64_t ld, cudaStream_t st);
 // Row pitch of the transposed scale tables [K/128][pitch]: R + T rounded up to
 // 4 floats (16-byte aligned rows for bulk copies); the tables carry
-// kScaleSlack floats after their last row so a 132-float copy stays in bounds.
+// kScaleSlack floats after their last row so a 260-float copy stays in bounds.
 inline int64_t scale_pitch(int64_t R, int64_t T) { return (R + T + 3) / 4 * 4; }
-constexpr int64_t kScaleSlack = 132;
+constexpr int64_t kScaleSlack = 264;
 
 cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st);
 // The same GEMM on CTA pairs (clusters of two): chunk_rows = 256, one
 // tcgen05.mma.cta_group::2 per 32-long K step over both CTAs' tiles; the
 // weight-block count per expert must be even (always true for gate/up).
 cudaError_t launch_gemm_pair(const GemmLaunch &g, cudaStream_t st);
+// Tall tiles (gemm_tall.cu): up to 256 rows per weight pass on one CTA,
+// clusters of two for the 1x128 requantization; chunk_rows 256, transposed
+// activation scales, EPI_SWIGLU_Q / EPI_GATE_F32 / EPI_F32; gate/up: nb = I/128,
+// down: nb = H/256.
+cudaError_t launch_gemm_tall(const GemmLaunch &g, cudaStream_t st);
 // The same grouped GEMM with power-of-two scales applied by the tensor core
 // (block-scaled MMA); transposed activation scales, EPI_SWIGLU_Q (with
 // power-of-two requantization) or EPI_GATE_F32 only.

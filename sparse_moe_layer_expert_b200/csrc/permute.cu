@@ -104,14 +104,15 @@ __global__ void __launch_bounds__(256) build_chunks_kernel(const int32_t *__rest
   for (int c = threadIdx.x; c < sh_chunks; c += blockDim.x) {
     const int64_t r0 = static_cast<int64_t>(c) * chunk_rows;
     const int n = static_cast<int>((T - r0) < chunk_rows ? (T - r0) : chunk_rows);
-    chunks[c] = make_int4(Nr | (1 << 16), static_cast<int>(r0), static_cast<int>(R + r0), n);
+    chunks[c] = make_int4(Nr | (1 << 16) | (c << 17), static_cast<int>(r0), static_cast<int>(R + r0),
+                          n | (sh_chunks << 16));
   }
   if (e < Nr && nch > 0) {
     const int sz = (cnt + nch - 1) / nch;  // <= chunk_rows: rows split evenly over the chunks
     for (int c = 0; c < nch; ++c) {
       const int r0 = off + c * sz;
       const int n = (cnt - c * sz) < sz ? (cnt - c * sz) : sz;
-      chunks[sh_chunks + cbase + c] = make_int4(e, r0, r0, n);
+      chunks[sh_chunks + cbase + c] = make_int4(e | (c << 17), r0, r0, n | (nch << 16));
     }
   }
   if (threadIdx.x == 0) {

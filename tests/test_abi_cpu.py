@@ -69,25 +69,27 @@ def test_gemm_variant_switch(m):
     L = m.lib
     for v in (m.MOE_GEMM_SINGLE, m.MOE_GEMM_PAIR, m.MOE_GEMM_AUTO):
         assert L.moe_set_gemm_variant(v) == m.MOE_OK
+    assert L.moe_set_gemm_variant(m.MOE_GEMM_TALL) == m.MOE_OK
+    assert L.moe_set_gemm_variant(m.MOE_GEMM_AUTO) == m.MOE_OK
     assert L.moe_set_gemm_variant(3) == m.MOE_ERR_INVALID_ARG
+    assert L.moe_set_gemm_variant(5) == m.MOE_ERR_INVALID_ARG
     assert L.moe_set_gemm_variant(-1) == m.MOE_ERR_INVALID_ARG
 
 
 def test_gemm_kernel_choice(m):
     v3 = m.config(7168, 2048, 256, 8, 1, 8, 4)
     try:
-        # AUTO: CTA pairs once the routed experts average 256 rows (T * 8 >= 256 * 256)
-        assert m.moe_gemm_kernel_for(v3, 64) == m.MOE_GEMM_SINGLE
-        assert m.moe_gemm_kernel_for(v3, 4096) == m.MOE_GEMM_SINGLE
-        assert m.moe_gemm_kernel_for(v3, 8191) == m.MOE_GEMM_SINGLE
-        assert m.moe_gemm_kernel_for(v3, 8192) == m.MOE_GEMM_PAIR
-        assert m.moe_gemm_kernel_for(v3, 16384) == m.MOE_GEMM_PAIR
+        # AUTO: single CTAs at every size
+        for T in (0, 64, 4096, 16384):
+            assert m.moe_gemm_kernel_for(v3, T) == m.MOE_GEMM_SINGLE
         # hidden 7168 = 56 blocks pairs up; 640 = 5 blocks does not
         odd = m.config(640, 256, 16, 4, 1, 0, 0)
-        assert m.moe_gemm_kernel_for(odd, 4096) == m.MOE_GEMM_SINGLE
         m.moe_set_gemm_variant(m.MOE_GEMM_PAIR)
         assert m.moe_gemm_kernel_for(v3, 64) == m.MOE_GEMM_PAIR
         assert m.moe_gemm_kernel_for(odd, 64) == m.MOE_GEMM_SINGLE
+        m.moe_set_gemm_variant(m.MOE_GEMM_TALL)
+        assert m.moe_gemm_kernel_for(v3, 4096) == m.MOE_GEMM_TALL
+        assert m.moe_gemm_kernel_for(odd, 4096) == m.MOE_GEMM_SINGLE
         m.moe_set_gemm_variant(m.MOE_GEMM_SINGLE)
         assert m.moe_gemm_kernel_for(v3, 16384) == m.MOE_GEMM_SINGLE
         pow2 = m.config(7168, 2048, 256, 8, 1, 8, 4, scale_mode=m.MOE_SCALE_POW2)

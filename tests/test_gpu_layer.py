@@ -430,25 +430,33 @@ def gemm_variant(m):
     m.moe_set_gemm_variant(m.MOE_GEMM_AUTO)
 
 
-@pytest.mark.parametrize("variant", ["single", "pair"])
+VARIANTS = ["single", "pair", "tall"]
+
+
+def set_variant(m, variant):
+    m.moe_set_gemm_variant({"single": m.MOE_GEMM_SINGLE, "pair": m.MOE_GEMM_PAIR, "tall": m.MOE_GEMM_TALL}[variant])
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
 def test_layer_gemm_variants_tiny(gemm_variant, oracle_lib, variant):
     m = gemm_variant
-    m.moe_set_gemm_variant(m.MOE_GEMM_SINGLE if variant == "single" else m.MOE_GEMM_PAIR)
+    set_variant(m, variant)
     prob = Problem(S.TINY, 256, seed=40)
     check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob))
 
 
-@pytest.mark.parametrize("variant", ["single", "pair"])
-@pytest.mark.parametrize("T", [128, 129, 256, 257, 600])
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("T", [1, 31, 33, 128, 129, 160, 256, 257, 600])
 def test_layer_gemm_variants_chunk_boundaries(gemm_variant, oracle_lib, variant, T):
     # every token sends slot 0..K_r-1 to experts 0..K_r-1 (bias far above the
     # affinity spread), so those experts hold exactly T rows each
     m = gemm_variant
-    m.moe_set_gemm_variant(m.MOE_GEMM_SINGLE if variant == "single" else m.MOE_GEMM_PAIR)
+    set_variant(m, variant)
     prob = Problem(S.TINY, T, seed=41 + T)
     kr = S.TINY["Kr"]
     prob.bias = prob.bias.clone()
     prob.bias[:kr] += 1.0
-    toks = np.unique(np.concatenate([np.arange(0, T, 9), [0, T - 1], np.arange(120, min(T, 136))]))
+    toks = np.unique(np.concatenate([np.arange(0, T, 9), [0, T - 1], np.arange(min(T, 120), min(T, 136)),
+                                     np.arange(min(T, 250), min(T, 262))]))
     r = check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob), tokens=toks)
     assert (r["counts"][:kr] == T).all()

@@ -64,6 +64,7 @@ def pick_tokens(m, layer, prob, n: int, seed: int) -> np.ndarray:
     token_of_row[R:] = np.arange(T)
     want = {}
     for _, _, out_row, rows in chunks:
+        rows &= 0xFFFF  # the expert's chunk count sits in the high bits
         for r in range(rows):
             row = out_row + r
             key = ("shared" if row >= R else "routed", r >= 128, (r % 128) // 32)
@@ -195,3 +196,29 @@ def test_v3_skewed_layer_pow2(m, oracle_lib, v3_layer_pow2):
     r = check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=False)
     c = r["counts"]
     assert c.max() >= 4 * c.mean()
+
+
+@pytest.fixture
+def tall(m):
+    m.moe_set_gemm_variant(m.MOE_GEMM_TALL)
+    yield m
+    m.moe_set_gemm_variant(m.MOE_GEMM_AUTO)
+
+
+def test_v3_prefill_layer_tall(tall, oracle_lib, v3_layer):
+    # tall tiles (up to 256 rows per weight pass): rows 128.. land in the
+    # second promotion warpgroup; pick_tokens covers every lane quarter of both
+    m = tall
+    layer, _ = v3_layer
+    prob = _problem(dict(S.PREFILL), 4096, 14, layer, "uniform")
+    assert m.moe_gemm_kernel_for(layer.cfg, 4096) == m.MOE_GEMM_TALL
+    toks = pick_tokens(m, layer, prob, 64, 14)
+    assert len(toks) >= 64
+    check_layer(m, oracle_lib, prob, layer, tokens=toks, check_weights=False)
+
+
+def test_v3_decode_layer_tall(tall, oracle_lib, v3_layer):
+    m = tall
+    layer, _ = v3_layer
+    prob = _problem(dict(S.DECODE), 64, 15, layer, "zero")
+    check_layer(m, oracle_lib, prob, layer, tokens=np.arange(64), check_weights=False)
