@@ -503,13 +503,79 @@ def time_blockscaled_gemm(M, torch, S, dev, gpu_id: str, Mrows: int, K: int, N: 
                 l2="B rotated over %d quantized copies (%.0f MB)" % (copies, copies * N * K / 1e6))
 
 
-def extra_workloads(M, torch, S, layer, args, seed: int, stream, dev, gpu_id: str, peaks: dict) -> dict:
+def time_backward(M, torch, S, layer, x, seed: int, stream, dev, gpu_id: str, peaks: dict, fp8_peak: float,
+                  fp8_src: str, steps: int = 5, warmup: int = 2) -> dict:
+    """Device time of moe_backward (routing held fixed) for the batch x that
+    the layer's last forward routed: G, U recomputed, the dgrad GEMMs
+    against the transposed weights (made once, set-up), the SwiGLU backward,
+    dx and every expert's FP32 weight gradients.  Algorithmic work: five
+    GEMMs of 2 * RS * H * I multiply-adds each counted in units of the down
+    projection (recompute 2, dh 1, dx 2, dW2 1, dW13 2: 16 RS H I flops);
+    bytes: the FP32 weight gradients written ([E, 3 I, H]) plus the weights
+    read twice (forward copy and transposed copy)."""
+    c = layer.cfg
+    H, I, E = c.hidden, c.inter, c.n_routed + c.n_shared
+    T = x.shape[0]
+    RS = T * c.top_k + T * c.n_shared
+    dout = S.gen_x(T, H, seed * 1009 + 23, device=dev)
+    dx = torch.empty((T, H), dtype=torch.float32, device=dev)
+    dW13 = torch.empty((E, 2 * I, H), dtype=torch.float32, device=dev)
+    dW2 = torch.empty((E, H, I), dtype=torch.float32, device=dev)
+    layer.forward(x, stream=stream)
+    wt = M.moe_transpose_weights(c, layer.weights(), stream=stream)
+    bws = layer.backward_workspace(T)
+
+    def bwd():
+        M.moe_backward(c, layer.weights(), wt, x, dout, layer.workspace(T), dx=dx, dW13=dW13, dW2=dW2, ws=bws,
+                       err=layer.err, stream=stream)
+
+    for _ in range(warmup):
+        bwd()
+    layer.check(stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    nf, nb = M.MOE_PROFILE_EVENTS, M.MOE_PROFILE_BWD_EVENTS
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(nf + nb)] for _ in range(steps)]
+    for e in ev + [e for row in sev for e in row]:
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(gpu_id)
+    with sampler:
+        ev[0].record(stream)
+        for k in range(steps):
+            M.moe_profile_events(sev[k])
+            bwd()
+            ev[k + 1].record(stream)
+        M.moe_profile_events(None)
+        torch.cuda.synchronize(dev)
+    layer.check(stream)
+    ms = ev[0].elapsed_time(ev[-1]) / steps
+    stage_ms = {name: round(sum(sev[k][nf + i].elapsed_time(sev[k][nf + i + 1]) for k in range(steps)) / steps, 4)
+                for i, name in enumerate(M.PROFILE_BWD_STAGES)}
+    flops = 16.0 * RS * H * I
+    wbytes = E * 3 * I * H * 4 + 2 * E * 3 * I * H
+    tfl = flops / (ms / 1e3) / 1e12
+    gbs = wbytes / (ms / 1e3) / 1e9
+    t_tc, t_mem = flops / (fp8_peak * 1e12), wbytes / (peaks["hbm"] * 1e9)
+    out = dict(workload=f"backward of the expert FFNs: T={T} H={H} I={I} E={E} (routing of the prefill batch held "
+                        "fixed), FP32 dx and weight gradients",
+               ms=round(ms, 4), tflops=round(tfl, 1), frac_fp8=round(tfl / fp8_peak, 4), fp8_peak=fp8_peak,
+               fp8_peak_src=fp8_src, algorithmic_flops=flops, weight_gradient_and_weight_bytes=wbytes,
+               achieved_gbs=round(gbs, 1), frac_hbm=round(gbs / peaks["hbm"], 4),
+               bound="hbm" if t_mem >= t_tc else "tensor",
+               roofline_ms=round(max(t_tc, t_mem) * 1e3, 4), stage_ms=stage_ms, clocks=sampler.summary())
+    del dW13, dW2, dx, wt
+    torch.cuda.empty_cache()
+    return out
+
+
+def extra_workloads(M, torch, S, layer, args, seed: int, stream, dev, gpu_id: str, peaks: dict, x=None) -> dict:
     """The other configurations of the workload set, measured in the same
     process on the same resident expert weights: the decode-shaped layer
     (T = 64, zero bias), the skewed layer (T = 16384, mixture input,
     group-limited routing 8 x 32 / top-4 groups, zero bias, then one bias
     update), the standalone block-scaled GEMM at both shapes and the device's
-    FP8 tensor ceiling."""
+    FP8 tensor ceiling; then the backward of the expert FFNs on the headline
+    batch x (FP32 gradients; default scale mode only)."""
     H, I, Nr, Kr = layer.cfg.hidden, layer.cfg.inter, layer.cfg.n_routed, layer.cfg.top_k
     res = {}
     ceil = fp8_ceiling(torch, dev, gpu_id)
@@ -571,6 +637,8 @@ def extra_workloads(M, torch, S, layer, args, seed: int, stream, dev, gpu_id: st
                  frac_of_nominal_4500=round(g["tflops"] / 4500.0, 4))
         res[f"gemm_M{Mr}_K{K}_N{N}"] = g
         torch.cuda.empty_cache()
+    if x is not None and layer.cfg.scale_mode == M.MOE_SCALE_AMAX:
+        res["backward"] = time_backward(M, torch, S, layer, x, seed, stream, dev, gpu_id, peaks, fp8_peak, fp8_src)
     return res
 
 
@@ -770,7 +838,7 @@ def main(argv=None):
     # ------------------------------------------------ other workloads (N = 1)
     extras = None
     if world == 1 and not args.no_extras and args.workload == "prefill" and not args.tokens and not args.experts:
-        extras = extra_workloads(M, torch, S, layer, args, seed, stream, dev, gpu_id, peaks)
+        extras = extra_workloads(M, torch, S, layer, args, seed, stream, dev, gpu_id, peaks, x=x)
 
     # ------------------------------------------------ CPU oracle baseline
     cpu = None

@@ -295,6 +295,13 @@ MOE_API int moe_workspace_layout(const moe_config *cfg, int64_t T, moe_ws_layout
  *   work lists, row copies) | 4 after gate/up GEMM (+SwiGLU, requant) |
  *   5 after down GEMM | 6 after combine */
 enum { MOE_PROFILE_EVENTS = 7 };
+/* With n_events >= MOE_PROFILE_EVENTS + MOE_PROFILE_BWD_EVENTS, every later
+ * moe_backward also records events[MOE_PROFILE_EVENTS + i] at:
+ *   0 start | 1 after G, U recomputed | 2 after the dout quantization and
+ *   the dh GEMM | 3 after the SwiGLU backward | 4 after the dx-rows GEMM |
+ *   5 after the dx combine | 6 after the weight-gradient tiles and the
+ *   128x1 quantizations | 7 after the dW2 GEMM | 8 after the dW13 GEMM */
+enum { MOE_PROFILE_BWD_EVENTS = 9 };
 MOE_API int moe_profile_events(void *const *events, int32_t n_events);
 
 /* ------------------------------------------------------------ backward */

@@ -7,7 +7,8 @@ binding.  Importing it raises ImportError when the library has not been built
 (`python sparse_moe_layer_expert_b200/build.py`); there is no fallback.
 """
 from ._binding import (  # noqa: F401
-    EXPORTS, LIB_PATH, MOE_PROFILE_EVENTS, MOE_ROUTE_NOALLOC_SCRATCH_BYTES, PROFILE_STAGES, MOE_DTYPE_BF16, MOE_DTYPE_F32, MOE_DEVERR_BAD_INDEX, MOE_DEVERR_TIMEOUT, MOE_ERR_CUDA,
+    EXPORTS, LIB_PATH, MOE_PROFILE_EVENTS, MOE_PROFILE_BWD_EVENTS, MOE_ROUTE_NOALLOC_SCRATCH_BYTES, PROFILE_STAGES,
+    PROFILE_BWD_STAGES, MOE_DTYPE_BF16, MOE_DTYPE_F32, MOE_DEVERR_BAD_INDEX, MOE_DEVERR_TIMEOUT, MOE_ERR_CUDA,
     MOE_ERR_DEVICE, MOE_ERR_INVALID_ARG, MOE_ERR_NO_DEVICE, MOE_ERR_NOT_IMPLEMENTED, MOE_ERR_TIMEOUT,
     MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_WORKSPACE_TOO_SMALL, MOE_OK, MOE_SCALE_AMAX, MOE_SCALE_POW2, MoeConfig, MoeWeights,
     MoeError, config, config_from,

@@ -54,7 +54,10 @@ MOE_GEMM_BLOCK_SCALED = 3
 MOE_GEMM_TALL = 4
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 16 << 20
 MOE_PROFILE_EVENTS = 7
+MOE_PROFILE_BWD_EVENTS = 9
 PROFILE_STAGES = ("quantize", "route", "group", "gemm_gate_up", "gemm_down", "combine")
+PROFILE_BWD_STAGES = ("recompute_gate_up", "dh", "swiglu_bwd", "dx_rows", "dx_combine", "wgrad_operands",
+                      "wgrad_w2", "wgrad_w13")
 
 
 class MoeConfig(C.Structure):

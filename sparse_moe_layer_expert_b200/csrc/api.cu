@@ -187,9 +187,13 @@ void make_layout(const moe_config *c, int64_t T, moe_ws_layout *L) {
   L->total = (cv.off + 255) & ~size_t(255);
 }
 
-thread_local cudaEvent_t g_prof_events[MOE_PROFILE_EVENTS];
+thread_local cudaEvent_t g_prof_events[MOE_PROFILE_EVENTS + MOE_PROFILE_BWD_EVENTS];
 thread_local bool g_prof_on = false;
+thread_local bool g_prof_bwd_on = false;
 
+inline cudaError_t prof_mark_bwd(int i, cudaStream_t st) {
+  return g_prof_bwd_on ? cudaEventRecord(g_prof_events[MOE_PROFILE_EVENTS + i], st) : cudaSuccess;
+}
 inline cudaError_t prof_mark(int i, cudaStream_t st) {
   return g_prof_on ? cudaEventRecord(g_prof_events[i], st) : cudaSuccess;
 }
@@ -873,7 +877,9 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
   const int64_t max_chunks = moe::max_chunks(T, Kr, Nr, Ns);
 
   // 128-row chunks of the forward's expert grouping (the single-CTA GEMM)
-  cudaError_t e = moe::launch_build_chunks(blk_hist, T, Kr, Nr, Ns, 128, counts, offsets, blk_base, chunks, meta,
+  cudaError_t e = prof_mark_bwd(0, st);
+  if (e == cudaSuccess)
+    e = moe::launch_build_chunks(blk_hist, T, Kr, Nr, Ns, 128, counts, offsets, blk_base, chunks, meta,
                                            nullptr, st);
   auto base_gemm = [&](moe::GemmLaunch &g) {
     g.chunks = chunks;
@@ -910,6 +916,7 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
     g.out_cols = 2 * I;
     e = moe::launch_gemm(g, st);
   }
+  if (e == cudaSuccess) e = prof_mark_bwd(1, st);
   if (e == cudaSuccess) e = moe::launch_dout_quant(dout, row_src, R, RS, H, dyq, dys, pitch, st);
   if (e == cudaSuccess) {
     // dh = g (dout W2): K = H against W2^T [E, I, H], the row's gate in the
@@ -938,7 +945,9 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
     g.out_cols = I;
     e = moe::launch_gemm(g, st);
   }
+  if (e == cudaSuccess) e = prof_mark_bwd(2, st);
   if (e == cudaSuccess) e = moe::launch_swiglu_bwd(GU, dh, row_gate, RS, I, ghbuf, dGU, dGUq, dGUs, pitch, st);
+  if (e == cudaSuccess) e = prof_mark_bwd(3, st);
   if (e == cudaSuccess) {
     // dx rows = [dG|dU] [W1; W3] (FP32): K = 2I against W13^T [E, H, 2I]
     moe::GemmLaunch g{};
@@ -965,7 +974,9 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
     e = moe::launch_gemm(g, st);
   }
   // dx_t = dout_t + the token's rows (shared, then its slots), FP32
+  if (e == cudaSuccess) e = prof_mark_bwd(4, st);
   if (e == cudaSuccess) e = moe::launch_combine(dout, dxr, pos, T, H, Kr, R, Ns, dx, 1, st, true);
+  if (e == cudaSuccess) e = prof_mark_bwd(5, st);
   // weight gradients: 128-token tiles of every expert, operands transposed
   if (e == cudaSuccess) e = moe::launch_wgrad_tiles(offsets, Nr, Ns, R, T, seg, tiles, tmeta, st);
   const int mt = static_cast<int>(B.max_tiles);
@@ -981,6 +992,7 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
   if (e == cudaSuccess)
     e = moe::launch_colquant(1, tiles, tmeta, mt, nullptr, 0, x, row_src, R, H, at<uint8_t *>(ws, B.xt), B.P,
                              at<float *>(ws, B.sx), st);
+  if (e == cudaSuccess) e = prof_mark_bwd(6, st);
   if (e == cudaSuccess) {
     moe::WgradLaunch g{};
     g.a_t = at<uint8_t *>(ws, B.dyt);
@@ -997,6 +1009,7 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
     g.wait_limit_ns = moe::kDefaultWaitLimitNs;
     e = moe::launch_gemm_wgrad(g, st);
   }
+  if (e == cudaSuccess) e = prof_mark_bwd(7, st);
   if (e == cudaSuccess) {
     moe::WgradLaunch g{};
     g.a_t = at<uint8_t *>(ws, B.dgut);
@@ -1013,6 +1026,7 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
     g.wait_limit_ns = moe::kDefaultWaitLimitNs;
     e = moe::launch_gemm_wgrad(g, st);
   }
+  if (e == cudaSuccess) e = prof_mark_bwd(8, st);
   return cuda_status(e);
 }
 
@@ -1039,14 +1053,17 @@ int moe_seq_balance_loss(const moe_config *cfg, int64_t T, int64_t seq_len, floa
 int moe_profile_events(void *const *events, int32_t n_events) {
   if (!events || n_events <= 0) {
     g_prof_on = false;
+    g_prof_bwd_on = false;
     return MOE_OK;
   }
   if (n_events < MOE_PROFILE_EVENTS) return MOE_ERR_INVALID_ARG;
-  for (int i = 0; i < MOE_PROFILE_EVENTS; ++i) {
+  const int n = n_events >= MOE_PROFILE_EVENTS + MOE_PROFILE_BWD_EVENTS ? MOE_PROFILE_EVENTS + MOE_PROFILE_BWD_EVENTS
+                                                                       : MOE_PROFILE_EVENTS;
+  for (int i = 0; i < n; ++i)
     if (!events[i]) return MOE_ERR_INVALID_ARG;
-    g_prof_events[i] = static_cast<cudaEvent_t>(events[i]);
-  }
+  for (int i = 0; i < n; ++i) g_prof_events[i] = static_cast<cudaEvent_t>(events[i]);
   g_prof_on = true;
+  g_prof_bwd_on = n > MOE_PROFILE_EVENTS;
   return MOE_OK;
 }
 
