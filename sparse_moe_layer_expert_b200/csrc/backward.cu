@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(256) transpose_blocks_kernel(const uint8_t *__
 
 // --------------------------------------------------------------- helpers
 // 16 lanes hold a 128-long group, 8 values each: amax over the group, S, the
-// codes (IEEE quotient x / S, E4M3 RNE satfinite, as the forward quantizer).
+// codes (the correctly rounded quotient x / S, E4M3 RNE satfinite, as the
+// forward quantizer).
 __device__ __forceinline__ float group_scale16(const float (&f)[8]) {
   float amax = 0.0f;
 #pragma unroll
@@ -78,13 +79,21 @@ __device__ __forceinline__ float group_scale16(const float (&f)[8]) {
   return amax / 448.0f;
 }
 
+// The correctly rounded quotient v / S of values sharing one divisor: through
+// the reciprocal y = RN(1/S) plus one residual correction (div_by_recip,
+// common.cuh) for S >= 2^-100, by the division itself below that.
+__device__ __forceinline__ float quot(float v, float S, float y) {
+  return S >= 0x1p-100f ? div_by_recip(v, S, y) : v / S;
+}
+
 __device__ __forceinline__ uint2 codes8_div(const float (&f)[8], float S) {
   uint32_t lo = 0, hi = 0;
   if (S != 0.0f) {
+    const float y = __frcp_rn(S);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) lo |= static_cast<uint32_t>(e4m3_rn_sat(f[i] / S)) << (8 * i);
+    for (int i = 0; i < 4; ++i) lo |= static_cast<uint32_t>(e4m3_rn_sat(quot(f[i], S, y))) << (8 * i);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) hi |= static_cast<uint32_t>(e4m3_rn_sat(f[4 + i] / S)) << (8 * i);
+    for (int i = 0; i < 4; ++i) hi |= static_cast<uint32_t>(e4m3_rn_sat(quot(f[4 + i], S, y))) << (8 * i);
   }
   return make_uint2(lo, hi);
 }
@@ -168,12 +177,14 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const float *__restrict
   const float Sg = ag / 448.0f, Su = au / 448.0f;
   uint32_t wg = 0, wu = 0;
   if (Sg != 0.0f) {
+    const float y = __frcp_rn(Sg);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) wg |= static_cast<uint32_t>(e4m3_rn_sat(dg[i] / Sg)) << (8 * i);
+    for (int i = 0; i < 4; ++i) wg |= static_cast<uint32_t>(e4m3_rn_sat(quot(dg[i], Sg, y))) << (8 * i);
   }
   if (Su != 0.0f) {
+    const float y = __frcp_rn(Su);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) wu |= static_cast<uint32_t>(e4m3_rn_sat(du[i] / Su)) << (8 * i);
+    for (int i = 0; i < 4; ++i) wu |= static_cast<uint32_t>(e4m3_rn_sat(quot(du[i], Su, y))) << (8 * i);
   }
   *reinterpret_cast<uint32_t *>(q + p * 2 * I + c) = wg;
   *reinterpret_cast<uint32_t *>(q + p * 2 * I + I + c) = wu;
@@ -291,8 +302,9 @@ __global__ void __launch_bounds__(256) colquant_kernel(const int4 *__restrict__ 
   __syncthreads();
   {
     const float S = fmaxf(fmaxf(part[0][c], part[1][c]), fmaxf(part[2][c], part[3][c])) / 448.0f;
+    const float y = S != 0.0f ? __frcp_rn(S) : 0.0f;
     for (int r = quarter * 32; r < quarter * 32 + 32; ++r)
-      codes[c][r] = S != 0.0f ? e4m3_rn_sat(vals[r][c] / S) : static_cast<uint8_t>(0);
+      codes[c][r] = S != 0.0f ? e4m3_rn_sat(quot(vals[r][c], S, y)) : static_cast<uint8_t>(0);
     if (quarter == 0) s_t[static_cast<int64_t>(col0 / 128) * C + c0 + c] = S;
   }
   __syncthreads();

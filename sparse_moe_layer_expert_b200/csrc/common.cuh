@@ -181,6 +181,20 @@ __device__ __forceinline__ void cp_async_wait() {
 
 // 1D bulk copy global -> shared of `bytes` (multiple of 16; both addresses
 // 16-byte aligned), completing `bytes` on `bar`.
+// 2D tiled bulk copy shared -> global (the box of the tensor map at
+// coordinates x, y; x * elem_size a multiple of 16, x and y >= 0), tracked by
+// the issuing thread's bulk groups: commit, then wait until the shared-memory
+// source has been read (wait_read) or the copy is complete (wait_all).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(

@@ -22,7 +22,14 @@
 // issuing tcgen05.mma kind::f8f6f4 (M = 128, N = 256, K = 32) into one of two
 // TMEM partials per K block, two promotion warpgroups folding the partial into
 // FP32 registers, here with a per-column multiplier sB[n] * sA[m] (packed
-// two-multiplier FMAs), and FP32 stores of the tile.  Every wait is bounded.
+// two-multiplier FMAs).  A tile has only as many K blocks as its expert has
+// 128-token tiles (one or two at prefill) but writes 128 x 256 FP32 outputs,
+// so the output stream sets the pace: the promotion threads put each 128 x
+// 128 block into shared memory as four 32-column boxes (128-byte swizzle) in
+// a ring of box slots, and one of them hands each box to a TMA store; the
+// stores drain to HBM while the next tile's K blocks are computed.  (The
+// ring holds one block next to three operand stages; fewer operand stages
+// for a deeper ring measured slower.)  Every wait is bounded.
 #include "common.cuh"
 #include "gemm_tiles.cuh"
 #include "kernels.h"
@@ -32,15 +39,17 @@ namespace moe {
 using namespace gemm_detail;
 
 namespace {
-constexpr int W_STAGES = 4;
+constexpr int W_STAGES = 3;
 constexpr int W_AB = 128 * 128;
 constexpr int W_BB = 128 * 128;
 constexpr int W_STAGE = W_AB + 2 * W_BB;
 constexpr int W_THREADS = 384;
 constexpr int W_SSLOTS = 6;
 constexpr int W_RING = 128 + 256;  // floats per slot: row scales, then column scales
-constexpr int W_OUTX = 8 * 32 * G_OPITCH;
-constexpr int W_SMEM = 1024 + W_STAGES * W_STAGE + W_SSLOTS * W_RING * 4 + W_OUTX * 4 + 256;
+constexpr int W_OBOX = 128 * 128;                // one 32-column FP32 box of 128 rows (bytes)
+constexpr int W_OSLOTS = 4;                       // box slots of the output ring (one 128 x 128 block)
+constexpr int W_OUT = W_OSLOTS * W_OBOX;
+constexpr int W_SMEM = 1024 + W_STAGES * W_STAGE + W_OUT + W_SSLOTS * W_RING * 4 + 256;
 static_assert(W_SMEM <= 232448, "shared memory budget");
 
 struct WgArgs {
@@ -50,7 +59,6 @@ struct WgArgs {
   const int32_t *seg;        // [E + 1] padded token segments (multiples of 128)
   const float *sA_t;         // [P/128][C_out]
   const float *sB_t;         // [P/128][C_in]
-  GemmArgs epi;              // output (FP32 [E * C_out, C_in]) for the shared epilogue
   int32_t *err;
   uint64_t limit_ns;
 };
@@ -72,6 +80,41 @@ struct WgTile {
   bool two;
 };
 
+// One 128 x 128 FP32 output block (this thread: row r, columns 64 wg .. +63
+// of the block, in acc) through shared memory to TMA stores: four boxes of
+// 32 columns x 128 rows (box k of the block in ring slot (nbox + k) %
+// W_OSLOTS), each row's 128 bytes in 16-byte chunks swizzled by the row
+// (chunk j at j ^ (r & 7)), as the tensor map's 128-byte swizzle expects; one
+// bulk group per box.  Before four slots are rewritten the issuing thread
+// waits until at most W_OSLOTS - 4 of its groups are still reading (the boxes
+// that last used those slots are done); all 256 promotion threads meet at
+// named barrier 2.
+__device__ __forceinline__ void store_block(const float (&acc)[64], uint8_t *ostage, const CUtensorMap *map,
+                                            int col0, int row0, int wg, int r, bool issuer, uint32_t &nbox) {
+  static_assert(W_OSLOTS >= 4 && W_OSLOTS <= 7, "ring of 4..7 box slots");
+  if (issuer) asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(W_OSLOTS - 4) : "memory");
+  named_bar_sync(2, 256);
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    uint8_t *box = ostage + ((nbox + wg * 2 + b) % W_OSLOTS) * W_OBOX + r * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = b * 32 + j * 4;
+      *reinterpret_cast<float4 *>(box + ((j ^ (r & 7)) << 4)) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+    }
+  }
+  fence_proxy_async_smem();
+  named_bar_sync(2, 256);
+  if (issuer) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      tma_store_2d(map, ostage + ((nbox + b) % W_OSLOTS) * W_OBOX, col0 + 32 * b, row0);
+      bulk_commit();
+    }
+  }
+  nbox += 4;
+}
+
 __device__ __forceinline__ WgTile wg_tile(const WgArgs &a, int t) {
   WgTile d;
   const int per = a.MB * a.NB;
@@ -91,13 +134,13 @@ __device__ __forceinline__ WgTile wg_tile(const WgArgs &a, int t) {
 
 __global__ void __launch_bounds__(W_THREADS, 1)
     gemm_wgrad_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                      const WgArgs args) {
+                      const __grid_constant__ CUtensorMap map_out, const WgArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *stages = smem;
-  float *sring = reinterpret_cast<float *>(smem + W_STAGES * W_STAGE);
-  float *outx = sring + W_SSLOTS * W_RING;
-  WgBars *bars = reinterpret_cast<WgBars *>(outx + W_OUTX);
+  uint8_t *ostage = smem + W_STAGES * W_STAGE;  // 1024-aligned: the boxes use the 128-byte swizzle
+  float *sring = reinterpret_cast<float *>(ostage + W_OUT);
+  WgBars *bars = reinterpret_cast<WgBars *>(sring + W_SSLOTS * W_RING);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -227,7 +270,7 @@ __global__ void __launch_bounds__(W_THREADS, 1)
     const int wg = (warp - 4) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;
-    uint32_t it = 0;
+    uint32_t it = 0, nbox = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
       if (named_bar_or(1, 256, *abortp != 0)) break;
       const WgTile td = wg_tile(args, tile);
@@ -270,17 +313,13 @@ __global__ void __launch_bounds__(W_THREADS, 1)
           mbar_arrive(&bars->sempty[slot]);
         }
       }
-      GemmTile ot;
-      ot.w_row0 = 0;
-      ot.w_row1 = td.two ? 128 : -1;
-      ot.a_row = 0;
-      ot.n = 128;
-      ot.out_row = td.e * args.C_out + td.mb * 128;
-      ot.out_col = td.nb * 256;
-      ot.from1 = 0;
-      ot.group = 1;
-      tile_epilogue<EPI_F32, false>(args.epi, ot, acc0, acc1, td.two, warp, lane, nullptr, outx);
+      // the tile's output: block A (columns nb*256 ..), then block B (+128)
+      const int orow = td.e * args.C_out + td.mb * 128;
+      store_block(acc0, ostage, &map_out, td.nb * 256, orow, wg, r, warp == 4 && lane == 0, nbox);
+      if (td.two) store_block(acc1, ostage, &map_out, td.nb * 256 + 128, orow, wg, r, warp == 4 && lane == 0, nbox);
     }
+    // the shared-memory source of the last stores stays valid until they are done
+    if (warp == 4 && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -299,6 +338,10 @@ cudaError_t launch_gemm_wgrad(const WgradLaunch &g, cudaStream_t st) {
     return cudaErrorInvalidValue;
   if (moe_host::encode_tmap_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b_t, g.P, g.C_in, g.P, 128, 128) != 0)
     return cudaErrorInvalidValue;
+  CUtensorMap mo;  // the FP32 output [E * C_out, C_in], 32-column x 128-row boxes
+  if (moe_host::encode_tmap_2d(&mo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.out, g.C_in,
+                               static_cast<uint64_t>(g.E) * g.C_out, g.C_in * 4, 32, 128) != 0)
+    return cudaErrorInvalidValue;
   WgArgs a{};
   a.E = g.E;
   a.MB = MB;
@@ -309,17 +352,13 @@ cudaError_t launch_gemm_wgrad(const WgradLaunch &g, cudaStream_t st) {
   a.seg = g.seg;
   a.sA_t = g.sa_t;
   a.sB_t = g.sb_t;
-  a.epi = GemmArgs{};
-  a.epi.out = g.out;
-  a.epi.ldo = g.C_in;
-  a.epi.gate_up = 0;
   a.err = g.err;
   a.limit_ns = g.wait_limit_ns;
   static std::atomic<uint64_t> attr_done{0};
   if (const cudaError_t e = smem_attr_once(gemm_wgrad_kernel, W_SMEM, attr_done)) return e;
   const int sms = moe_host::sm_count();
   const int grid = static_cast<int>(ntiles < sms ? ntiles : sms);
-  gemm_wgrad_kernel<<<grid, W_THREADS, W_SMEM, st>>>(ma, mb, a);
+  gemm_wgrad_kernel<<<grid, W_THREADS, W_SMEM, st>>>(ma, mb, mo, a);
   return cudaGetLastError();
 }
 
