@@ -34,6 +34,15 @@
 //   EPI_BF16      C = bf16(acc) (plain GEMM)
 //   EPI_F32       C = acc in FP32 (the backward's recomputed G, U and dh)
 //
+// FP32 outputs (EPI_GATE_F32, EPI_F32) leave through TMA stores: the
+// promotion threads put a 128 x 128 block into shared memory as boxes of 32
+// rows x 32 columns (128-byte swizzle) and one thread stores every box whose
+// 32 rows lie inside the tile; the rows of a tile's last, partial quarter
+// (rows beyond belong to the next chunk) are stored by their threads.  The
+// stores drain while the next tile's K blocks run (a down-projection tile has
+// only I/128 K blocks for 128 x 256 FP32 outputs).  Those two epilogues run
+// with three operand stages, which leaves room for one staged block.
+//
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warp 2 scale producer, warp 3 idle, warps 4..11 promotion +
 // epilogue (two warpgroups).  Every wait is bounded (see common.cuh) so a
@@ -61,9 +70,64 @@ constexpr int G_SA_SPAN = 132;            // activation scales copied per K bloc
 constexpr int G_AMAX = 2 * 128;           // floats, SwiGLU amax exchange (per warpgroup, per row)
 constexpr int G_WSC = 2 * 2 * G_KBMAX;    // floats: weight-scale rows of 2 tiles x 2 blocks
 constexpr int G_OUTX = 8 * 32 * G_OPITCH; // floats: one 32-row x 16-float buffer per promotion warp
-constexpr int G_SMEM =
-    1024 + G_STAGES * G_STAGE + G_SSLOTS * G_RING * 4 + G_AMAX * 4 + G_WSC * 4 + G_OUTX * 4 + 256;
-static_assert(G_SMEM <= 232448, "shared memory budget");
+constexpr int G_OBOX = 32 * 128;          // one staged output box: 32 rows x 32 FP32 columns (bytes)
+constexpr int G_OBLK = 16 * G_OBOX;       // a 128 x 128 FP32 block: 4 row quarters x 4 column boxes
+
+// Shared-memory plan per epilogue: FP32 outputs through TMA stores take three
+// operand stages and one staged block; the others four stages and the
+// per-warp transpose buffers.
+template <int EPI>
+struct GLayout {
+  static constexpr bool kTma = EPI == EPI_GATE_F32 || EPI == EPI_F32;
+  static constexpr int kStages = kTma ? 3 : 4;
+  static constexpr int kOut = kTma ? G_OBLK : G_OUTX * 4;  // bytes, directly after the stages (1024-aligned)
+  static constexpr int kSmem =
+      1024 + kStages * G_STAGE + kOut + G_SSLOTS * G_RING * 4 + G_AMAX * 4 + G_WSC * 4 + 256;
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+// Store one 128 x 128 FP32 block of a tile (this thread: row r = 32 q +
+// lane, columns 64 wg .. +63 of the block in acc, times gate) at output
+// (row0, col0): the thread writes its two 32-column boxes of quarter q, each
+// row's 128 bytes as 16-byte chunks at j ^ (lane & 7) (the tensor map's
+// 128-byte swizzle); one thread stores the boxes of the quarters whose 32
+// rows are all inside the tile's n rows; the threads of a partial quarter
+// store their own rows (row < n) directly.  The issuing thread first waits
+// until its previous stores have read the staging block; the 256 promotion
+// threads meet at named barrier 2.
+__device__ __forceinline__ void store_rows_block(const float (&acc)[64], float gate, uint8_t *ostage,
+                                                 const CUtensorMap *map, float *out, int64_t ldo, int64_t row0,
+                                                 int col0, int n, int wg, int q, int lane, bool issuer) {
+  if (issuer) bulk_wait_read();
+  named_bar_sync(2, 256);
+  const bool full_q = 32 * q + 32 <= n;
+  if (full_q) {
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      uint8_t *box = ostage + (q * 4 + wg * 2 + b) * G_OBOX + lane * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = b * 32 + j * 4;
+        *reinterpret_cast<float4 *>(box + ((j ^ (lane & 7)) << 4)) =
+            make_float4(acc[c] * gate, acc[c + 1] * gate, acc[c + 2] * gate, acc[c + 3] * gate);
+      }
+    }
+  } else if (32 * q + lane < n) {
+    float4 *dst = reinterpret_cast<float4 *>(out + (row0 + 32 * q + lane) * ldo + col0 + wg * 64);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      dst[j] = make_float4(acc[4 * j] * gate, acc[4 * j + 1] * gate, acc[4 * j + 2] * gate, acc[4 * j + 3] * gate);
+  }
+  fence_proxy_async_smem();
+  named_bar_sync(2, 256);
+  if (issuer) {
+    for (int qq = 0; qq < 4 && 32 * qq + 32 <= n; ++qq)
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb)
+        tma_store_2d(map, ostage + (qq * 4 + cb) * G_OBOX, col0 + 32 * cb, static_cast<int32_t>(row0 + 32 * qq));
+    bulk_commit();
+  }
+}
 
 struct GemmBars {
   uint64_t full[G_STAGES];
@@ -82,19 +146,23 @@ struct GemmBars {
 template <int EPI>
 __global__ void __launch_bounds__(G_THREADS, 1)
     gemm_fp8_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_a0,
-                    const __grid_constant__ CUtensorMap map_a1, const GemmArgs args) {
+                    const __grid_constant__ CUtensorMap map_a1, const __grid_constant__ CUtensorMap map_out,
+                    const GemmArgs args) {
+  using L = GLayout<EPI>;
+  constexpr int NST = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *stages = smem;
-  float *sring = reinterpret_cast<float *>(smem + G_STAGES * G_STAGE);
+  uint8_t *ostage = smem + NST * G_STAGE;  // staged FP32 block, or the per-warp transpose buffers
+  float *outx = reinterpret_cast<float *>(ostage);
+  float *sring = reinterpret_cast<float *>(ostage + L::kOut);
   float *amax_x = sring + G_SSLOTS * G_RING;
   float *wsc = amax_x + G_AMAX;
-  float *outx = wsc + G_WSC;
-  GemmBars *bars = reinterpret_cast<GemmBars *>(outx + G_OUTX);
+  GemmBars *bars = reinterpret_cast<GemmBars *>(wsc + G_WSC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < G_STAGES; ++i) {
+    for (int i = 0; i < NST; ++i) {
       mbar_init(&bars->full[i], 1);
       mbar_init(&bars->empty[i], 1);
     }
@@ -158,8 +226,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           const uint32_t bytes = G_AB + (two ? 2 : 1) * G_WB;
           const uint64_t pol_w = td.group > 1 ? pol_wk : pol_w1;
           for (int kb = 0; kb < KB; ++kb, ++it) {
-            const int s = it % G_STAGES;
-            if (!mbar_wait(&bars->empty[s], ((it / G_STAGES) & 1) ^ 1, ctl)) {
+            const int s = it % NST;
+            if (!mbar_wait(&bars->empty[s], ((it / NST) & 1) ^ 1, ctl)) {
               stop = true;
               break;
             }
@@ -174,9 +242,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         // let copies still in flight land before the CTA can exit
         int quiet = 0;
         const WaitCtl drain{&quiet, nullptr, 100000000ull};
-        const uint32_t n_inflight = it < G_STAGES ? it : G_STAGES;
+        const uint32_t n_inflight = it < NST ? it : NST;
         for (uint32_t j = it - n_inflight; j < it; ++j)
-          mbar_wait(&bars->full[j % G_STAGES], (j / G_STAGES) & 1, drain);
+          mbar_wait(&bars->full[j % NST], (j / NST) & 1, drain);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
@@ -193,9 +261,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           // D[128 activation rows, 256 (or 128) weight rows]
           const uint32_t idesc = idesc_e4m3_f32(128, two ? 256 : 128);
           for (int kb = 0; kb < KB; ++kb, ++it) {
-            const int s = it % G_STAGES;
+            const int s = it % NST;
             const uint32_t buf = it & 1;
-            if (!mbar_wait2(&bars->tempty[buf], ((it >> 1) & 1) ^ 1, &bars->full[s], (it / G_STAGES) & 1, ctl)) {
+            if (!mbar_wait2(&bars->tempty[buf], ((it >> 1) & 1) ^ 1, &bars->full[s], (it / NST) & 1, ctl)) {
               stop = true;
               break;
             }
@@ -337,8 +405,23 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         }
       }
 
-      tile_epilogue<EPI, false>(args, td, acc0, acc1, two, warp, lane, amx, outx);
+      if constexpr (L::kTma) {
+        // FP32 rows through TMA stores: block A at out_col + 64 wg, block B
+        // at +128 (down projection) or +half (a gate/up pair)
+        const int64_t cB = args.gate_up ? args.half : 128;
+        const float gt = (EPI == EPI_GATE_F32 && r < td.n) ? __ldg(args.row_gate + td.out_row + r) : 1.0f;
+        float *outp = static_cast<float *>(args.out);
+        store_rows_block(acc0, gt, ostage, &map_out, outp, args.ldo, td.out_row, td.out_col, td.n, wg, q, lane,
+                         warp == 4 && lane == 0);
+        if (two)
+          store_rows_block(acc1, gt, ostage, &map_out, outp, args.ldo, td.out_row, static_cast<int>(td.out_col + cB),
+                           td.n, wg, q, lane, warp == 4 && lane == 0);
+      } else {
+        tile_epilogue<EPI, false>(args, td, acc0, acc1, two, warp, lane, amx, outx);
+      }
     }
+    // the staged block stays valid until the last stores have read it
+    if (L::kTma && warp == 4 && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -349,10 +432,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 
 template <int EPI>
 static cudaError_t launch_epi(const CUtensorMap &mw, const CUtensorMap &m0, const CUtensorMap &m1,
-                              const GemmArgs &a, int grid, cudaStream_t st) {
+                              const CUtensorMap &mo, const GemmArgs &a, int grid, cudaStream_t st) {
   static std::atomic<uint64_t> attr_done{0};
-  if (const cudaError_t e = smem_attr_once(gemm_fp8_kernel<EPI>, G_SMEM, attr_done)) return e;
-  gemm_fp8_kernel<EPI><<<grid, G_THREADS, G_SMEM, st>>>(mw, m0, m1, a);
+  if (const cudaError_t e = smem_attr_once(gemm_fp8_kernel<EPI>, GLayout<EPI>::kSmem, attr_done)) return e;
+  gemm_fp8_kernel<EPI><<<grid, G_THREADS, GLayout<EPI>::kSmem, st>>>(mw, m0, m1, mo, a);
   return cudaGetLastError();
 }
 
@@ -367,15 +450,24 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st) {
   if (moe_host::encode_tmap_2d(&m1, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a1, K, g.a1_rows,
                                g.a1_ld ? static_cast<uint64_t>(g.a1_ld) : K, 128, 128) != 0)
     return cudaErrorInvalidValue;
+  // FP32 outputs: [out_rows, ldo] in 32 x 32 boxes for the TMA-store epilogue
+  // (the other epilogues get a copy of the weight map, never used)
+  CUtensorMap mo = mw;
+  if (g.epi == EPI_GATE_F32 || g.epi == EPI_F32) {
+    if ((g.ldo * 4) % 16 != 0 || g.out_rows <= 0 ||
+        moe_host::encode_tmap_2d(&mo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.out, static_cast<uint64_t>(g.ldo),
+                                 static_cast<uint64_t>(g.out_rows), static_cast<uint64_t>(g.ldo) * 4, 32, 32) != 0)
+      return cudaErrorInvalidValue;
+  }
   GemmArgs a = make_args(g);
   const int sms = moe_host::sm_count();
   const int64_t max_tiles = static_cast<int64_t>(g.max_chunks) * g.nb;
   const int grid = static_cast<int>(max_tiles < sms ? max_tiles : sms);
   switch (g.epi) {
-    case EPI_SWIGLU_Q: return launch_epi<EPI_SWIGLU_Q>(mw, m0, m1, a, grid, st);
-    case EPI_GATE_F32: return launch_epi<EPI_GATE_F32>(mw, m0, m1, a, grid, st);
-    case EPI_F32: return launch_epi<EPI_F32>(mw, m0, m1, a, grid, st);
-    default: return launch_epi<EPI_BF16>(mw, m0, m1, a, grid, st);
+    case EPI_SWIGLU_Q: return launch_epi<EPI_SWIGLU_Q>(mw, m0, m1, mo, a, grid, st);
+    case EPI_GATE_F32: return launch_epi<EPI_GATE_F32>(mw, m0, m1, mo, a, grid, st);
+    case EPI_F32: return launch_epi<EPI_F32>(mw, m0, m1, mo, a, grid, st);
+    default: return launch_epi<EPI_BF16>(mw, m0, m1, mo, a, grid, st);
   }
 }
 
