@@ -568,6 +568,81 @@ def time_backward(M, torch, S, layer, x, seed: int, stream, dev, gpu_id: str, pe
     return out
 
 
+def time_ep_emulated(M, torch, S, layer, seed: int, stream, dev, W: int = 8, T: int = 4096, reps: int = 3) -> dict:
+    """The expert-parallel forward of W ranks (T tokens each; rank d owns
+    routed experts [d N_r/W, (d+1) N_r/W)) with all W ranks' work run on this
+    one GPU (sparse_moe_layer_expert_b200.ep.LibraryOps; the all-to-all
+    exchanges are device copies between the ranks' buffers).  Device time of
+    each phase from CUDA events around it, summed over the ranks and divided
+    by W: the compute one rank of a W-GPU run does per layer.  The bytes each
+    rank would send and receive over NVLink give the exchange time at the
+    pool's measured 770 GB/s per direction (a projection: no NVLink here)."""
+    from sparse_moe_layer_expert_b200.ep import LibraryOps, LocalExchange
+    ops = [LibraryOps(layer, W, r) for r in range(W)]
+    xs = [S.gen_x(T, layer.cfg.hidden, seed * 1009 + 31 + r, device=dev) for r in range(W)]
+    H = layer.cfg.hidden
+    phases = ("quant_route", "dispatch", "exchange_rows", "experts", "exchange_back", "shared", "combine")
+    acc = {k: 0.0 for k in phases}
+
+    def timed(name, fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        r = fn()
+        e1.record(stream)
+        return r, (name, e0, e1)
+
+    sent = back_bytes = 0
+    for it in range(reps + 1):  # the first round is a warm-up
+        evs = []
+        st, disp = [], []
+        for r in range(W):
+            v, e = timed("quant_route", lambda: ops[r].quant_route(xs[r]))
+            st.append(v)
+            evs.append(e)
+        for r in range(W):
+            v, e = timed("dispatch", lambda: ops[r].dispatch(*st[r]))
+            disp.append(v)
+            evs.append(e)
+        send_counts = [d[1] for d in disp]
+        recv, e = timed("exchange_rows", lambda: LocalExchange.rows([d[0] for d in disp], send_counts))
+        evs.append(e)
+        partial = []
+        for d in range(W):
+            v, e = timed("experts", lambda: ops[d].experts(recv[d]))
+            partial.append(v)
+            evs.append(e)
+        recv_counts = LocalExchange.counts(send_counts)
+        back, e = timed("exchange_back", lambda: LocalExchange.rows(partial, recv_counts))
+        evs.append(e)
+        for r in range(W):
+            y_sh, e = timed("shared", lambda: ops[r].shared(disp[r][3]))
+            evs.append(e)
+            _, e = timed("combine", lambda: ops[r].combine(xs[r], disp[r][2], back[r], y_sh))
+            evs.append(e)
+        torch.cuda.synchronize(dev)
+        layer.check(stream)
+        if it > 0:
+            for name, e0, e1 in evs:
+                acc[name] += e0.elapsed_time(e1) / reps
+        sent = sum(sum(c) - c[r] for r, c in enumerate(send_counts)) / W
+        back_bytes = sent * H * 2
+    row_bytes = M.moe_ep_row_bytes(layer.cfg)
+    per_rank = {k: round(v / W, 4) for k, v in acc.items()}
+    compute = sum(v for k, v in per_rank.items() if not k.startswith("exchange"))
+    nvl = 770.0
+    t_send = sent * row_bytes / (nvl * 1e9) * 1e3
+    t_back = back_bytes / (nvl * 1e9) * 1e3
+    return dict(workload=f"expert parallelism emulated on one GPU: W={W} ranks x T={T} tokens, V3 layer, rank d owns "
+                         f"{layer.cfg.n_routed // W} routed experts",
+                ms_per_rank=per_rank, compute_ms_per_rank=round(compute, 4),
+                tokens_per_s_per_rank_compute=round(T / (compute / 1e3), 1),
+                rows_sent_to_other_ranks_per_rank=round(sent, 1), row_bytes=row_bytes,
+                nvlink_projection_ms=dict(send=round(t_send, 4), back=round(t_back, 4),
+                                          how="bytes one rank sends to the other ranks / 770 GB/s per direction "
+                                              "(the pool's measured peer copy); the exchanges here are device "
+                                              "copies, not NVLink"))
+
+
 def extra_workloads(M, torch, S, layer, args, seed: int, stream, dev, gpu_id: str, peaks: dict, x=None) -> dict:
     """The other configurations of the workload set, measured in the same
     process on the same resident expert weights: the decode-shaped layer
@@ -639,6 +714,9 @@ def extra_workloads(M, torch, S, layer, args, seed: int, stream, dev, gpu_id: st
         torch.cuda.empty_cache()
     if x is not None and layer.cfg.scale_mode == M.MOE_SCALE_AMAX:
         res["backward"] = time_backward(M, torch, S, layer, x, seed, stream, dev, gpu_id, peaks, fp8_peak, fp8_src)
+    if layer.cfg.n_routed % 8 == 0 and layer.cfg.n_shared == 1:
+        res["expert_parallel_emulated"] = time_ep_emulated(M, torch, S, layer, seed, stream, dev)
+        torch.cuda.empty_cache()
     return res
 
 
