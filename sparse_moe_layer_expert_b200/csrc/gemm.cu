@@ -34,6 +34,14 @@
 //   EPI_BF16      C = bf16(acc) (plain GEMM)
 //   EPI_F32       C = acc in FP32 (the backward's recomputed G, U and dh)
 //
+// Rows over TMEM lanes: the MMA issuer (warp 1) shares sub-partition 1 with
+// the promotion warps of TMEM lanes 32..63, which its instruction issue
+// slows; so the tile's last 32 rows (often padding in a short chunk, whose
+// warps then skip their reads) go to lanes 32..63: tile rows 0-31 / 32-63 /
+// 64-95 / 96-127 sit in lanes 0-31 / 64-95 / 96-127 / 32-63.  The
+// activation tile is loaded as four 32-row TMA boxes into those places (only
+// the boxes the chunk has rows in).
+//
 // FP32 outputs (EPI_GATE_F32, EPI_F32) leave through TMA stores: the
 // promotion threads put a 128 x 128 block into shared memory as boxes of 32
 // rows x 32 columns (128-byte swizzle) and one thread stores every box whose
@@ -71,6 +79,13 @@ constexpr int G_AMAX = 2 * 128;           // floats, SwiGLU amax exchange (per w
 constexpr int G_WSC = 2 * 2 * G_KBMAX;    // floats: weight-scale rows of 2 tiles x 2 blocks
 constexpr int G_OUTX = 8 * 32 * G_OPITCH; // floats: one 32-row x 16-float buffer per promotion warp
 constexpr int G_OBOX = 32 * 128;          // one staged output box: 32 rows x 32 FP32 columns (bytes)
+constexpr int G_ABOX = 32 * 128;          // one 32-row activation box
+// TMEM lane quarter of tile-row quarter qa, and the tile-row quarter of lane quarter q
+__host__ __device__ constexpr int lane_q_of_rows(int qa) { return qa == 0 ? 0 : (qa == 3 ? 1 : qa + 1); }
+__host__ __device__ constexpr int rows_q_of_lane(int q) { return q == 0 ? 0 : (q == 1 ? 3 : q - 1); }
+static_assert(rows_q_of_lane(lane_q_of_rows(0)) == 0 && rows_q_of_lane(lane_q_of_rows(1)) == 1 &&
+                  rows_q_of_lane(lane_q_of_rows(2)) == 2 && rows_q_of_lane(lane_q_of_rows(3)) == 3,
+              "row quarters and lane quarters are inverse maps");
 constexpr int G_OBLK = 16 * G_OBOX;       // a 128 x 128 FP32 block: 4 row quarters x 4 column boxes
 
 // Shared-memory plan per epilogue: FP32 outputs through TMA stores take three
@@ -97,7 +112,7 @@ struct GLayout {
 // threads meet at named barrier 2.
 __device__ __forceinline__ void store_rows_block(const float (&acc)[64], float gate, uint8_t *ostage,
                                                  const CUtensorMap *map, float *out, int64_t ldo, int64_t row0,
-                                                 int col0, int n, int wg, int q, int lane, bool issuer) {
+                                                 int col0, int n, int wg, int q, int lane, bool issuer) {  // q: row quarter
   if (issuer) bulk_wait_read();
   named_bar_sync(2, 256);
   const bool full_q = 32 * q + 32 <= n;
@@ -223,7 +238,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           if (!tile_ok(args, td)) continue;
           const CUtensorMap *amap = td.from1 ? &map_a1 : &map_a0;
           const bool two = td.w_row1 >= 0;
-          const uint32_t bytes = G_AB + (two ? 2 : 1) * G_WB;
+          const int nbox = (td.n + 31) / 32;  // activation boxes holding the chunk's rows (1..4)
+          const uint32_t bytes = nbox * G_ABOX + (two ? 2 : 1) * G_WB;
           const uint64_t pol_w = td.group > 1 ? pol_wk : pol_w1;
           for (int kb = 0; kb < KB; ++kb, ++it) {
             const int s = it % NST;
@@ -234,7 +250,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             uint8_t *st = stages + s * G_STAGE;
             mbar_arrive_expect_tx(&bars->full[s], bytes);
             const int x = kb * 128;
-            tma_load_2d_hint(st, amap, &bars->full[s], x, td.a_row, pol_a);
+            for (int b = 0; b < nbox; ++b)
+              tma_load_2d_hint(st + lane_q_of_rows(b) * G_ABOX, amap, &bars->full[s], x, td.a_row + 32 * b, pol_a);
             tma_load_2d_hint(st + G_AB, &map_w, &bars->full[s], x, td.w_row0, pol_w);
             if (two) tma_load_2d_hint(st + G_AB + G_WB, &map_w, &bars->full[s], x, td.w_row1, pol_w);
           }
@@ -354,7 +371,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     // ------------------------------------------------- promotion + epilogue
     const int wg = (warp - 4) >> 2;  // which 64 columns of each weight block
     const int q = warp & 3;          // TMEM lane quarter
-    const int r = q * 32 + lane;     // activation row of this thread inside the tile
+    const int rq = rows_q_of_lane(q);  // the tile rows those lanes hold
+    const int r = rq * 32 + lane;    // activation row of this thread inside the tile
     float *amx = amax_x;             // [2 warpgroups][128 rows]
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -365,7 +383,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const int soff = args.sa_transposed ? (td.out_row & 3) : 0;  // row offset inside a scale slot
       // a warp whose 32 rows are all padding (short chunks) skips its TMEM
       // reads and FMAs; it still takes every wait and arrival of the ring
-      const bool live = q * 32 < td.n;
+      const bool live = rq * 32 < td.n;
       float acc0[64], acc1[64];
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
@@ -411,13 +429,13 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         const int64_t cB = args.gate_up ? args.half : 128;
         const float gt = (EPI == EPI_GATE_F32 && r < td.n) ? __ldg(args.row_gate + td.out_row + r) : 1.0f;
         float *outp = static_cast<float *>(args.out);
-        store_rows_block(acc0, gt, ostage, &map_out, outp, args.ldo, td.out_row, td.out_col, td.n, wg, q, lane,
+        store_rows_block(acc0, gt, ostage, &map_out, outp, args.ldo, td.out_row, td.out_col, td.n, wg, rq, lane,
                          warp == 4 && lane == 0);
         if (two)
           store_rows_block(acc1, gt, ostage, &map_out, outp, args.ldo, td.out_row, static_cast<int>(td.out_col + cB),
-                           td.n, wg, q, lane, warp == 4 && lane == 0);
+                           td.n, wg, rq, lane, warp == 4 && lane == 0);
       } else {
-        tile_epilogue<EPI, false>(args, td, acc0, acc1, two, warp, lane, amx, outx);
+        tile_epilogue<EPI, false>(args, td, acc0, acc1, two, warp, lane, amx, outx, rq);
       }
     }
     // the staged block stays valid until the last stores have read it
@@ -445,10 +463,11 @@ cudaError_t launch_gemm(const GemmLaunch &g, cudaStream_t st) {
   const uint64_t K = static_cast<uint64_t>(g.K);
   if (moe_host::encode_tmap_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w, K, g.w_rows, K, 128, 128) != 0)
     return cudaErrorInvalidValue;
-  if (moe_host::encode_tmap_2d(&m0, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a0, K, g.a0_rows, K, 128, 128) != 0)
+  // activations in 32-row boxes (placed in the lane quarters above)
+  if (moe_host::encode_tmap_2d(&m0, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a0, K, g.a0_rows, K, 128, 32) != 0)
     return cudaErrorInvalidValue;
   if (moe_host::encode_tmap_2d(&m1, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a1, K, g.a1_rows,
-                               g.a1_ld ? static_cast<uint64_t>(g.a1_ld) : K, 128, 128) != 0)
+                               g.a1_ld ? static_cast<uint64_t>(g.a1_ld) : K, 128, 32) != 0)
     return cudaErrorInvalidValue;
   // FP32 outputs: [out_rows, ldo] in 32 x 32 boxes for the TMA-store epilogue
   // (the other epilogues get a copy of the weight map, never used)

@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(X_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty);  // TMEM goes back to the tensor core
       ++tcount;
-      tile_epilogue<EPI, true>(args, td, acc0, acc1, two, warp, lane, amx, outx);
+      tile_epilogue<EPI, true>(args, td, acc0, acc1, two, warp, lane, amx, outx, warp & 3);
     }
   }
 

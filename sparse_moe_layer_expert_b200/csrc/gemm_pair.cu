@@ -340,7 +340,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
           mbar_arrive(&bars->sempty[slot]);
         }
       }
-      if (sd.n > 0) tile_epilogue<EPI, false>(args, sd, acc0, acc1, true, warp, lane, amx, outx);
+      if (sd.n > 0) tile_epilogue<EPI, false>(args, sd, acc0, acc1, true, warp, lane, amx, outx, warp & 3);
     }
   }
 

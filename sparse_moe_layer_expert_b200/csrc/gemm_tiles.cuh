@@ -133,11 +133,13 @@ __device__ __forceinline__ bool tile_ok(const GemmArgs &a, const GemmTile &d) {
 constexpr int G_OPITCH = 20;  // floats per row of an output transpose buffer (16 + pad)
 
 template <int EPI, bool POW2>
+// rq: the tile-row quarter whose rows the thread's TMEM lane quarter holds
+// (the lane quarter itself unless the kernel permutes rows over lanes).
 __device__ __forceinline__ void tile_epilogue(const GemmArgs &args, const GemmTile &td, float (&acc0)[64],
                                               float (&acc1)[64], bool two, int warp, int lane, float *amx,
-                                              float *outx) {
+                                              float *outx, int rq) {
   const int wg = (warp - 4) >> 2;
-  const int q = warp & 3;
+  const int q = rq;
   const int r = q * 32 + lane;
   const bool valid = r < td.n;
   const int64_t orow = static_cast<int64_t>(td.out_row) + r;
