@@ -6,6 +6,8 @@
 #include <atomic>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -83,6 +85,16 @@ int check_device() {
   if (major != 10) return MOE_ERR_NO_DEVICE;
   return MOE_OK;
 }
+
+// NVTX ranges (host side, header-only NVTX3: inert unless a profiler is
+// attached) around each public call and the stages of the layer, so that a
+// timeline tool can attribute launches to them.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 int check_cfg(const moe_config *c) {
   if (!c) return MOE_ERR_INVALID_ARG;
@@ -281,6 +293,7 @@ int fp8_quant_128x128_pow2(const void *w, int64_t n, int64_t k, uint8_t *q, floa
 
 int fp8_blockscaled_gemm(const uint8_t *A, const float *sA, const uint8_t *B, const float *sB, void *C, int64_t M,
                          int64_t N, int64_t K, int32_t *err_flag, void *stream) {
+  const NvtxRange nvtx_call("fp8_blockscaled_gemm");
   if (M < 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
   if (N % 128 || K % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return MOE_OK;
@@ -327,6 +340,7 @@ size_t moe_route_workspace_size(const moe_config *cfg, int64_t T) {
 
 int moe_route(const moe_config *cfg, const void *x, const void *wr, const float *bias, int64_t T, int32_t *idx,
               float *gate, int32_t *counts, void *ws, size_t ws_bytes, int32_t *err_flag, void *stream) {
+  const NvtxRange nvtx_call("moe_route");
   if (const int c = check_cfg(cfg)) return c;
   if (T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
   if (!counts) return MOE_ERR_INVALID_ARG;
@@ -462,6 +476,7 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
   if (e == cudaSuccess) e = moe::launch_copy_rows(P.xq, P.xq_ld, P.xs, row_src, R, T, Ns, H, ap, as_t, pitch, st);
   if (e == cudaSuccess) e = prof_mark(3, st);
   if (e == cudaSuccess) {
+    const NvtxRange nvtx_stage("gemm_gate_up");
     // gate/up projection + SwiGLU + 1x128 requantization
     moe::GemmLaunch g{};
     g.w = w->w13_dev;
@@ -501,6 +516,7 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
   }
   if (e == cudaSuccess) e = prof_mark(4, st);
   if (e == cudaSuccess) {
+    const NvtxRange nvtx_stage("gemm_down");
     // down projection, scaled by the gate of each row
     moe::GemmLaunch g{};
     g.w = w->w2_dev;
@@ -545,6 +561,7 @@ static cudaError_t run_expert_path(const ExpertPath &P) {
 int moe_forward(const moe_config *cfg, const moe_weights *w, const float *bias, const void *x, int64_t T, void *out,
                 int32_t out_dtype, int32_t *idx_out, int32_t *counts_out, void *ws, size_t ws_bytes,
                 int32_t *err_flag, void *stream) {
+  const NvtxRange nvtx_call("moe_forward");
   if (const int c = check_cfg(cfg)) return c;
   if (T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
   if (out_dtype != MOE_DTYPE_BF16 && out_dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
@@ -643,6 +660,7 @@ int moe_ep_dispatch(const moe_config *cfg, int32_t world, const uint8_t *xq, con
                     const float *gate, int64_t T, uint8_t *send_rows, int64_t send_cap_rows, int32_t *send_counts,
                     int32_t *send_offsets, int32_t *row_of, uint8_t *self_rows, void *ws, size_t ws_bytes,
                     int32_t *err_flag, void *stream) {
+  const NvtxRange nvtx_call("moe_ep_dispatch");
   if (const int c = check_cfg(cfg)) return c;
   if (world < 1 || world > 64 || cfg->n_routed % world) return MOE_ERR_INVALID_ARG;
   if (T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
@@ -674,6 +692,7 @@ size_t moe_ep_experts_workspace_size(const moe_config *cfg_local, int64_t n_rows
 
 int moe_ep_experts(const moe_config *cfg_local, const moe_weights *w_local, const uint8_t *rows, int64_t n_rows,
                    int64_t row_bytes, void *partial_out, void *ws, size_t ws_bytes, int32_t *err_flag, void *stream) {
+  const NvtxRange nvtx_call("moe_ep_experts");
   if (const int c = check_cfg_local(cfg_local)) return c;
   if (n_rows < 0 || n_rows > kMaxTokens) return MOE_ERR_INVALID_ARG;
   const int64_t H = cfg_local->hidden, Kr = cfg_local->top_k;
@@ -721,6 +740,7 @@ int moe_ep_experts(const moe_config *cfg_local, const moe_weights *w_local, cons
 
 int moe_ep_combine(const moe_config *cfg, int32_t world, const void *x, int64_t T, const int32_t *row_of,
                    const void *back, const void *y_shared, void *out, int32_t out_dtype, void *stream) {
+  const NvtxRange nvtx_call("moe_ep_combine");
   if (const int c = check_cfg(cfg)) return c;
   if (world < 1 || world > 64 || T < 0 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
   if (out_dtype != MOE_DTYPE_BF16 && out_dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
@@ -826,6 +846,7 @@ int moe_backward(const moe_config *cfg, const moe_weights *w, const uint8_t *w13
                  const uint8_t *w2t, const float *s2t, const void *x, const void *dout, int64_t T, float *dx,
                  float *dW13, float *dW2, const void *fwd_ws, size_t fwd_ws_bytes, void *ws, size_t ws_bytes,
                  int32_t *err_flag, void *stream) {
+  const NvtxRange nvtx_call("moe_backward");
   if (const int c = check_cfg(cfg)) return c;
   if (cfg->scale_mode != MOE_SCALE_AMAX) return MOE_ERR_NOT_IMPLEMENTED;
   if (T < 1 || T > kMaxTokens) return MOE_ERR_INVALID_ARG;
