@@ -241,3 +241,25 @@ def test_backward_entry_points_validate_on_the_host(m):
     assert L.moe_backward(C.byref(cfg), C.byref(w), *small) == m.MOE_ERR_WORKSPACE_TOO_SMALL
     assert L.moe_backward(C.byref(cfg), C.byref(w), *args) == m.MOE_ERR_NO_DEVICE
     assert L.moe_transpose_weights(C.byref(cfg), C.byref(w), 16, 16, 16, 16, None) == m.MOE_ERR_NO_DEVICE
+
+
+def test_profile_event_hook_validation(m):
+    """The measurement hook takes the forward's 7 event handles, or 7 + 9 to
+    also mark the backward's stages; a null handle among those it keeps is
+    rejected; a null array turns it off.  (Handles are only stored here: no
+    forward runs while the fake ones are set.)"""
+    import ctypes as C
+    L = m.lib
+    nf, nb = m.MOE_PROFILE_EVENTS, m.MOE_PROFILE_BWD_EVENTS
+    assert (nf, nb) == (7, 9)
+    try:
+        fake = (C.c_void_p * (nf + nb))(*range(1, nf + nb + 1))
+        assert L.moe_profile_events(fake, nf) == m.MOE_OK
+        assert L.moe_profile_events(fake, nf + nb) == m.MOE_OK
+        assert L.moe_profile_events(fake, nf - 1) == m.MOE_ERR_INVALID_ARG
+        holes = (C.c_void_p * (nf + nb))(*range(1, nf + nb + 1))
+        holes[nf + 3] = None  # a backward handle missing: rejected when all 16 are given
+        assert L.moe_profile_events(holes, nf + nb) == m.MOE_ERR_INVALID_ARG
+        assert L.moe_profile_events(holes, nf) == m.MOE_OK  # forward-only: the hole is not kept
+    finally:
+        assert L.moe_profile_events(None, 0) == m.MOE_OK

@@ -178,3 +178,31 @@ def test_backward_rejects_pow2_and_small_workspace(m):
         m.moe_backward(layer.cfg, layer.weights(), wt, x, x, layer.workspace(8),
                        ws=torch.empty(1024, dtype=torch.uint8, device="cuda"), err=layer.err)
     assert e.value.status == m.MOE_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_backward_profile_events(m):
+    """With 7 + 9 event handles the backward marks its stages on the stream:
+    every stage time is non-negative and they add up to the whole call."""
+    prob = Problem(S.TINY, 300, seed=9)
+    layer = build_gpu_layer(m, prob)
+    x = prob.x.cuda()
+    layer.forward(x)
+    dout = S.gen_x(300, S.TINY["H"], 1009).cuda()
+    layer.backward(x, dout)  # set-up (transposed weights) outside the measured call
+    nf, nb = m.MOE_PROFILE_EVENTS, m.MOE_PROFILE_BWD_EVENTS
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(nf + nb)]
+    for e in ev:
+        e.record()
+    torch.cuda.synchronize()
+    try:
+        m.moe_profile_events(ev)
+        layer.backward(x, dout)
+    finally:
+        m.moe_profile_events(None)
+    torch.cuda.synchronize()
+    layer.check()
+    stages = [ev[nf + i].elapsed_time(ev[nf + i + 1]) for i in range(nb - 1)]
+    assert len(stages) == len(m.PROFILE_BWD_STAGES)
+    assert all(t >= 0.0 for t in stages), stages
+    total = ev[nf].elapsed_time(ev[nf + nb - 1])
+    assert abs(sum(stages) - total) <= 1e-3 * max(total, 1e-3) + 1e-3
