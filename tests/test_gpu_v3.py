@@ -222,3 +222,56 @@ def test_v3_decode_layer_tall(tall, oracle_lib, v3_layer):
     layer, _ = v3_layer
     prob = _problem(dict(S.DECODE), 64, 15, layer, "zero")
     check_layer(m, oracle_lib, prob, layer, tokens=np.arange(64), check_weights=False)
+
+
+def test_v3_expert_parallel_emulated(m, oracle_lib, v3_layer):
+    """The expert-parallel forward of 8 ranks x 256 tokens on the V3 layer, all
+    ranks' kernels on this GPU (exchanges as device copies), against the
+    oracle's single-device layer on 8 sampled tokens per rank (off near-ties).
+    The reading (R-EP) returns each destination rank's partial sum and the
+    shared expert's output as bf16, so the max bound of an element also takes
+    half a bf16 ulp of each such term, from the oracle's own per-expert
+    outputs; the relative Frobenius bound is the stated one."""
+    from sparse_moe_layer_expert_b200.ep import LibraryOps, forward_local
+    from _moe_util import half_ulp_bf16, assert_close, oracle_cfg, NEAR_TIE
+    from test_gpu_layer import h_tie_allowance
+    dec = oracle_lib.e4m3_decode_table()
+    layer, _ = v3_layer
+    W, T = 8, 256
+    cfg = dict(S.PREFILL)
+    prob = _problem(cfg, T, 21, layer, "uniform")
+    layer.bias.copy_(prob.bias)
+    ops = [LibraryOps(layer, W, r) for r in range(W)]
+    xs = [S.gen_x(T, cfg["H"], 300 + r, device="cuda") for r in range(W)]
+    outs = forward_local(ops, xs, m.MOE_DTYPE_F32)
+    layer.check()
+    ocf = oracle_cfg(oracle_lib, cfg)
+    Nr, per = cfg["Nr"], cfg["Nr"] // W
+    experts = {}
+    rng = np.random.default_rng(21)
+    for r in range(W):
+        x = xs[r].cpu()
+        oi, og, gap, _ = oracle_lib.route(ocf, x, prob.wr, prob.bias)
+        toks = np.sort(rng.choice(np.nonzero(gap >= NEAR_TIE)[0], 8, replace=False))
+        for e in set(oi[toks].reshape(-1).tolist()) | {Nr}:
+            if e not in experts:
+                experts[e] = prob.oracle_expert(oracle_lib, e)
+        res = oracle_lib.forward(ocf, x, prob.wr, prob.bias, [experts.get(e) for e in range(Nr + 1)], tokens=toks)
+        assert np.array_equal(res["idx"], oi[toks])
+        xq, xsc = oracle_lib.quant_1x128(x[torch.as_tensor(toks)])
+        allow = np.zeros((len(toks), cfg["H"]))
+        for i, t in enumerate(toks):
+            # (and, as in every layer test, what codes of h at a rounding
+            # near-tie can move each expert's output by)
+            ysh, hsh, _, hssh = oracle_lib.expert_ffn(ocf, xq[i:i + 1], xsc[i:i + 1], *experts[Nr], want_h=True)
+            allow[i] += half_ulp_bf16(ysh[0]) + h_tie_allowance(dec, hsh[0], hssh[0], experts[Nr][2], experts[Nr][3])
+            part = {}
+            for k in range(cfg["Kr"]):
+                e = int(oi[t, k])
+                y, h, _, hs = oracle_lib.expert_ffn(ocf, xq[i:i + 1], xsc[i:i + 1], *experts[e], want_h=True)
+                part[e // per] = part.get(e // per, 0.0) + og[t, k] * y[0]
+                allow[i] += og[t, k] * h_tie_allowance(dec, h[0], hs[0], experts[e][2], experts[e][3])
+            for d in part:
+                allow[i] += half_ulp_bf16(part[d])
+        got = outs[r].cpu().numpy().astype(np.float64)[toks]
+        assert_close(got, res["out"], what=f"expert-parallel V3 output, rank {r} of {W}", tie_allow=allow)
