@@ -42,14 +42,16 @@
 // activation tile is loaded as four 32-row TMA boxes into those places (only
 // the boxes the chunk has rows in).
 //
-// FP32 outputs (EPI_GATE_F32, EPI_F32) leave through TMA stores: the
-// promotion threads put a 128 x 128 block into shared memory as boxes of 32
-// rows x 32 columns (128-byte swizzle) and one thread stores every box whose
-// 32 rows lie inside the tile; the rows of a tile's last, partial quarter
-// (rows beyond belong to the next chunk) are stored by their threads.  The
-// stores drain while the next tile's K blocks run (a down-projection tile has
-// only I/128 K blocks for 128 x 256 FP32 outputs).  Those two epilogues run
-// with three operand stages, which leaves room for one staged block.
+// FP32 outputs (EPI_GATE_F32, EPI_F32) leave through TMA stores, warp by
+// warp: each promotion warp puts its 32 rows x 64 columns of a 128 x 128
+// block into its own 8 KB of shared memory as two boxes of 32 rows x 32
+// columns (128-byte swizzle) and its lane 0 stores them; the rows of a
+// tile's last, partial quarter (rows beyond belong to the next chunk) are
+// stored by their threads.  No barrier joins the warps at the end of a tile,
+// so one warp's epilogue does not hold up the others, and the stores drain
+// while the next tile's K blocks run (a down-projection tile has only I/128
+// K blocks for 128 x 256 FP32 outputs).  Those two epilogues run with three
+// operand stages, which leaves room for the 64 KB of staging.
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warp 2 scale producer, warp 3 idle, warps 4..11 promotion +
@@ -101,46 +103,58 @@ struct GLayout {
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
-// Store one 128 x 128 FP32 block of a tile (this thread: row r = 32 q +
-// lane, columns 64 wg .. +63 of the block in acc, times gate) at output
-// (row0, col0): the thread writes its two 32-column boxes of quarter q, each
-// row's 128 bytes as 16-byte chunks at j ^ (lane & 7) (the tensor map's
-// 128-byte swizzle); one thread stores the boxes of the quarters whose 32
-// rows are all inside the tile's n rows; the threads of a partial quarter
-// store their own rows (row < n) directly.  The issuing thread first waits
-// until its previous stores have read the staging block; the 256 promotion
-// threads meet at named barrier 2.
-__device__ __forceinline__ void store_rows_block(const float (&acc)[64], float gate, uint8_t *ostage,
-                                                 const CUtensorMap *map, float *out, int64_t ldo, int64_t row0,
-                                                 int col0, int n, int wg, int q, int lane, bool issuer) {  // q: row quarter
-  if (issuer) bulk_wait_read();
-  named_bar_sync(2, 256);
-  const bool full_q = 32 * q + 32 <= n;
-  if (full_q) {
+// This warp's 32 rows x 64 columns of a 128 x 128 FP32 block, times gate,
+// into its 8 KB of staging as two boxes of 32 rows x 32 columns, each row's
+// 128 bytes as 16-byte chunks at j ^ (lane & 7) (the tensor map's 128-byte
+// swizzle).  Lane 0 first waits until its previous stores have read the area.
+__device__ __forceinline__ void stage_rows_warp(const float (&acc)[64], float gate, uint8_t *wstage, int lane) {
+  if (lane == 0) bulk_wait_read();
+  __syncwarp();
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      uint8_t *box = ostage + (q * 4 + wg * 2 + b) * G_OBOX + lane * 128;
+  for (int b = 0; b < 2; ++b) {
+    uint8_t *box = wstage + b * G_OBOX + lane * 128;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = b * 32 + j * 4;
-        *reinterpret_cast<float4 *>(box + ((j ^ (lane & 7)) << 4)) =
-            make_float4(acc[c] * gate, acc[c + 1] * gate, acc[c + 2] * gate, acc[c + 3] * gate);
-      }
+    for (int j = 0; j < 8; ++j) {
+      const int c = b * 32 + j * 4;
+      *reinterpret_cast<float4 *>(box + ((j ^ (lane & 7)) << 4)) =
+          make_float4(acc[c] * gate, acc[c + 1] * gate, acc[c + 2] * gate, acc[c + 3] * gate);
     }
-  } else if (32 * q + lane < n) {
-    float4 *dst = reinterpret_cast<float4 *>(out + (row0 + 32 * q + lane) * ldo + col0 + wg * 64);
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      dst[j] = make_float4(acc[4 * j] * gate, acc[4 * j + 1] * gate, acc[4 * j + 2] * gate, acc[4 * j + 3] * gate);
   }
-  fence_proxy_async_smem();
-  named_bar_sync(2, 256);
-  if (issuer) {
-    for (int qq = 0; qq < 4 && 32 * qq + 32 <= n; ++qq)
-#pragma unroll
-      for (int cb = 0; cb < 4; ++cb)
-        tma_store_2d(map, ostage + (qq * 4 + cb) * G_OBOX, col0 + 32 * cb, static_cast<int32_t>(row0 + 32 * qq));
-    bulk_commit();
+}
+
+// Store this warp's part of one 128 x 128 FP32 block of a tile: rows
+// 32 q .. 32 q + 31 (this thread: row 32 q + lane) and columns 64 wg .. +63
+// of the block, at output (row0, col0).  A warp whose 32 rows all lie inside
+// the tile's n rows stages them and its lane 0 stores the two boxes with TMA.
+// A warp of the tile's last, partial quarter (rows beyond n belong to the
+// next chunk) stages them too and then writes each of its m rows with one
+// warp-wide access (8 bytes per lane, the row's 256 bytes contiguous).  No
+// thread waits for another warp: the eight promotion warps leave a tile
+// independently.
+__device__ __forceinline__ void store_rows_warp(const float (&acc)[64], float gate, uint8_t *wstage,
+                                                const CUtensorMap *map, float *out, int64_t ldo, int64_t row0,
+                                                int col0, int n, int wg, int q, int lane) {  // q: row quarter
+  const int m = n - 32 * q;  // rows of this quarter inside the tile
+  if (m <= 0) return;
+  stage_rows_warp(acc, gate, wstage, lane);
+  if (m >= 32) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int32_t y0 = static_cast<int32_t>(row0 + 32 * q);
+      tma_store_2d(map, wstage, col0 + 64 * wg, y0);
+      tma_store_2d(map, wstage + G_OBOX, col0 + 64 * wg + 32, y0);
+      bulk_commit();
+    }
+  } else {
+    __syncwarp();
+    // lane l holds columns 2l, 2l + 1: box l / 16, chunk (l % 16) / 2, half l % 2
+    const uint8_t *src = wstage + (lane >> 4) * G_OBOX + (lane & 1) * 8;
+    const int ch = (lane & 15) >> 1;
+    float *dst = out + (row0 + 32 * q) * ldo + col0 + wg * 64 + 2 * lane;
+    for (int i = 0; i < m; ++i)
+      *reinterpret_cast<float2 *>(dst + i * ldo) =
+          *reinterpret_cast<const float2 *>(src + i * 128 + ((ch ^ (i & 7)) << 4));
   }
 }
 
@@ -376,7 +390,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     float *amx = amax_x;             // [2 warpgroups][128 rows]
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-      if (named_bar_or(1, 256, *abortp != 0)) break;
+      // the SwiGLU epilogue exchanges amax between the warpgroups, so they
+      // stop together; the FP32 epilogues have no cross-warp step
+      if (L::kTma ? (*abortp != 0) : named_bar_or(1, 256, *abortp != 0)) break;
       const GemmTile td = get_tile(args, tile);
       if (!tile_ok(args, td)) continue;
       const bool two = td.w_row1 >= 0;
@@ -384,6 +400,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       // a warp whose 32 rows are all padding (short chunks) skips its TMEM
       // reads and FMAs; it still takes every wait and arrival of the ring
       const bool live = rq * 32 < td.n;
+      // the row's gate (down projection), loaded before the K loop so its
+      // latency is not part of the epilogue
+      const float gt = (EPI == EPI_GATE_F32 && r < td.n) ? __ldg(args.row_gate + td.out_row + r) : 1.0f;
       float acc0[64], acc1[64];
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
@@ -427,19 +446,18 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         // FP32 rows through TMA stores: block A at out_col + 64 wg, block B
         // at +128 (down projection) or +half (a gate/up pair)
         const int64_t cB = args.gate_up ? args.half : 128;
-        const float gt = (EPI == EPI_GATE_F32 && r < td.n) ? __ldg(args.row_gate + td.out_row + r) : 1.0f;
         float *outp = static_cast<float *>(args.out);
-        store_rows_block(acc0, gt, ostage, &map_out, outp, args.ldo, td.out_row, td.out_col, td.n, wg, rq, lane,
-                         warp == 4 && lane == 0);
+        uint8_t *wstage = ostage + (warp - 4) * 2 * G_OBOX;  // this warp's two boxes
+        store_rows_warp(acc0, gt, wstage, &map_out, outp, args.ldo, td.out_row, td.out_col, td.n, wg, rq, lane);
         if (two)
-          store_rows_block(acc1, gt, ostage, &map_out, outp, args.ldo, td.out_row, static_cast<int>(td.out_col + cB),
-                           td.n, wg, rq, lane, warp == 4 && lane == 0);
+          store_rows_warp(acc1, gt, wstage, &map_out, outp, args.ldo, td.out_row, static_cast<int>(td.out_col + cB),
+                          td.n, wg, rq, lane);
       } else {
         tile_epilogue<EPI, false>(args, td, acc0, acc1, two, warp, lane, amx, outx, rq);
       }
     }
-    // the staged block stays valid until the last stores have read it
-    if (L::kTma && warp == 4 && lane == 0) bulk_wait_all();
+    // the staging area stays valid until each warp's last stores have read it
+    if (L::kTma && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
