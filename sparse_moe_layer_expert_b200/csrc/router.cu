@@ -419,8 +419,10 @@ int router_ksplit(int64_t T, int Nr, int H) {
   const int64_t base = ((T + 127) / 128) * ((Nr + 127) / 128);
   const int kb_total = H / 64;
   if (base <= 0) return 1;
+  // as many K splits as fit the SMs in one wave: a second, partial wave
+  // would add a whole split's time for a few CTAs
   const int64_t sms = moe_host::sm_count();
-  int64_t ks = (sms + base - 1) / base;
+  int64_t ks = sms / base;
   if (ks > 16) ks = 16;
   if (ks > kb_total) ks = kb_total;
   if (ks < 1) ks = 1;
