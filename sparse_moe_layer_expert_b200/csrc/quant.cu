@@ -45,31 +45,46 @@ __device__ __forceinline__ uint2 codes8(const float (&f)[8], float S) {
   return make_uint2(lo, hi);
 }
 
-// 1x128 tiles: 16 lanes per tile, 8 bf16 (one 16-byte load) per lane.
+// 1x128 tiles: 16 lanes per tile, 8 bf16 (one 16-byte load) per lane; each
+// 16-lane set takes 2 consecutive tiles, all loads issued first.
 template <bool POW2>
 __global__ void __launch_bounds__(256) quant_1x128_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
                                                            int64_t cols, int64_t ldx, uint8_t *__restrict__ q,
                                                            float *__restrict__ s) {
-  const int64_t groups_per_row = cols / 128;
-  const int64_t total = rows * groups_per_row;
-  const int64_t gid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+  constexpr int G = 2;
+  const int64_t gpr = cols / 128;
+  const int64_t total = rows * gpr;
+  const int64_t gid0 = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4) * G;
   const int sub = threadIdx.x & 15;
-  const bool valid = gid < total;
-  const int64_t r = valid ? gid / groups_per_row : 0;
-  const int64_t g = valid ? gid - r * groups_per_row : 0;
-  uint4 v = make_uint4(0, 0, 0, 0);
-  if (valid) v = __ldg(reinterpret_cast<const uint4 *>(x + r * ldx + g * 128 + sub * 8));
-  float f[8];
-  bf16x8_to_f32(v, f);
-  float amax = 0.0f;
+  int64_t r = gid0 / gpr;
+  int64_t g = gid0 - r * gpr;
+  int64_t rr[G], gg[G];
+  uint4 v[G];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  for (int k = 0; k < G; ++k) {
+    rr[k] = r;
+    gg[k] = g;
+    v[k] = make_uint4(0, 0, 0, 0);
+    if (gid0 + k < total) v[k] = __ldg(reinterpret_cast<const uint4 *>(x + r * ldx + g * 128 + sub * 8));
+    if (++g == gpr) {
+      g = 0;
+      ++r;
+    }
+  }
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float S = POW2 ? pow2_scale(amax) : amax / 448.0f;
-  if (valid) {
-    *reinterpret_cast<uint2 *>(q + r * cols + g * 128 + sub * 8) = codes8(f, S);
-    if (sub == 0) s[r * groups_per_row + g] = S;
+  for (int k = 0; k < G; ++k) {
+    float f[8];
+    bf16x8_to_f32(v[k], f);
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float S = POW2 ? pow2_scale(amax) : amax / 448.0f;
+    if (gid0 + k < total) {
+      *reinterpret_cast<uint2 *>(q + rr[k] * cols + gg[k] * 128 + sub * 8) = codes8(f, S);
+      if (sub == 0) s[rr[k] * gpr + gg[k]] = S;
+    }
   }
 }
 
@@ -114,7 +129,7 @@ cudaError_t launch_quant_1x128(const void *x, int64_t rows, int64_t cols, int64_
                                cudaStream_t st, bool pow2) {
   const int64_t groups = rows * (cols / 128);
   if (groups == 0) return cudaSuccess;
-  const int64_t threads = groups * 16;
+  const int64_t threads = (groups + 1) / 2 * 16;  // 16 lanes per pair of tiles
   const int64_t blocks = (threads + 255) / 256;
   const auto *xb = static_cast<const __nv_bfloat16 *>(x);
   if (pow2)
