@@ -16,8 +16,10 @@
 //  rank_kernel         per 128-token block: stable ranks (warp matches over
 //                      8 ranges of the block) -> row of every (token, slot),
 //                      per-row gate and source
-//  copy_rows_kernel    one warp per row: FP8 row copy (16-byte vectors) and
-//                      the row's scales into the transposed scale table
+//  copy_rows_kernel    one warp per row: FP8 row copy (16-byte vectors, eight
+//                      loads in flight per lane) and, per CTA of 8 rows, the
+//                      rows' scales into the transposed scale table as 8
+//                      consecutive floats per K block
 #include "common.cuh"
 #include "kernels.h"
 
@@ -203,22 +205,54 @@ __global__ void __launch_bounds__(256) copy_rows_kernel(const uint8_t *__restric
                                                          const int32_t *__restrict__ row_src, int64_t R, int64_t T,
                                                          int Ns, int H, uint8_t *__restrict__ ap,
                                                          float *__restrict__ as_t, int64_t ld) {
-  const int lane = threadIdx.x & 31;
-  const int64_t p = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  constexpr int U = 8;        // 16-byte loads in flight per lane
+  constexpr int KC = 32;      // K blocks of scales staged per pass
+  __shared__ float sc[8][KC + 1];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * 8;
+  const int64_t p = p0 + w;
   const int64_t rows = R + (Ns ? T : 0);
-  if (p >= rows) return;
   const int hv = H / 16, kb = H / 128;
-  int64_t t;
-  if (p < R) {
-    t = row_src[p];
-    if (t < 0 || t >= T) return;
-    const uint4 *src = reinterpret_cast<const uint4 *>(xq + t * xq_ld);
-    uint4 *dst = reinterpret_cast<uint4 *>(ap + p * H);
-    for (int i = lane; i < hv; i += 32) dst[i] = __ldg(src + i);
-  } else {
-    t = p - R;
+  int64_t t = -1;
+  if (p < rows) {
+    if (p < R) {
+      t = row_src[p];
+      if (t < 0 || t >= T) t = -1;
+    } else {
+      t = p - R;
+    }
   }
-  for (int i = lane; i < kb; i += 32) as_t[i * ld + p] = __ldg(xs + t * kb + i);
+  if (t >= 0 && p < R) {
+    const uint4 *s = reinterpret_cast<const uint4 *>(xq + t * xq_ld);
+    uint4 *d = reinterpret_cast<uint4 *>(ap + p * H);
+    for (int base = 0; base < hv; base += 32 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * 32 + lane;
+        if (i < hv) v[u] = __ldg(s + i);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * 32 + lane;
+        if (i < hv) d[i] = v[u];
+      }
+    }
+  }
+  // scales: the block's 8 rows go to as_t[k * ld + p0 .. p0 + 7], written
+  // as 8 consecutive floats per K block
+  for (int k0 = 0; k0 < kb; k0 += KC) {
+    const int nk = kb - k0 < KC ? kb - k0 : KC;
+    if (lane < nk) sc[w][lane] = t >= 0 ? __ldg(xs + t * kb + k0 + lane) : 0.0f;
+    __syncthreads();
+    const int j = threadIdx.x & 7, k = threadIdx.x >> 3;
+    const int64_t pj = p0 + j;
+    if (k < nk && pj < rows) {
+      const bool live = pj >= R || (row_src[pj] >= 0 && row_src[pj] < T);
+      if (live) as_t[static_cast<int64_t>(k0 + k) * ld + pj] = sc[j][k];
+    }
+    __syncthreads();
+  }
 }
 
 cudaError_t launch_hist(const int32_t *idx, int64_t T, int Kr, int Nr, int allow_empty, int32_t *blk_hist,
