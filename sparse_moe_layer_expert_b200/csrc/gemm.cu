@@ -39,8 +39,8 @@
 // slows; so the tile's last 32 rows (often padding in a short chunk, whose
 // warps then skip their reads) go to lanes 32..63: tile rows 0-31 / 32-63 /
 // 64-95 / 96-127 sit in lanes 0-31 / 64-95 / 96-127 / 32-63.  The
-// activation tile is loaded as four 32-row TMA boxes into those places (only
-// the boxes the chunk has rows in).
+// activation tile is loaded as four 32-row TMA boxes into those places (the
+// boxes the chunk has no rows in from past the tensor's last row: zeros).
 //
 // FP32 outputs (EPI_GATE_F32, EPI_F32) leave through TMA stores, warp by
 // warp: each promotion warp puts its 32 rows x 64 columns of a 128 x 128
@@ -253,7 +253,12 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           const CUtensorMap *amap = td.from1 ? &map_a1 : &map_a0;
           const bool two = td.w_row1 >= 0;
           const int nbox = (td.n + 31) / 32;  // activation boxes holding the chunk's rows (1..4)
-          const uint32_t bytes = nbox * G_ABOX + (two ? 2 : 1) * G_WB;
+          const uint32_t bytes = 4 * G_ABOX + (two ? 2 : 1) * G_WB;
+          // the quarters without rows get a box from past the map's last row,
+          // which TMA fills with zeros: the MMA then multiplies zeros there
+          // instead of a stale stage's codes (the same result for the rows
+          // that are kept, at a lower tensor-core power under the power cap)
+          const int zrow = static_cast<int>(td.from1 ? args.a_rows1 : args.a_rows0);
           const uint64_t pol_w = td.group > 1 ? pol_wk : pol_w1;
           for (int kb = 0; kb < KB; ++kb, ++it) {
             const int s = it % NST;
@@ -264,8 +269,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             uint8_t *st = stages + s * G_STAGE;
             mbar_arrive_expect_tx(&bars->full[s], bytes);
             const int x = kb * 128;
-            for (int b = 0; b < nbox; ++b)
-              tma_load_2d_hint(st + lane_q_of_rows(b) * G_ABOX, amap, &bars->full[s], x, td.a_row + 32 * b, pol_a);
+            for (int b = 0; b < 4; ++b)
+              tma_load_2d_hint(st + lane_q_of_rows(b) * G_ABOX, amap, &bars->full[s], x,
+                               b < nbox ? td.a_row + 32 * b : zrow, pol_a);
             tma_load_2d_hint(st + G_AB, &map_w, &bars->full[s], x, td.w_row0, pol_w);
             if (two) tma_load_2d_hint(st + G_AB + G_WB, &map_w, &bars->full[s], x, td.w_row1, pol_w);
           }
