@@ -213,7 +213,8 @@ MOE_API int moe_route(const moe_config *cfg, const void *x_dev, const void *wr_d
  * library, held until the process exits) and allocates nothing.
  *   - Limit: the partials moe_route would keep in its workspace must fit,
  *     i.e. moe_route_workspace_size(cfg, T) - 256 <= 16 MiB (for
- *     n_routed = 256 every T <= 8192 fits); larger calls return
+ *     n_routed = 256 on a 148-SM device every T <= 16384 fits); larger
+ *     calls return
  *     MOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
  *   - Every call looks up the scratch's device address in the current
  *     device's context (cudaGetSymbolAddress, which allocates nothing), so
