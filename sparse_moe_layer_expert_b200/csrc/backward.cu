@@ -303,8 +303,22 @@ __global__ void __launch_bounds__(256) colquant_kernel(const int4 *__restrict__ 
   {
     const float S = fmaxf(fmaxf(part[0][c], part[1][c]), fmaxf(part[2][c], part[3][c])) / 448.0f;
     const float y = S != 0.0f ? __frcp_rn(S) : 0.0f;
-    for (int r = quarter * 32; r < quarter * 32 + 32; ++r)
-      codes[c][r] = S != 0.0f ? e4m3_rn_sat(quot(vals[r][c], S, y)) : static_cast<uint8_t>(0);
+    // 32 codes of this channel as two 16-byte words, converted in pairs
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r0 = quarter * 32 + 16 * h;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (S != 0.0f) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r = r0 + 4 * k;
+          const uint32_t lo = e4m3x2_rn_sat(quot(vals[r][c], S, y), quot(vals[r + 1][c], S, y));
+          const uint32_t hi = e4m3x2_rn_sat(quot(vals[r + 2][c], S, y), quot(vals[r + 3][c], S, y));
+          w[k] = lo | (hi << 16);
+        }
+      }
+      *reinterpret_cast<uint4 *>(&codes[c][r0]) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
     if (quarter == 0) s_t[static_cast<int64_t>(col0 / 128) * C + c0 + c] = S;
   }
   __syncthreads();
