@@ -147,7 +147,8 @@ def check_layer(m, oracle_lib, prob: Problem, layer, tokens=None, oracle_experts
     o16 = out16.cpu()[torch.as_tensor(tok)]
     assert_close(bf16_to_f64(o16), res["out"], bf16_out=True, what="layer output (bf16)", tie_allow=out_tie)
     assert torch.equal(o16, out32.cpu()[torch.as_tensor(tok)].to(torch.bfloat16))
-    return dict(counts=counts, idx=idx, n_exempt=n_exempt, n_stated_near_tie=n_stated, idx_ref=oi, s_ref=s_o)
+    return dict(counts=counts, idx=idx, n_exempt=n_exempt, n_stated_near_tie=n_stated, idx_ref=oi, s_ref=s_o,
+                out=out32.cpu().numpy())
 
 
 def h_tie_allowance(dec, h_o, hs_o, W2q, s2, mode=0):
@@ -216,7 +217,8 @@ def check_requantized(oracle_lib, hq, hs, hq_o, hs_o, h_o, mode=0):
     if mode == 1:
         amax_o = np.abs(h_o.astype(np.float64)).reshape(hs_o.shape[0], hs_o.shape[1], 128).max(axis=2)
         t = np.log2(np.where(amax_o > 0, amax_o, 448.0) / 448.0)
-        near = np.abs(t - np.round(t)) * np.log(2) < 1e-5
+        # an all-zero tile (amax 0) has S = 0 on both sides: no threshold
+        near = (amax_o > 0) & (np.abs(t - np.round(t)) * np.log(2) < 1e-5)
         assert near.mean() < 1e-3, f"{near.mean():.2e} of the tiles sit at a scale threshold"
         assert np.array_equal(hs[~near], hs_o[~near]), "power-of-two re-quantization scales"
         keep = np.repeat(~near, 128, axis=1)
@@ -298,6 +300,26 @@ def test_layer_every_token_picks_the_same_experts(m, oracle_lib):
     assert (c[:kr] == 700).all() and (c[kr:] == 0).all()
 
 
+def _degenerate_tokens(prob):
+    """Tokens 0..31 all zero (every 1x128 tile has amax 0: S = 0, every code
+    0; every affinity is sigmoid(0) = 1/2, so the bias alone selects; h = 0
+    takes the zero-scale path of the requantization), 32..63 scaled by 2^-10
+    and the rest by 2^8 (affinities near 0 and 1, scales far from 1); powers
+    of two keep the bf16 values exact."""
+    x = prob.x.clone()
+    x[:32] = 0
+    x[32:64] = (x[32:64].float() * 2.0 ** -10).to(torch.bfloat16)
+    x[64:] = (x[64:].float() * 2.0 ** 8).to(torch.bfloat16)
+    prob.x = x
+    return prob
+
+
+def test_layer_zero_tiny_and_large_tokens(m, oracle_lib):
+    prob = _degenerate_tokens(Problem(S.TINY, 96, seed=12))
+    r = check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob))
+    assert np.all(r["out"][:32] == 0.0), "an all-zero token's layer output is zero"
+
+
 def test_layer_empty_batch(m, oracle_lib):
     # T = 0: nothing to compute; the loads are all zero and the bias update
     # of an empty step leaves every bias unchanged (load == mean == 0)
@@ -346,6 +368,11 @@ def test_layer_pow2_wider_hidden_and_many_chunks(m, oracle_lib):
 def test_layer_pow2_group_limited_skewed(m, oracle_lib):
     prob = Problem(dict(S.TINY, n_groups=4, topk_groups=2, **POW2), 512, seed=25, x_kind="mixture")
     check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob), tokens=np.arange(0, 512, 7))
+
+
+def test_layer_pow2_zero_tiny_and_large_tokens(m, oracle_lib):
+    prob = _degenerate_tokens(Problem(dict(S.TINY, **POW2), 96, seed=12))
+    check_layer(m, oracle_lib, prob, build_gpu_layer(m, prob))
 
 
 def test_forward_rejects_unknown_scale_mode(m):
