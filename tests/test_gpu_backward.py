@@ -66,7 +66,7 @@ def expert_tie_allowance(oracle_lib, OB, dec, r, x_rows, d_rows, W13q, s13):
     return dx_a, dW13_a, dW2_a
 
 
-def run_backward_case(m, oracle_lib, cfg, T, seed, bias_shift=None):
+def run_backward_case(m, oracle_lib, cfg, T, seed, bias_shift=None, zero_dout=0):
     import oracle.backward as OB
     prob = Problem(cfg, T, seed=seed)
     if bias_shift is not None:
@@ -77,6 +77,8 @@ def run_backward_case(m, oracle_lib, cfg, T, seed, bias_shift=None):
     idx_out = torch.empty((T, cfg["Kr"]), dtype=torch.int32, device="cuda")
     layer.forward(x, idx_out=idx_out)
     dout = S.gen_x(T, cfg["H"], seed + 1000)
+    if zero_dout:
+        dout[:zero_dout] = 0
     dx, dW13, dW2 = layer.backward(x, dout.cuda())
     layer.check()
     experts = [prob.oracle_expert(oracle_lib, e) for e in range(prob.E)]
@@ -137,6 +139,8 @@ def run_backward_case(m, oracle_lib, cfg, T, seed, bias_shift=None):
                          tie_allow=w_allow[e][1])
         else:
             assert not dW13_h[e].any() and not dW2_h[e].any(), f"expert {e} has no token but a gradient"
+    if zero_dout:
+        assert not dx.cpu()[:zero_dout].any(), "a token with zero dout has a nonzero dx"
     return ref
 
 
@@ -149,6 +153,14 @@ def test_backward_tiny_multi_tile_experts(m, oracle_lib):
     # 128-token tiles of the weight gradients (the last one 44 rows)
     ref = run_backward_case(m, oracle_lib, dict(S.TINY), 300, 3, bias_shift=S.TINY["Kr"])
     assert set(ref["dW13"].keys()) == set(range(S.TINY["Kr"])) | {S.TINY["Nr"]}
+
+
+def test_backward_zero_dout_tokens(m, oracle_lib):
+    # every token picks experts 0..K_r-1 and the first 128 tokens carry a zero
+    # dout: their dh, dG, dU and dx are exactly zero, and the first 128-token
+    # tile of each expert's dG|dU operand is all zero (the 128x1 quantizer's
+    # zero-scale path)
+    run_backward_case(m, oracle_lib, dict(S.TINY), 300, 5, bias_shift=S.TINY["Kr"], zero_dout=128)
 
 
 def test_backward_tiny_ragged_no_shared(m, oracle_lib):
