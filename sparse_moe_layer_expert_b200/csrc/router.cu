@@ -224,13 +224,15 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float *__restric
   if (n_groups > 0) {
     // group g = experts [g*gs, (g+1)*gs); score = sum of its two largest c
     const int gs = Nr / n_groups;
+    int grp[EPL];  // the group of each of this lane's experts, divided once
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) grp[i] = (lane + 32 * i) / gs;
     float my_score = -INFINITY;  // lane g holds the score of group g
     for (int g = 0; g < n_groups; ++g) {
       float b1 = -INFINITY, b2 = -INFINITY;
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        if (ok[i] && e / gs == g) {
+        if (ok[i] && grp[i] == g) {
           if (c[i] > b1) {
             b2 = b1;
             b1 = c[i];
@@ -261,10 +263,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float *__restric
       keep |= 1u << gi;
     }
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      if (ok[i] && !((keep >> (e / gs)) & 1u)) ok[i] = false;
-    }
+    for (int i = 0; i < EPL; ++i)
+      if (ok[i] && !((keep >> grp[i]) & 1u)) ok[i] = false;
   }
   int sel_e = -1;   // lane r keeps the r-th choice
   float sel_s = 0.0f;
