@@ -228,7 +228,34 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float *__restric
 #pragma unroll
     for (int i = 0; i < EPL; ++i) grp[i] = (lane + 32 * i) / gs;
     float my_score = -INFINITY;  // lane g holds the score of group g
-    for (int g = 0; g < n_groups; ++g) {
+    if (gs == 32) {
+      // lane l's expert i is expert 32 i + l, in group i: the top two of each
+      // group over the lanes, all groups' butterflies side by side
+      float b1[EPL], b2[EPL];
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        b1[i] = ok[i] ? c[i] : -INFINITY;
+        b2[i] = -INFINITY;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const float o1 = __shfl_xor_sync(0xffffffffu, b1[i], o);
+          const float o2 = __shfl_xor_sync(0xffffffffu, b2[i], o);
+          if (b1[i] >= o1) {
+            b2[i] = fmaxf(b2[i], o1);
+          } else {
+            b2[i] = fmaxf(o2, b1[i]);
+            b1[i] = o1;
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (lane == i && i < n_groups) my_score = b1[i] + b2[i];
+    }
+    for (int g = 0; g < n_groups && gs != 32; ++g) {
       float b1 = -INFINITY, b2 = -INFINITY;
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
