@@ -1,8 +1,9 @@
 """Benchmark of the FP8 DeepSeekMoE layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed]
-                    [--scale-mode amax|pow2] [--balance-steps S] [--impl ours|reference]
-                    [--no-cpu-baseline] [--no-e2e] [--e2e-serial]
+                    [--scale-mode amax|pow2] [--gemm auto|single|pair|tall] [--balance-steps S]
+                    [--impl ours|reference] [--no-cpu-baseline] [--no-e2e] [--e2e-serial]
+                    [--no-extras] [--tokens T] [--experts E]
 
 One step = the whole path over T tokens of seeded synthetic input with V3
 shapes (hidden 7168, intermediate 2048, 256 routed + 1 shared experts,
@@ -23,10 +24,18 @@ every step copies its input in from pinned host memory and reads its output
 back, on two copy streams that overlap the neighbouring steps' compute
 (--e2e-serial: copies in series on the launching stream).
 
+Unless --no-extras, the same process then measures, on the same resident
+weights, the other configurations under "workloads": the decode-shaped and
+the skewed layers, the standalone block-scaled GEMM at both shapes, the
+device's FP8 tensor ceiling, the backward of the expert FFNs on the headline
+batch and expert parallelism over 8 ranks emulated on the one GPU.
+
 --scale-mode pow2 runs the power-of-two scale variant (scales applied by the
-tensor core); the default is the pages' S = amax/448.  `--impl reference`
-times the CPU oracle (the slow double-precision reference of the same layer)
-on the host cores, on a bounded sample of the workload.
+tensor core); the default is the pages' S = amax/448.  --gemm picks the
+grouped-GEMM kernel (single CTAs by default).  --tokens / --experts shrink
+the workload for profiling.  `--impl reference` times the CPU oracle (the
+slow double-precision reference of the same layer) on the host cores, on a
+bounded sample of the workload.
 """
 from __future__ import annotations
 
