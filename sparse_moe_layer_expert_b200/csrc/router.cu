@@ -187,16 +187,23 @@ __device__ __forceinline__ float affinity(const float *__restrict__ partial, int
   return 1.0f / (1.0f + expf(-z));
 }
 
+// Unsigned key with the order of the floats (-0 taken as +0), and back.
+__device__ __forceinline__ uint32_t ord_key(float v) {
+  const uint32_t u = __float_as_uint(v + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord_val(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Largest v over the warp, ties to the smallest index i: two warp-wide
+// reductions (the largest key, then the smallest index holding it).
 __device__ __forceinline__ void warp_argmax(float &v, int &i) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
-    if (ov > v || (ov == v && oi < i)) {
-      v = ov;
-      i = oi;
-    }
-  }
+  const uint32_t k = ord_key(v);
+  const uint32_t best = __reduce_max_sync(0xffffffffu, k);
+  const uint32_t bi = __reduce_min_sync(0xffffffffu, k == best ? static_cast<uint32_t>(i) : 0xffffffffu);
+  v = ord_val(best);
+  i = static_cast<int>(bi);
 }
 }  // namespace
 
